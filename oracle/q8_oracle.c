@@ -1,0 +1,408 @@
+/*
+ * q8_oracle.c -- plain, slow CPU oracle for the int8 quantized linear.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA library; it is written from the
+ * definitions on the source pages:
+ *
+ *   [SmolVLM-Q8]  export/_smolvlm_q8.py (SmolVLM-500M-Instruct ExecuTorch WebGPU recipe)
+ *   [ROCm-INT8]   code/quant/int8_linear.py (Ming-Image-0.1-Design ROCm INT8)
+ *   [tiny-llm]    src/tinyllm/quant.py (tiny-llm, "INT8 weight-only quantization")
+ *   [ET-21229]    pytorch/executorch PR #21229, "Add linear_dq8ca_q4gsw +
+ *                 choose_qparams_affine (8da4w)"
+ *
+ * Conventions
+ *   - fp32 steps that decide an integer code are done in fp32 exactly as the
+ *     pages' torch code does them: one IEEE operation at a time, no fused
+ *     multiply-add (build with -ffp-contract=off, no fast-math), rounding with
+ *     nearbyintf() in the default round-to-nearest-even mode (torch.round).
+ *   - dot products are accumulated sequentially in k, in fp64 (float inputs)
+ *     or int64 (integer inputs); results are returned in fp64 so that the
+ *     caller can round them once to the output type.
+ *   - parallelism (OpenMP) is over output rows only; every sum runs in one
+ *     thread in a fixed order, so results do not depend on the thread count.
+ *
+ * Parity pins: every function here is checked by the CPU test suite against
+ * hand-worked values, closed forms and brute force (see tests/test_oracle_*.py).
+ */
+#include <math.h>
+#include <float.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#include "q8_oracle.h"
+
+/* ------------------------------------------------------------------ helpers */
+
+/* bf16 bits -> fp32 value (exact: bf16 is the top half of an fp32). */
+static float bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static float clampf(float v, float lo, float hi) {
+    if (v < lo) return lo;
+    if (v > hi) return hi;
+    return v;
+}
+
+int q8o_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void q8o_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* --------------------------------------------------- weight quantization (a1)
+ * [ROCm-INT8] quantize_weight and QUANT_RULE: per output channel (row n),
+ * scale = absmax(row) / 127 in fp32; q = clamp(round(w / scale), -127, 127);
+ * a row whose scale comes out 0 gets scale 1.0 and all codes 0.
+ * [tiny-llm] module docstring: same grid (s_j = max|W_j| / 127, clip to +-127).
+ * wsum[n] = sum_k q[n,k] is the per-row code sum that [SmolVLM-Q8]'s delegated
+ * op linear_q8ta_q8csw takes as its weight_sums operand (fix_q8ta_fake).
+ * Returns 0, or 1 if a code sum does not fit int32.
+ */
+int q8o_quantize_weight(const float* W, int64_t N, int64_t K,
+                        int8_t* q, float* s, int32_t* wsum) {
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(|:bad)
+    for (int64_t n = 0; n < N; ++n) {
+        const float* w = W + n * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(w[k]);
+            if (a > amax) amax = a;
+        }
+        float scale = amax / 127.0f;          /* fp32 IEEE division */
+        int zero = (scale == 0.0f);
+        if (zero) scale = 1.0f;
+        int64_t sum = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            int code = 0;
+            if (!zero) {
+                float r = nearbyintf(w[k] / scale);   /* true division, ties to even */
+                r = clampf(r, -127.0f, 127.0f);
+                code = (int)r;
+            }
+            q[n * K + k] = (int8_t)code;
+            sum += code;
+        }
+        s[n] = scale;
+        if (wsum) {
+            if (sum > INT32_MAX || sum < INT32_MIN) bad = 1;
+            wsum[n] = (int32_t)sum;
+        }
+    }
+    return bad;
+}
+
+/* ------------------------------------------ affine activation qparams (a2, R5)
+ * The pages use torchao's per-tensor MinMaxObserver ([SmolVLM-Q8] act_observer,
+ * qparams) and per-row choose_qparams_affine ([ET-21229]) without printing the
+ * formula.  This is the textbook asymmetric int8 scheme both implement:
+ *   range widened to contain 0:  mn = min(min x, 0), mx = max(max x, 0)
+ *   scale      s = (mx - mn) / 255                (fp32), floored at FLT_EPSILON
+ *   zero point z = clamp(-128 - round(mn / s), -128, 127)
+ * An all-zero range therefore gives s = FLT_EPSILON, z = -128.
+ */
+void q8o_qparams_from_minmax(float mn, float mx, float* s_out, int32_t* z_out) {
+    if (mn > 0.0f) mn = 0.0f;
+    if (mx < 0.0f) mx = 0.0f;
+    float scale = (mx - mn) / 255.0f;
+    if (scale < FLT_EPSILON) scale = FLT_EPSILON;
+    float zf = -128.0f - nearbyintf(mn / scale);
+    zf = clampf(zf, -128.0f, 127.0f);
+    *s_out = scale;
+    *z_out = (int32_t)zf;
+}
+
+/* One activation code: clamp(round(x * inv) + z, -128, 127), inv = 1/s in fp32.
+ * [SmolVLM-Q8] fake_quant and the quantized_decomposed quantize_per_tensor it
+ * mirrors multiply by the reciprocal scale rather than dividing. */
+static int8_t act_code(float x, float inv, int32_t z) {
+    float t = x * inv;
+    float r = nearbyintf(t) + (float)z;
+    r = clampf(r, -128.0f, 127.0f);
+    return (int8_t)(int)r;
+}
+
+/* [ET-21229] choose_qparams_affine: per-row asymmetric int8 scale / zero point
+ * from the row's min and max, then (optionally) the row's codes with them. */
+void q8o_choose_qparams(const uint16_t* x, int64_t M, int64_t K,
+                        float* s, int32_t* z, int8_t* xq) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = x + m * K;
+        float mn = 0.0f, mx = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_to_f32(row[k]);
+            if (v < mn) mn = v;
+            if (v > mx) mx = v;
+        }
+        float sc;
+        int32_t zp;
+        q8o_qparams_from_minmax(mn, mx, &sc, &zp);
+        s[m] = sc;
+        z[m] = zp;
+        if (xq) {
+            float inv = 1.0f / sc;
+            for (int64_t k = 0; k < K; ++k)
+                xq[m * K + k] = act_code(bf16_to_f32(row[k]), inv, zp);
+        }
+    }
+}
+
+/* Running min/max of a float tensor (the per-tensor observer's statistics). */
+void q8o_minmax(const float* x, int64_t n, float* mn, float* mx) {
+    float lo = x[0], hi = x[0];
+    for (int64_t i = 1; i < n; ++i) {
+        if (x[i] < lo) lo = x[i];
+        if (x[i] > hi) hi = x[i];
+    }
+    *mn = lo;
+    *mx = hi;
+}
+
+/* --------------------------------------------- static activation codes (a3)
+ * [SmolVLM-Q8] Q8Linear.forward: first pass xq1 = q(x, s1, z1).  With a second
+ * pass (module docstring "Two passes"), the residual of the first pass
+ *     r = x - fake_quant(x, s1, z1) = x - (xq1 - z1) * s1
+ * (each operation rounded to fp32 on its own) is quantized with (s2, z2). */
+static void static_quant_run(const float* x, int64_t n, float s1, int32_t z1,
+                             int8_t* xq1, int has2, float s2, int32_t z2, int8_t* xq2) {
+    float inv1 = 1.0f / s1;
+    float inv2 = has2 ? 1.0f / s2 : 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        int8_t c1 = act_code(x[i], inv1, z1);
+        xq1[i] = c1;
+        if (has2) {
+            float d1 = (float)((int32_t)c1 - z1) * s1;
+            float r = x[i] - d1;
+            xq2[i] = act_code(r, inv2, z2);
+        }
+    }
+}
+
+void q8o_static_quant(const float* x, int64_t M, int64_t K, float s1, int32_t z1,
+                      int8_t* xq1, int has2, float s2, int32_t z2, int8_t* xq2) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        static_quant_run(x + m * K, K, s1, z1, xq1 + m * K, has2, s2, z2,
+                         has2 ? xq2 + m * K : NULL);
+}
+
+/* ------------------------------------------------------------ W8A16 (a4)
+ * [tiny-llm] module docstring (the factorisation identity) and Int8Linear.forward:
+ *     y[m,n] = s_w[n] * sum_k x[m,k] * q[n,k]
+ * x is bf16, q int8: each product is exact in fp64 and the k-sequential fp64
+ * sum rounds at relative 2^-53 per step; the scale is applied once after it.  absum[m,n] = sum_k |x * q| * |s_w| bounds the rounding of any
+ * other summation order.  rows == NULL means every row m. */
+void q8o_linear_w8a16(const uint16_t* x, const int8_t* q, const float* s_w,
+                      int64_t M, int64_t N, int64_t K,
+                      const int64_t* rows, int64_t nrows,
+                      double* y, double* absum) {
+    int64_t R = rows ? nrows : M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < R; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        const uint16_t* xr = x + m * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const int8_t* qr = q + n * K;
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = (double)bf16_to_f32(xr[k]) * (double)qr[k];
+                acc += p;
+                mag += fabs(p);
+            }
+            y[i * N + n] = acc * (double)s_w[n];
+            if (absum) absum[i * N + n] = mag * fabs((double)s_w[n]);
+        }
+    }
+}
+
+/* ------------------------------------------------------ W8A8 (a5, a6)
+ * [SmolVLM-Q8] Q8Linear.forward: y = linear(dq(q(x,s1,z1)), dq_per_channel(W8, s_w))
+ * and, with a second pass, + linear(dq(q(r,s2,z2)), W8) (same int8 weight, no
+ * bias the second time).  Written out:
+ *     y[m,n] = s_w[n] * ( s1 * sum_k (xq1 - z1) q  +  s2 * sum_k (xq2 - z2) q )
+ * The two integer sums are exact (int64).  acc1/acc2 (optional) return the raw
+ * int32 dot products sum_k xq * q, the values the integer MMA accumulates.
+ * absum[m,n] = |s_w| * sum_k (|(xq1-z1) s1| + |(xq2-z2) s2|) |q|. */
+void q8o_linear_w8a8(const float* x, float s1, int32_t z1,
+                     int has2, float s2, int32_t z2,
+                     const int8_t* q, const float* s_w,
+                     int64_t M, int64_t N, int64_t K,
+                     const int64_t* rows, int64_t nrows,
+                     double* y, double* absum, int32_t* acc1, int32_t* acc2) {
+    int64_t R = rows ? nrows : M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < R; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        int8_t* c1 = (int8_t*)malloc((size_t)K);
+        int8_t* c2 = (int8_t*)calloc((size_t)K, 1);
+        static_quant_run(x + m * K, K, s1, z1, c1, has2, s2, z2, c2);
+        for (int64_t n = 0; n < N; ++n) {
+            const int8_t* qr = q + n * K;
+            int64_t t1 = 0, t2 = 0, a1 = 0, a2 = 0, g1 = 0, g2 = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t w = qr[k];
+                t1 += ((int64_t)c1[k] - z1) * w;
+                a1 += (int64_t)c1[k] * w;
+                g1 += llabs(((int64_t)c1[k] - z1) * w);
+                if (has2) {
+                    t2 += ((int64_t)c2[k] - z2) * w;
+                    a2 += (int64_t)c2[k] * w;
+                    g2 += llabs(((int64_t)c2[k] - z2) * w);
+                }
+            }
+            double v = (double)s1 * (double)t1;
+            double mag = (double)s1 * (double)g1;
+            if (has2) {
+                v += (double)s2 * (double)t2;
+                mag += (double)s2 * (double)g2;
+            }
+            y[i * N + n] = (double)s_w[n] * v;
+            if (absum) absum[i * N + n] = fabs((double)s_w[n]) * mag;
+            if (acc1) acc1[i * N + n] = (int32_t)a1;
+            if (acc2 && has2) acc2[i * N + n] = (int32_t)a2;
+        }
+        free(c1);
+        free(c2);
+    }
+}
+
+/* --------------------------------------------------- int4 group weights (a7)
+ * [ET-21229] names a 4-bit group-symmetric weight ("q4gsw") but prints neither
+ * grid nor packing.  Reading taken (the int8 rule of [ROCm-INT8] restated for
+ * 4 bits and per group of G consecutive k):
+ *   gs[n,g] = absmax(W[n, gG:(g+1)G]) / 7 (fp32); a group whose scale comes out
+ *   0 gets gs = 1 and codes 0; q4 = clamp(round(W / gs), -7, 7).
+ * Packing: byte k/2 of row n holds code k in its low nibble when k is even and
+ * in its high nibble when k is odd (two's complement nibbles). */
+void q8o_quantize_weight_q4gs(const float* W, int64_t N, int64_t K, int G,
+                              uint8_t* q4, float* gs) {
+    int64_t ng = K / G;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const float* w = W + n * K;
+        for (int64_t g = 0; g < ng; ++g) {
+            float amax = 0.0f;
+            for (int64_t k = g * G; k < (g + 1) * G; ++k) {
+                float a = fabsf(w[k]);
+                if (a > amax) amax = a;
+            }
+            float scale = amax / 7.0f;
+            int zero = (scale == 0.0f);
+            if (zero) scale = 1.0f;
+            gs[n * ng + g] = scale;
+            for (int64_t k = g * G; k < (g + 1) * G; ++k) {
+                int code = 0;
+                if (!zero) {
+                    float r = nearbyintf(w[k] / scale);
+                    code = (int)clampf(r, -7.0f, 7.0f);
+                }
+                uint8_t nib = (uint8_t)(code & 0xF);
+                uint8_t* byte = q4 + n * (K / 2) + k / 2;
+                if ((k & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | nib);
+                else              *byte = (uint8_t)((*byte & 0x0F) | (nib << 4));
+            }
+        }
+    }
+}
+
+/* Signed value of code k in a packed row (see q8o_quantize_weight_q4gs). */
+static int q4_code(const uint8_t* row, int64_t k) {
+    int nib = (k & 1) ? (row[k / 2] >> 4) & 0xF : row[k / 2] & 0xF;
+    return nib >= 8 ? nib - 16 : nib;
+}
+
+/* [ET-21229] linear_dq8ca_q4gsw:
+ *     out[m,n] = s[m] * sum_k (xq[m,k] - z[m]) * dequant(w)[n,k]
+ * with dequant(w)[n,k] = gs[n, k/G] * q4[n,k].  Evaluated as
+ *     s[m] * sum_g gs[n,g] * ( sum_{k in g} (xq - z) q4 )
+ * with the inner sums exact (int64) and the outer sum in fp64.
+ * absum[m,n] = |s[m]| * sum_g |gs[n,g]| * sum_{k in g} |(xq - z) q4|. */
+void q8o_linear_dq8ca_q4gsw(const int8_t* xq, const float* s, const int32_t* z,
+                            const uint8_t* q4, const float* gs, int G,
+                            int64_t M, int64_t N, int64_t K,
+                            const int64_t* rows, int64_t nrows,
+                            double* y, double* absum) {
+    int64_t R = rows ? nrows : M;
+    int64_t ng = K / G;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < R; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        const int8_t* xr = xq + m * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t* wr = q4 + n * (K / 2);
+            double acc = 0.0, mag = 0.0;
+            for (int64_t g = 0; g < ng; ++g) {
+                int64_t part = 0, pabs = 0;
+                for (int64_t k = g * G; k < (g + 1) * G; ++k) {
+                    int64_t p = ((int64_t)xr[k] - z[m]) * q4_code(wr, k);
+                    part += p;
+                    pabs += llabs(p);
+                }
+                acc += (double)gs[n * ng + g] * (double)part;
+                mag += fabs((double)gs[n * ng + g]) * (double)pabs;
+            }
+            y[i * N + n] = (double)s[m] * acc;
+            if (absum) absum[i * N + n] = fabs((double)s[m]) * mag;
+        }
+    }
+}
+
+/* ------------------------------------------------ int8 GEMM, int32 out (a8)
+ * acc[m,n] = sum_k a[m,k] * b[n,k], exact. */
+void q8o_gemm_s8s8_s32(const int8_t* a, const int8_t* b,
+                       int64_t M, int64_t N, int64_t K,
+                       const int64_t* rows, int64_t nrows, int32_t* acc) {
+    int64_t R = rows ? nrows : M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < R; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t t = 0;
+            for (int64_t k = 0; k < K; ++k)
+                t += (int64_t)a[m * K + k] * (int64_t)b[n * K + k];
+            acc[i * N + n] = (int32_t)t;
+        }
+    }
+}
+
+/* ------------------------------------------------------- output rounding
+ * Round an fp64 value once to bf16 (8 significant bits, ties to even), returned
+ * as its 16-bit pattern.  Used to form "the fp64 result rounded to bf16".
+ * Finite normal-range inputs only (the outputs of the linears above). */
+uint16_t q8o_round_bf16(double v) {
+    if (v == 0.0) return signbit(v) ? 0x8000 : 0x0000;
+    int e;
+    double m = frexp(v, &e);                 /* v = m * 2^e, 0.5 <= |m| < 1 */
+    double r = nearbyint(ldexp(m, 8));       /* 8 significant bits, ties even */
+    double b = ldexp(r, e - 8);              /* exactly a bf16 value */
+    float f = (float)b;                      /* exact */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+void q8o_round_bf16_array(const double* v, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = q8o_round_bf16(v[i]);
+}

@@ -1,0 +1,69 @@
+"""Mutation checks for the oracle's pins: each case plants one plausible mistake in a copy
+of the oracle source (on the CPU), rebuilds it, and requires that at least one pin fails.
+This shows the pins would catch that mistake in the real oracle."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import oracle.build as ob
+import test_oracle_pins as pins
+
+MUTANTS = [
+    # (name, text in q8_oracle.c, replacement, pins that must catch it)
+    ("ties away from zero (weights)", "float r = nearbyintf(w[k] / scale);   /* true",
+     "float r = roundf(w[k] / scale);   /* true", ["test_golden_weight_rows"]),
+    ("reciprocal instead of division (weights)", "float r = nearbyintf(w[k] / scale);   /* true",
+     "float r = nearbyintf(w[k] * (1.0f / scale));   /* true",
+     ["test_weight_codes_divide_not_reciprocal"]),
+    ("zero row keeps scale 0", "if (zero) scale = 1.0f;\n        int64_t sum",
+     "if (zero) scale = 0.0f;\n        int64_t sum", ["test_zero_row_rule_and_clamp"]),
+    ("row max instead of absmax", "float a = fabsf(w[k]);\n            if (a > amax) amax = a;\n        }\n        float scale = amax / 127.0f;",
+     "float a = w[k];\n            if (a > amax) amax = a;\n        }\n        float scale = amax / 127.0f;",
+     ["test_golden_weight_rows"]),
+    ("range not widened to 0", "if (mn > 0.0f) mn = 0.0f;", "",
+     ["test_qparams_from_minmax_matches_row_rule"]),
+    ("zero point sign", "float zf = -128.0f - nearbyintf(mn / scale);",
+     "float zf = -128.0f + nearbyintf(mn / scale);", ["test_golden_activation_rows"]),
+    ("divide activations by s", "float t = x * inv;", "float t = x / (1.0f / inv);",
+     ["test_activation_codes_multiply_by_reciprocal"]),
+    ("residual sign", "float r = x[i] - d1;", "float r = d1 - x[i];",
+     ["test_static_codes_use_fp32_reciprocal"]),
+    ("w8a8 drops the zero point", "t1 += ((int64_t)c1[k] - z1) * w;", "t1 += (int64_t)c1[k] * w;",
+     ["test_w8a8_matches_page_forward_and_exact_sums"]),
+    ("w8a8 second pass dropped", "v += (double)s2 * (double)t2;", "v += 0.0;",
+     ["test_w8a8_matches_page_forward_and_exact_sums"]),
+    ("w8a16 scale of wrong row", "y[i * N + n] = acc * (double)s_w[n];",
+     "y[i * N + n] = acc * (double)s_w[(n + 1) % N];", ["test_w8a16_factorisation_identity"]),
+    ("w8a16 transposed weight index", "(double)bf16_to_f32(xr[k]) * (double)qr[k];",
+     "(double)bf16_to_f32(xr[k]) * (double)q[k * N + n];",
+     ["test_w8a16_factorisation_identity"]),
+    ("q4 nibble order swapped", "if ((k & 1) == 0) *byte", "if ((k & 1) == 1) *byte",
+     ["test_golden_q4_groups"]),
+    ("q4 group scale index", "acc += (double)gs[n * ng + g] * (double)part;",
+     "acc += (double)gs[n * ng] * (double)part;", ["test_dq8ca_q4gsw_reductions"]),
+    ("q4 zero point dropped", "int64_t p = ((int64_t)xr[k] - z[m]) * q4_code(wr, k);",
+     "int64_t p = ((int64_t)xr[k]) * q4_code(wr, k);", ["test_dq8ca_q4gsw_reductions"]),
+    ("bf16 rounding truncates", "double r = nearbyint(ldexp(m, 8));",
+     "double r = trunc(ldexp(m, 8));", ["test_round_bf16"]),
+]
+
+
+@pytest.mark.parametrize("name,old,new,catchers", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(tmp_path, name, old, new, catchers):
+    src = open(ob.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique/found: {old!r}"
+    mut = tmp_path / "q8_oracle.c"
+    mut.write_text(src.replace(old, new))
+    (tmp_path / "q8_oracle.h").write_text(open(os.path.join(ob.HERE, "q8_oracle.h")).read())
+    so = str(tmp_path / "libmut.so")
+    subprocess.check_call(["gcc", *ob.CFLAGS, str(mut), "-o", so, "-lm"])
+    caught = []
+    with oracle.use_library(so):
+        for fn in catchers:
+            try:
+                getattr(pins, fn)()
+            except AssertionError:
+                caught.append(fn)
+    assert caught, f"mutant '{name}' survived pins {catchers}"

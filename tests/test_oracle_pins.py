@@ -1,0 +1,406 @@
+"""Pins for the CPU oracle: checks against what the pages and mathematics fix.
+
+Nothing here compares the oracle with itself.  Each check is one of:
+  * a hand-worked value from tests/golden/ (each file cites the page rule it follows);
+  * brute force in exact rational arithmetic (tests/exact.py) on tiny inputs;
+  * a closed-form bound or invariant (nearest-grid error, two-pass bound, zero point);
+  * a special case that reduces to a library routine (numpy matmul, torch bf16 cast).
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import q8_workloads as wl
+from exact import bf16_bits_to_fraction, f32, rn32, rn_bf16, rne_int
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _parse(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            rows.append([part.split() for part in line.split("|")])
+    return rows
+
+
+def _bf16(values):
+    return wl.bf16_bits(torch.tensor(values, dtype=torch.float32).to(torch.bfloat16))
+
+
+# ----------------------------------------------------------------- golden rows
+
+
+def test_golden_weight_rows():
+    """Int8Linear's quantize_weight rule (ROCm INT8 page) on hand-worked rows."""
+    rows = _parse("weight_int8_rows.txt")
+    W = np.array([[float(v) for v in r[0]] for r in rows], np.float32)
+    q, s, ws = oracle.quantize_weight(W)
+    for i, r in enumerate(rows):
+        assert q[i].tolist() == [int(v) for v in r[2]], f"row {i} codes"
+        assert ws[i] == int(r[3][0]), f"row {i} code sum"
+        assert s[i] == pytest.approx(float(r[1][0]), rel=1e-7), f"row {i} scale"
+    assert s[0] == 1.0 and s[1] == 2.0 and s[2] == 1.0      # exact scales
+
+
+def test_golden_activation_rows():
+    """choose_qparams_affine (executorch PR #21229) on hand-worked rows."""
+    rows = _parse("act_qparams_rows.txt")
+    x = _bf16([[float(v) for v in r[0]] for r in rows])
+    s, z, xq = oracle.choose_qparams(x)
+    for i, r in enumerate(rows):
+        assert z[i] == int(r[1][0]), f"row {i} zero point"
+        assert xq[i].tolist() == [int(v) for v in r[2]], f"row {i} codes"
+    assert s[0] == np.float32(4.0) / np.float32(255.0)
+    assert s[1] == np.finfo(np.float32).eps
+    assert s[2] == np.float32(4.0) / np.float32(255.0)
+
+
+def test_golden_q4_groups():
+    """int4 group-symmetric codes and nibble packing on hand-worked groups."""
+    rows = _parse("weight_q4gs_groups.txt")
+    W = np.array([[float(v) for r in rows for v in r[0]]], np.float32)   # 1 x 12, G = 4
+    q4, gs = oracle.quantize_weight_q4gs(W, 4)
+    want_bytes = [int(b, 16) for r in rows for b in r[3]]
+    assert q4[0].tolist() == want_bytes
+    assert gs[0].tolist() == [float(r[1][0]) for r in rows]
+
+
+# ------------------------------------------------------ weight codes, brute force
+
+
+def _weight_codes_exact(w_row):
+    amax = max(abs(f32(v)) for v in w_row)
+    s = rn32(amax / 127) if amax else Fraction(0)
+    if s == 0:
+        return Fraction(1), [0] * len(w_row)
+    codes = [max(-127, min(127, rne_int(rn32(f32(v) / s)))) for v in w_row]
+    return s, codes
+
+
+def test_quantize_weight_exact_rational():
+    W = wl.weight(12, 37, seed=11).numpy()
+    W[3] = 0.0
+    W[5, :] = 0.0
+    W[5, 7] = -1e-3
+    W[8] *= 1e-30                                    # tiny but normal scales
+    q, s, ws = oracle.quantize_weight(W)
+    for n in range(W.shape[0]):
+        s_ex, codes = _weight_codes_exact(W[n])
+        assert Fraction(float(s[n])) == s_ex
+        assert q[n].tolist() == codes
+        assert int(ws[n]) == sum(codes)
+
+
+def _find_div_vs_recip_case():
+    """A weight row where round(w / s) and round(w * (1/s)) differ in fp32."""
+    rng = np.random.default_rng(5)
+    for _ in range(200000):
+        amax = np.float32(rng.uniform(0.5, 2.0))
+        s = amax / np.float32(127.0)
+        k = int(rng.integers(-120, 120))
+        w = np.float32((k + 0.5) * float(s))
+        if abs(w) >= amax:
+            continue
+        by_div = rne_int(rn32(f32(w) / f32(s)))
+        by_rec = rne_int(rn32(f32(w) * rn32(1 / f32(s))))
+        if by_div != by_rec:
+            return np.array([[amax, w]], np.float32), by_div
+    raise AssertionError("no case found")
+
+
+def test_weight_codes_divide_not_reciprocal():
+    """The ROCm page divides (round(w / scale)); a case where a reciprocal would differ."""
+    W, want = _find_div_vs_recip_case()
+    q, _, _ = oracle.quantize_weight(W)
+    assert int(q[0, 1]) == want
+
+
+def test_weight_codes_nearest_grid_point():
+    """|q*s - w| <= s/2 (up to the fp32 division) and ties go to the even code."""
+    W = wl.weight(64, 256, seed=12).numpy()
+    q, s, _ = oracle.quantize_weight(W)
+    err = np.abs(q.astype(np.float64) * s[:, None].astype(np.float64) - W.astype(np.float64))
+    assert np.all(err <= s[:, None] * (0.5 + 2.0 ** -20))
+    assert np.abs(q).max() == 127                   # the absmax element of each row hits 127
+    assert np.all(np.abs(q).max(axis=1) == 127)
+
+
+def test_zero_row_rule_and_clamp():
+    """All-zero row: scale 1.0, codes 0 (ROCm page); p3's 'scale 0' reading is not used."""
+    W = np.zeros((3, 16), np.float32)
+    W[1, 4] = 3.0
+    q, s, ws = oracle.quantize_weight(W)
+    assert s[0] == 1.0 and s[2] == 1.0 and not q[0].any() and not q[2].any()
+    assert q[1, 4] == 127 and ws[1] == 127
+
+
+# -------------------------------------------------------- activation codes
+
+
+def _act_codes_exact(x_vals, s, z):
+    inv = rn32(1 / s)
+    out = []
+    for v in x_vals:
+        t = rne_int(rn32(v * inv)) + z
+        out.append(max(-128, min(127, t)))
+    return out
+
+
+def _qparams_exact(mn, mx):
+    mn = min(mn, Fraction(0))
+    mx = max(mx, Fraction(0))
+    s = rn32(rn32(mx - mn) / 255)
+    eps = Fraction(2) ** -23
+    if s < eps:
+        s = eps
+    z = max(-128, min(127, -128 - rne_int(rn32(mn / s))))
+    return s, z
+
+
+def test_choose_qparams_exact_rational():
+    xt = wl.normal_bf16((9, 33), 1.0, seed=13)
+    xt[2] = torch.abs(xt[2])                         # positive-only row
+    xt[3] = -torch.abs(xt[3])                        # negative-only row
+    xt[4] = 0.0                                      # all zero
+    xt[5] *= 1000.0
+    bits = wl.bf16_bits(xt)
+    s, z, xq = oracle.choose_qparams(bits)
+    for m in range(bits.shape[0]):
+        vals = [bf16_bits_to_fraction(b) for b in bits[m]]
+        s_ex, z_ex = _qparams_exact(min(vals), max(vals))
+        assert Fraction(float(s[m])) == s_ex, m
+        assert int(z[m]) == z_ex, m
+        assert xq[m].tolist() == _act_codes_exact(vals, s_ex, z_ex), m
+
+
+def test_activation_code_invariants():
+    """Real 0 maps to z; the row min maps to -128 and the max to 127 when the row
+    straddles 0 (the affine grid's end points)."""
+    bits = wl.bf16_bits(wl.normal_bf16((64, 128), 1.0, seed=14))
+    s, z, xq = oracle.choose_qparams(bits)
+    vals = bits.view(np.uint16).astype(np.uint32) << 16
+    xf = vals.view(np.float32).reshape(bits.shape)
+    for m in range(xf.shape[0]):
+        assert xq[m, np.argmin(xf[m])] == -128
+        assert xq[m, np.argmax(xf[m])] == 127
+    zero_bits = _bf16([[0.0, 1.0, -2.0]])
+    s0, z0, xq0 = oracle.choose_qparams(zero_bits)
+    assert xq0[0, 0] == z0[0]
+
+
+def test_qparams_from_minmax_matches_row_rule():
+    """The per-tensor observer formula and the per-row one are the same function."""
+    bits = wl.bf16_bits(wl.normal_bf16((4, 50), 2.0, seed=15))
+    s, z, _ = oracle.choose_qparams(bits, want_codes=False)
+    xf = (bits.astype(np.uint32) << 16).view(np.float32)
+    for m in range(4):
+        s_t, z_t = oracle.qparams_from_minmax(xf[m].min(), xf[m].max())
+        assert (np.float32(s_t), z_t) == (s[m], z[m])
+    s_ex, z_ex = _qparams_exact(Fraction(-1), Fraction(3))
+    assert oracle.qparams_from_minmax(-1.0, 3.0) == (float(s_ex), z_ex)
+    # ranges that exclude 0 are widened to contain it (golden activation row 2 by hand)
+    s425 = float(np.float32(4.0) / np.float32(255.0))
+    assert oracle.qparams_from_minmax(1.0, 4.0) == (s425, -128)
+    assert oracle.qparams_from_minmax(-4.0, -1.0) == (s425, 127)
+
+
+def test_static_codes_use_fp32_reciprocal():
+    """fake_quant (SmolVLM q8 page) multiplies by 1/s; exact-rational check of codes and of
+    the residual r = x - (xq1 - z1) * s1, each step rounded to fp32."""
+    x = wl.normal((5, 40), 4.0, seed=16).numpy()
+    s1, z1 = oracle.qparams_from_minmax(-9.0, 11.0)
+    s2, z2 = float(np.float32(s1) / np.float32(255.0)), 0
+    xq1, xq2 = oracle.static_quant(x, (s1, z1), (s2, z2))
+    S1, S2 = f32(s1), f32(s2)
+    for m in range(x.shape[0]):
+        vals = [f32(v) for v in x[m]]
+        c1 = _act_codes_exact(vals, S1, z1)
+        assert xq1[m].tolist() == c1
+        r = [rn32(v - rn32((c - z1) * S1)) for v, c in zip(vals, c1)]
+        assert xq2[m].tolist() == _act_codes_exact(r, S2, z2)
+
+
+def _find_recip_vs_div_act_case():
+    """An activation x and scale s where round(x * (1/s)) and round(x / s) differ in fp32."""
+    rng = np.random.default_rng(7)
+    for _ in range(200000):
+        s = np.float32(rng.uniform(0.01, 0.1))
+        k = int(rng.integers(-100, 100))
+        x = np.float32((k + 0.5) * float(s))
+        by_rec = rne_int(rn32(f32(x) * rn32(1 / f32(s))))
+        by_div = rne_int(rn32(f32(x) / f32(s)))
+        if by_rec != by_div:
+            return x, s, by_rec
+    raise AssertionError("no case found")
+
+
+def test_activation_codes_multiply_by_reciprocal():
+    """fake_quant / quantize_per_tensor multiply by 1/s; a case where dividing would differ."""
+    x, s, want = _find_recip_vs_div_act_case()
+    xq1, _ = oracle.static_quant(np.array([[x]], np.float32), (float(s), 0))
+    assert int(xq1[0, 0]) == max(-128, min(127, want))
+
+
+def test_quant_error_bounds_single_and_two_pass():
+    """Single pass: |x - dq(q(x))| <= s1/2.  Two passes with s2 = s1/255, z2 = 0:
+    |x - dq1 - dq2| <= s1/510 (SmolVLM q8 page, module docstring), up to fp32 rounding."""
+    s1, z1 = oracle.qparams_from_minmax(-6.0, 6.0)
+    lo, hi = (-128 - z1) * s1, (127 - z1) * s1
+    x = np.random.default_rng(17).uniform(lo, hi, size=(8, 4096)).astype(np.float32)
+    s2 = float(np.float32(s1) / np.float32(255.0))
+    xq1, xq2 = oracle.static_quant(x, (s1, z1), (s2, 0))
+    d1 = (xq1.astype(np.float64) - z1) * s1
+    d2 = xq2.astype(np.float64) * s2
+    e1 = np.abs(x - d1).max()
+    e2 = np.abs(x - d1 - d2).max()
+    assert e1 <= s1 / 2 * (1 + 2.0 ** -18)
+    assert e2 <= s1 / 510 * (1 + 2.0 ** -10) + 4 * np.spacing(np.float32(max(abs(lo), hi)))
+    assert e2 < e1 / 100
+
+
+# ------------------------------------------------------------------ linears
+
+
+def test_int8_to_bf16_cast_is_exact():
+    """tiny-llm page: the int8 -> bf16 cast is exact (|q| <= 127 < 256)."""
+    q = torch.arange(-128, 128, dtype=torch.int32)
+    assert torch.equal(q.to(torch.bfloat16).to(torch.int32), q)
+
+
+def test_w8a16_factorisation_identity():
+    """y = s * (x q^T) equals x dq(W)^T (tiny-llm module docstring) -- numpy fp64 GEMM."""
+    x = wl.normal_bf16((5, 96), 1.0, seed=18)
+    q, s, _ = oracle.quantize_weight(wl.weight(40, 96, seed=19).numpy())
+    y, a = oracle.linear_w8a16(wl.bf16_bits(x), q, s)
+    ref = x.double().numpy() @ (q.astype(np.float64) * s.astype(np.float64)[:, None]).T
+    assert np.all(np.abs(y - ref) <= 1e-12 * a + 1e-300)
+    assert np.abs(y).max() > 0
+
+
+def test_w8a16_exact_rational_small():
+    x = wl.normal_bf16((3, 7), 1.0, seed=20)
+    bits = wl.bf16_bits(x)
+    q, s, _ = oracle.quantize_weight(wl.weight(5, 7, seed=21).numpy())
+    y, _ = oracle.linear_w8a16(bits, q, s)
+    for m in range(3):
+        for n in range(5):
+            exact = sum(bf16_bits_to_fraction(bits[m, k]) * int(q[n, k]) for k in range(7))
+            assert y[m, n] == float(exact * f32(s[n]))
+
+
+def test_w8a16_rows_subset_and_thread_independence():
+    x = wl.bf16_bits(wl.normal_bf16((9, 64), 1.0, seed=22))
+    q, s, _ = oracle.quantize_weight(wl.weight(33, 64, seed=23).numpy())
+    oracle.set_num_threads(1)
+    y1, _ = oracle.linear_w8a16(x, q, s)
+    oracle.set_num_threads(8)
+    y8, _ = oracle.linear_w8a16(x, q, s)
+    ys, _ = oracle.linear_w8a16(x, q, s, rows=[7, 2])
+    assert np.array_equal(y1, y8)
+    assert np.array_equal(ys, y1[[7, 2]])
+
+
+def test_w8a8_matches_page_forward_and_exact_sums():
+    """Q8Linear.forward (SmolVLM q8 page): linear(dq(q(x,s1)), dq(W)) + linear(dq(q(r,s2)), dq(W)),
+    evaluated here with numpy fp64 matmuls on the dequantized operands; the raw int32 sums
+    against an int64 matmul; and one entry in exact rational arithmetic."""
+    x, calib = wl.w8a8_inputs(6, K=64)
+    x = x.numpy()
+    s1, z1 = oracle.qparams_from_minmax(*oracle.minmax(calib.numpy()))
+    s2 = float(np.float32(s1) / np.float32(255.0))
+    q, sw, wsum = oracle.quantize_weight(wl.weight(24, 64, seed=24).numpy())
+    for second in (None, (s2, 0)):
+        y, a, acc1, acc2 = oracle.linear_w8a8(x, (s1, z1), q, sw, second=second)
+        xq1, xq2 = oracle.static_quant(x, (s1, z1), second)
+        dqw = q.astype(np.float64) * sw.astype(np.float64)[:, None]
+        ref = ((xq1.astype(np.float64) - z1) * s1) @ dqw.T
+        if second is not None:
+            ref += (xq2.astype(np.float64) * s2) @ dqw.T
+            assert np.array_equal(acc2, xq2.astype(np.int64) @ q.astype(np.int64).T)
+        assert np.all(np.abs(y - ref) <= 1e-12 * a)
+        assert np.array_equal(acc1, xq1.astype(np.int64) @ q.astype(np.int64).T)
+        t = sum((int(xq1[2, k]) - z1) * int(q[5, k]) for k in range(64))
+        ex = f32(s1) * t
+        if second is not None:
+            ex += f32(s2) * sum(int(xq2[2, k]) * int(q[5, k]) for k in range(64))
+        assert abs(Fraction(y[2, 5]) - f32(sw[5]) * ex) <= abs(f32(sw[5]) * ex) * Fraction(1, 2**50)
+
+
+def test_w8a8_zero_point_term_matters():
+    """A nonzero z1 changes y by s_w s1 z1 sum_k q -- the weight_sums correction term."""
+    x = wl.normal((2, 32), 1.0, seed=25).numpy()
+    q, sw, wsum = oracle.quantize_weight(wl.weight(8, 32, seed=26).numpy())
+    s1 = 0.05
+    ya, _, acc_a, _ = oracle.linear_w8a8(x, (s1, 0), q, sw)
+    yb, _, acc_b, _ = oracle.linear_w8a8(x, (s1, 10), q, sw)
+    # codes shift by exactly 10 (no clamping for these magnitudes)
+    assert np.array_equal(acc_b - acc_a, 10 * np.broadcast_to(wsum, acc_a.shape))
+    assert np.allclose(ya, yb, rtol=1e-12, atol=1e-12)
+
+
+def test_q4gs_nearest_grid_and_packing():
+    W = wl.weight(16, 256, seed=27).numpy()
+    for G in (32, 128):
+        q4, gs = oracle.quantize_weight_q4gs(W, G)
+        lo = (q4 & 0xF).astype(np.int8)
+        hi = (q4 >> 4).astype(np.int8)
+        codes = np.empty((16, 256), np.int64)
+        codes[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+        codes[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+        assert codes.min() >= -7 and codes.max() <= 7
+        g = np.repeat(gs.astype(np.float64), G, axis=1)
+        assert np.all(np.abs(codes * g - W) <= g * (0.5 + 2.0 ** -20))
+
+
+def test_dq8ca_q4gsw_reductions():
+    """8da4w: (a) against numpy fp64 matmul of (xq - z) and the dequantized weight;
+    (b) with G = K and gs = 1 it is s[m] * sum_k (xq - z) q4, an integer matmul."""
+    bits = wl.bf16_bits(wl.normal_bf16((5, 128), 1.0, seed=28))
+    s, z, xq = oracle.choose_qparams(bits)
+    W = wl.weight(12, 128, seed=29).numpy()
+    for G in (32, 128):
+        q4, gs = oracle.quantize_weight_q4gs(W, G)
+        y, a = oracle.linear_dq8ca_q4gsw(xq, s, z, q4, gs, G)
+        lo = (q4 & 0xF).astype(np.int64)
+        hi = (q4 >> 4).astype(np.int64)
+        codes = np.empty((12, 128), np.int64)
+        codes[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+        codes[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+        dqw = codes * np.repeat(gs.astype(np.float64), G, axis=1)
+        xa = (xq.astype(np.float64) - z[:, None]) * s.astype(np.float64)[:, None]
+        ref = xa @ dqw.T
+        assert np.all(np.abs(y - ref) <= 1e-12 * a)
+        if G == 128:
+            ones = np.ones_like(gs)
+            y1, _ = oracle.linear_dq8ca_q4gsw(xq, s, z, q4, ones, G)
+            ints = (xq.astype(np.int64) - z[:, None]) @ codes.T
+            assert np.array_equal(y1, ints * s.astype(np.float64)[:, None])
+
+
+def test_gemm_s8s8_s32_exact():
+    rng = np.random.default_rng(30)
+    a = rng.integers(-128, 128, size=(7, 300), dtype=np.int8)
+    b = rng.integers(-128, 128, size=(9, 300), dtype=np.int8)
+    assert np.array_equal(oracle.gemm_s8s8_s32(a, b), a.astype(np.int64) @ b.astype(np.int64).T)
+
+
+def test_round_bf16():
+    """Once-rounding fp64 -> bf16: torch's fp32 -> bf16 cast on fp32-exact values, ties to even,
+    and values that an fp64 -> fp32 -> bf16 double rounding would get wrong."""
+    v = wl.normal((1000,), 3.0, seed=31)
+    want = wl.bf16_bits(v.to(torch.bfloat16))
+    assert np.array_equal(oracle.round_bf16(v.double().numpy()), want)
+    one = 1.0
+    cases = [one + 2 ** -8, one + 3 * 2 ** -8, -(one + 2 ** -8), one + 2 ** -8 + 2 ** -40]
+    got = oracle.round_bf16(np.array(cases))
+    exp = [rn_bf16(Fraction(c)) for c in cases]
+    assert [bf16_bits_to_fraction(g) for g in got] == exp
+    assert got[3] == 0x3F81                          # just above the tie: rounds up
