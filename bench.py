@@ -1,0 +1,513 @@
+#!/usr/bin/env python
+"""Benchmark of the int8 quantized linears on B200.
+
+Headline workload: the W8A16 decode sweep -- bf16 activations (M in {1, 4, 16}) times int8
+per-channel weights of shapes (K, N) in {(960, 2560), (2048, 8192), (4096, 11008),
+(4096, 32000)}, bf16 output.  One step runs every (shape, M) case once, as one CUDA graph
+of 12 GEMV launches; the metric is algorithmic bytes moved (int8 weights + fp32 scales +
+bf16 activations + bf16 outputs) per second.  Two copies of every weight rotate between
+steps (390 MB, over 3x the 126 MB L2), and within a step cases run M-major, so a weight
+is never re-read from L2.
+
+Extra sub-benchmarks (same JSON line, key "paths"): W8A8 static int8 linear (K = 960) and
+the quantizers.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched under torch.distributed.run) every rank runs an independent replica
+(the path has no exchange step); time is the max over ranks and the value counts all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import q8_workloads as wl  # noqa: E402
+
+METRIC = "W8A16 decode GB/s (% of HBM peak); W8A8/8da4w prefill TOPS (% int8 peak)"
+UNIT = "GB/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-paths", action="store_true", help="skip the sub-benchmarks")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- distributed
+
+
+class Dist:
+    def __init__(self, gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import torch.distributed as dist
+
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        else:
+            torch.cuda.set_device(0)
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 20 ms on this rank's GPU while the timed region runs."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="q8clk_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "20"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = list(csv.reader(io.StringIO(open(self.path).read())))
+        os.unlink(self.path)
+        return rows
+
+    @staticmethod
+    def summarize(rows, t0: float, t1: float) -> dict:
+        def ts(r):
+            try:
+                return datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                return None
+
+        good = [r for r in rows if len(r) >= 10]
+        inside = [r for r in good if ts(r) is not None and t0 <= ts(r) <= t1]
+        window = "timed region"
+        if len(inside) < 3:
+            inside, window = good, "warm-up + timed region (timed region shorter than 3 samples)"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in inside]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in inside:
+            for name, v in zip(names, r[6:10]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(inside[0][3]),
+                "reasons": sorted(reasons), "samples": len(inside), "window": window,
+                "power_w_max": max(float(r[4]) for r in inside)}
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+
+def w8a16_bytes(M, N, K):
+    return N * K + 4 * N + 2 * M * K + 2 * M * N
+
+
+class W8A16Sweep:
+    """Device-resident W8A16 decode sweep: 2 rotating copies of every weight."""
+
+    COPIES = 2
+
+    def __init__(self, dev):
+        import int8_quantized_linear_q8_b200 as q8
+
+        self.q8 = q8
+        g = torch.Generator(device=dev)
+        self.shapes = []
+        for i, sh in enumerate(wl.W8A16_SWEEP_SHAPES):
+            g.manual_seed(wl.W8A16_SWEEP_SEED_W * 1000 + i)
+            W = torch.randn(sh.N, sh.K, generator=g, device=dev) * 0.02
+            q, s, _ = q8.q8_quantize_weight(W, want_wsum=False)
+            del W
+            copies = [q] + [q.clone() for _ in range(self.COPIES - 1)]
+            self.shapes.append((sh, copies, s))
+        self.xs, self.ys = {}, {}
+        for M in wl.W8A16_SWEEP_M:
+            for i, (sh, _, _) in enumerate(self.shapes):
+                g.manual_seed(wl.W8A16_SWEEP_SEED_X * 1000 + 10 * i + M)
+                self.xs[(i, M)] = torch.randn(M, sh.K, generator=g, device=dev).to(torch.bfloat16)
+                self.ys[(i, M)] = torch.empty(M, sh.N, dtype=torch.bfloat16, device=dev)
+        self.cases = [(i, M) for M in wl.W8A16_SWEEP_M for i in range(len(self.shapes))]
+        self.step_bytes = sum(w8a16_bytes(M, self.shapes[i][0].N, self.shapes[i][0].K)
+                              for i, M in self.cases)
+        self.weight_bytes = sum(sh.N * sh.K * self.COPIES for sh, _, _ in self.shapes)
+        torch.cuda.synchronize()
+
+    def launch(self, i, M, copy):
+        sh, copies, s = self.shapes[i]
+        self.q8.q8_linear_w8a16(self.xs[(i, M)], copies[copy], s, y=self.ys[(i, M)])
+
+    def step(self, copy):
+        for i, M in self.cases:
+            self.launch(i, M, copy)
+
+    def graphs(self):
+        """One CUDA graph per weight copy, each one full step."""
+        out = []
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for c in range(self.COPIES):
+                self.step(c)   # warm the launch path outside capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        for c in range(self.COPIES):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                self.step(c)
+            out.append(gr)
+        torch.cuda.synchronize()
+        return out
+
+
+def time_graphs(graphs, steps: int, warmup: int, dist: Dist):
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    e0.record(st)
+    for i in range(steps):
+        graphs[i % len(graphs)].replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    dist.barrier()
+    ms = e0.elapsed_time(e1)
+    return dist.max(ms), t0, t1
+
+
+def per_case_times(sweep: W8A16Sweep, reps: int = 50):
+    """Average device time of each case's kernel, alone, from a graph of `reps` launches
+    alternating weight copies (events on the launching stream)."""
+    out = []
+    for i, M in sweep.cases:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            sweep.launch(i, M, 0)
+        torch.cuda.current_stream().wait_stream(s)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for r in range(reps):
+                sweep.launch(i, M, r % sweep.COPIES)
+        gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(3):
+            gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1000.0 / (3 * reps)
+        sh = sweep.shapes[i][0]
+        b = w8a16_bytes(M, sh.N, sh.K)
+        out.append({"K": sh.K, "N": sh.N, "M": M, "us": round(us, 3),
+                    "GBps": round(b / us / 1e3, 1)})
+        del gr
+    return out
+
+
+def e2e_w8a16(sweep: W8A16Sweep, steps: int, warmup: int, dist: Dist):
+    """Same metric through the public API with host buffers: every step copies each case's
+    activations host->device (pinned) and reads each output back device->host."""
+    q8 = sweep.q8
+    hx = {k: v.cpu().pin_memory() for k, v in sweep.xs.items()}
+    hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in sweep.ys.items()}
+    dx = {k: torch.empty_like(v) for k, v in sweep.xs.items()}
+    h2d = sum(v.numel() * v.element_size() for v in hx.values())
+    d2h = sum(v.numel() * v.element_size() for v in hy.values())
+
+    def step(c):
+        for i, M in sweep.cases:
+            sh, copies, s = sweep.shapes[i]
+            dx[(i, M)].copy_(hx[(i, M)], non_blocking=True)
+            q8.q8_linear_w8a16(dx[(i, M)], copies[c], s, y=sweep.ys[(i, M)])
+            hy[(i, M)].copy_(sweep.ys[(i, M)], non_blocking=True)
+
+    for i in range(warmup):
+        step(i % sweep.COPIES)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i % sweep.COPIES)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dist.max(e0.elapsed_time(e1))
+    value = dist.world * steps * sweep.step_bytes / (ms * 1e-3) / 1e9
+    return {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / steps, 4)}
+
+
+def cpu_baseline_w8a16(sweep: W8A16Sweep, budget_s: float = 12.0):
+    """The oracle, as it stands, on the host cores: the M = 1 case of each sweep shape
+    (full weights), repeated until about `budget_s` seconds have passed."""
+    import oracle
+
+    hq = [(sh, copies[0].cpu().numpy(), s.cpu().numpy()) for sh, copies, s in sweep.shapes]
+    hx = {i: sweep.xs[(i, 1)].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+          for i in range(len(hq))}
+    done_bytes, t0, reps = 0, time.perf_counter(), 0
+    while True:
+        for i, (sh, q, s) in enumerate(hq):
+            oracle.linear_w8a16(hx[i], q, s)
+            done_bytes += w8a16_bytes(1, sh.N, sh.K)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": round(done_bytes / el / 1e9, 3), "unit": UNIT,
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"M=1 case of each of the 4 sweep shapes (full weights), {reps} passes, "
+                      f"{el:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- sub-benchmarks
+
+
+def bench_w8a8_paths(dev, reps=30):
+    """W8A8 static (K = 960, N in {960, 2560}, M in {1, 256, 2048}; one and two passes):
+    achieved int8 TOPS (2 M N K per pass) and GB/s (fp32 x in, fp32 y out, int8 W)."""
+    import int8_quantized_linear_q8_b200 as q8
+
+    out = []
+    K = wl.W8A8_K
+    x_all, calib = wl.w8a8_inputs(max(wl.W8A8_M), K=K)
+    mm = torch.empty(2, device=dev)
+    q8.q8_observe_minmax(calib.to(dev), mm, reset=True)
+    first = q8.q8_qparams_from_minmax(*mm.cpu().tolist())
+    second = (float(np.float32(first[0]) / np.float32(255.0)), 0)
+    for N in wl.W8A8_N:
+        W = wl.weight(N, K, seed=wl.W8A8_SEED_W).to(dev)
+        q, s, ws = q8.q8_quantize_weight(W)
+        for M in wl.W8A8_M:
+            x = x_all[:M].contiguous().to(dev)
+            y = torch.empty(M, N, device=dev)
+            for two in (False, True):
+                sec = second if two else None
+                wsb = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, M, N, K, int(two))
+                work = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+                fn = lambda: q8.q8_linear_w8a8(x, first, q, ws, s, second=sec, y=y, workspace=work)
+                us = _graph_time(fn, reps)
+                ops = 2.0 * M * N * K * (2 if two else 1)
+                byts = 4 * M * K + N * K + 8 * N + 4 * M * N
+                out.append({"K": K, "N": N, "M": M, "two_pass": two, "us": round(us, 2),
+                            "TOPS": round(ops / us / 1e6, 2), "GBps": round(byts / us / 1e3, 1)})
+    return out
+
+
+def _graph_time(fn, reps):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for _ in range(reps):
+            fn()
+    gr.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1000.0 / (3 * reps)
+
+
+# ----------------------------------------------------------------------------- arms
+
+
+def run_ours(args):
+    dist = Dist(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    import int8_quantized_linear_q8_b200 as q8
+    from int8_quantized_linear_q8_b200 import build as q8build
+
+    if dist.rank == 0:
+        q8build.build()
+    dist.barrier()
+    q8.lib()
+
+    sweep = W8A16Sweep(dev)
+    graphs = sweep.graphs()
+    clk = ClockSampler(dist.local)
+    clk.start()
+    ms, t0, t1 = time_graphs(graphs, args.steps, args.warmup, dist)
+    rows = clk.stop()
+    clocks = ClockSampler.summarize(rows, t0, t1) if isinstance(rows, list) else rows
+    del graphs
+    ms_per_step = ms / args.steps
+    value = dist.world * args.steps * sweep.step_bytes / (ms * 1e-3) / 1e9
+    peaks = measured_peaks()
+    per_rank_gbps = args.steps * sweep.step_bytes / (ms * 1e-3) / 1e9
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 activations; N(0,0.02^2) fp32 weights "
+                "quantized per channel on the GPU)",
+        "config": {"workload": "W8A16 decode sweep: bf16 x [M,K] (M in 1,4,16) times int8 "
+                               "W [N,K], (K,N) in (960,2560),(2048,8192),(4096,11008),"
+                               "(4096,32000); bf16 out",
+                   "step": "12 GEMV launches (every shape x M), one CUDA graph",
+                   "bytes_per_step": sweep.step_bytes,
+                   "l2": f"inputs larger than L2: {sweep.COPIES} rotating weight copies "
+                         f"({sweep.weight_bytes / 1e6:.0f} MB) vs 126 MB L2; M-major order",
+                   "parallelism": f"replicas x{dist.world}"},
+        "roofline": {"bound": "hbm", "kernel": "k_w8a16_gemv",
+                     "achieved": round(per_rank_gbps, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(per_rank_gbps / peaks["hbm_gbs"], 4),
+                     "peak_source": peaks["source"], "traffic": None,
+                     "bytes_per_launch_avg": sweep.step_bytes // len(sweep.cases)},
+        "gpu_launches": args.steps * len(sweep.cases),
+        "clocks": clocks,
+    }
+    if dist.rank == 0:
+        result["cases"] = per_case_times(sweep)
+    result["e2e"] = e2e_w8a16(sweep, max(10, min(args.steps // 10, 200)), 3, dist)
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline_w8a16(sweep)
+    if dist.rank == 0 and not args.no_paths:
+        result["paths"] = {"w8a8_static_k960": bench_w8a8_paths(dev)}
+    dist.barrier()
+    if dist.rank == 0:
+        print(json.dumps(result), flush=True)
+    dist.close()
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on the host cores, on the same metric
+    (W8A16 decode GB/s).  Each step is a bounded sample of the workload: the M = 1 case of
+    each sweep shape restricted to its first 256 output channels."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+
+    shapes = wl.W8A16_SWEEP_SHAPES
+    data = []
+    rows = 256
+    for i, sh in enumerate(shapes):
+        W = wl.weight(rows, sh.K, seed=wl.W8A16_SWEEP_SEED_W * 1000 + i)
+        q, s, _ = oracle.quantize_weight(W.numpy())
+        x = wl.bf16_bits(wl.normal_bf16((1, sh.K), 1.0, seed=wl.W8A16_SWEEP_SEED_X * 1000 + i))
+        data.append((sh, q, s, x))
+    step_bytes = sum(w8a16_bytes(1, rows, sh.K) for sh, _, _, _ in data)
+
+    def step():
+        for sh, q, s, x in data:
+            oracle.linear_w8a16(x, q, s)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = args.steps * step_bytes / el / 1e9
+    sample = "per step: M=1 case of each of the 4 sweep shapes, first 256 output channels"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(el * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": "W8A16 decode sweep (M=1 sample)",
+                                        "bytes_per_step": step_bytes},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,212 @@
+/*
+ * q8.h -- C ABI of the B200 (sm_100a) int8 quantized-linear library, libq8.so.
+ *
+ * The per-output-channel quantized linear
+ *
+ *     y[m,n] = s_w[n] * sum_k xhat[m,k] * q[n,k]
+ *
+ * in its weight-only (W8A16), static int8-activation (W8A8, one or two passes)
+ * and dynamic int8-activation x int4-group-weight (8da4w) forms, plus the
+ * quantizers that produce its operands.  Sources of each definition:
+ *
+ *   [ROCm-INT8]  code/quant/int8_linear.py (Ming-Image-0.1-Design ROCm INT8):
+ *                quantize_weight, QUANT_RULE, Int8Linear
+ *   [tiny-llm]   src/tinyllm/quant.py (tiny-llm): module docstring (the
+ *                factorisation identity), Int8Linear.forward
+ *   [SmolVLM-Q8] export/_smolvlm_q8.py (SmolVLM-500M-Instruct ExecuTorch WebGPU):
+ *                module docstring ("Two passes"), fake_quant, Q8Linear,
+ *                act_observer, fix_q8ta_fake (linear_q8ta_q8csw operands)
+ *   [ET-21229]   pytorch/executorch PR #21229 description: choose_qparams_affine
+ *                and linear_dq8ca_q4gsw (8da4w)
+ *
+ * Conventions shared by every call
+ *   - Pointers named as device pointers must be device memory of the current
+ *     CUDA device, owned by the caller (the library allocates nothing and keeps
+ *     no pointer after a call returns).  Host-only calls are marked.
+ *   - Tensors are row-major with the innermost dimension contiguous and
+ *     start on a 16-byte boundary (Q8_ERR_ALIGN otherwise).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Every device call only enqueues work on it and returns before
+ *     the work completes; nothing synchronises, nothing aborts.  Argument
+ *     errors are detected on the host before anything is enqueued and leave
+ *     all outputs untouched.
+ *   - Shapes: 0 <= M; 1 <= N; 16 <= K <= 65535 and K % 16 == 0 (int32
+ *     accumulators cannot overflow: 255 * 128 * 65535 < 2^31).  M == 0 is a
+ *     valid no-op.
+ *   - The device must be sm_100 (B200); other devices return
+ *     Q8_ERR_UNSUPPORTED_ARCH.  There is no CPU fallback.
+ *   - Calls that overlap on the GPU may share nothing they write.
+ */
+#ifndef Q8_H
+#define Q8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    Q8_OK = 0,
+    Q8_ERR_NULL = 1,              /* a required pointer is NULL                        */
+    Q8_ERR_SHAPE = 2,             /* a size is out of range (see conventions)          */
+    Q8_ERR_ALIGN = 3,             /* a pointer is not 16-byte aligned                  */
+    Q8_ERR_ARG = 4,               /* another argument is invalid (dtype, G, scale)     */
+    Q8_ERR_UNSUPPORTED_ARCH = 5,  /* the current device is not sm_100                  */
+    Q8_ERR_LAUNCH = 6,            /* a CUDA runtime / driver call failed               */
+    Q8_ERR_WORKSPACE = 7,         /* workspace NULL or smaller than q8_workspace_bytes */
+    Q8_ERR_DEVICE = 8             /* a kernel recorded a device-side failure           */
+} q8_status;
+
+typedef enum { Q8_F32 = 0, Q8_BF16 = 1 } q8_dtype;
+
+/* Static per-tensor affine activation parameters: real x ~ (code - zero_point) * scale,
+ * codes in [-128, 127].  scale must be finite and > 0; zero_point in [-128, 127]. */
+typedef struct {
+    float scale;
+    int32_t zero_point;
+} q8_qparams;
+
+/* Which call a workspace is sized for (q8_workspace_bytes). */
+typedef enum { Q8_OP_LINEAR_W8A8 = 0, Q8_OP_LINEAR_DQ8CA_Q4GSW = 1 } q8_op;
+
+/* Host.  Human-readable name of a status code (static string). */
+const char* q8_status_string(q8_status s);
+
+/* Host.  Library ABI version (major * 10000 + minor * 100 + patch). */
+int q8_version(void);
+
+/* ------------------------------------------------------------------ quantizers */
+
+/* Per-output-channel symmetric int8 weight codes.  [ROCm-INT8] quantize_weight and
+ * QUANT_RULE; [tiny-llm] module docstring.  For each row n of W:
+ *     s_w[n] = absmax(W[n,:]) / 127            (fp32 IEEE division)
+ *     q[n,k] = clamp(round(W[n,k] / s_w[n]), -127, 127)   (division, ties to even)
+ * and a row whose scale comes out 0 gets s_w[n] = 1.0 and all codes 0.
+ * wsum[n] = sum_k q[n,k] (the weight_sums operand of [SmolVLM-Q8]'s delegated
+ * linear_q8ta_q8csw), written when wsum != NULL.
+ *   W     device fp32 [N, K]  (read)
+ *   q     device int8 [N, K]  (written)
+ *   s_w   device fp32 [N]     (written)
+ *   wsum  device int32 [N]    (written; nullable)
+ * Codes and scales are bit-identical to the CPU reference definition. */
+q8_status q8_quantize_weight(const float* W, int64_t N, int64_t K,
+                             int8_t* q, float* s_w, int32_t* wsum, void* stream);
+
+/* Per-row asymmetric int8 activation parameters.  [ET-21229] choose_qparams_affine
+ * (formula of the per-tensor observer in [SmolVLM-Q8] act_observer), per row m:
+ *     mn = min(0, min_k x), mx = max(0, max_k x)
+ *     s[m] = max((mx - mn) / 255, FLT_EPSILON)      (fp32)
+ *     z[m] = clamp(-128 - round(mn / s[m]), -128, 127)
+ *     xq[m,k] = clamp(round(x[m,k] * (1 / s[m])) + z[m], -128, 127)   (if xq != NULL)
+ *   x     device bf16 [M, K] (read; xt must be Q8_BF16)
+ *   s     device fp32 [M], z device int32 [M], xq device int8 [M, K] (nullable)
+ * Bit-identical to the CPU reference definition. */
+q8_status q8_choose_qparams(const void* x, q8_dtype xt, int64_t M, int64_t K,
+                            float* s, int32_t* z, int8_t* xq, void* stream);
+
+/* Static per-tensor activation codes ([SmolVLM-Q8] Q8Linear.forward, fake_quant):
+ *     xq1 = clamp(round(x * (1/s1)) + z1, -128, 127)
+ * and, when second != NULL, the two-pass residual codes
+ *     r   = x - (xq1 - z1) * s1      (each step rounded to fp32)
+ *     xq2 = clamp(round(r * (1/s2)) + z2, -128, 127).
+ *   x device fp32 [M, K]; xq1 device int8 [M, K]; xq2 device int8 [M, K] (required
+ *   iff second != NULL).  `first` / `*second` are read on the host.
+ * This is the activation step q8_linear_w8a8 runs; exported for parity tests and
+ * for callers that keep codes. */
+q8_status q8_quantize_static(const float* x, int64_t M, int64_t K, q8_qparams first,
+                             const q8_qparams* second, int8_t* xq1, int8_t* xq2,
+                             void* stream);
+
+/* Per-tensor observer statistics ([SmolVLM-Q8] act_observer / MinMaxObserver: min and
+ * max of everything observed).  minmax is a device fp32 [2] = {min, max}; with
+ * reset != 0 it is first set to {+inf, -inf}; then it is lowered / raised by the
+ * n values of x (device fp32).  n == 0 with reset == 0 is a no-op. */
+q8_status q8_observe_minmax(const float* x, int64_t n, float* minmax, int reset,
+                            void* stream);
+
+/* Host.  Per-tensor affine qparams from an observed range (same formula as
+ * q8_choose_qparams): out->scale = max((max(mx,0) - min(mn,0)) / 255, FLT_EPSILON),
+ * out->zero_point = clamp(-128 - round(min(mn,0) / scale), -128, 127).
+ * Q8_ERR_ARG if mn or mx is not finite or mn > mx. */
+q8_status q8_qparams_from_minmax(float mn, float mx, q8_qparams* out);
+
+/* int4 group-symmetric weight codes for the 8da4w linear ([ET-21229] names the
+ * "q4gsw" weight; its grid is not printed there, so the int8 rule above is used per
+ * group): for each row n and group g of G consecutive k,
+ *     gs[n,g] = absmax(W[n, gG:(g+1)G]) / 7        (fp32)
+ *     code    = clamp(round(W / gs[n,g]), -7, 7)   (a zero-scale group: gs = 1, codes 0)
+ * packed two per byte: byte k/2 of row n holds code k in its low nibble (k even)
+ * or its high nibble (k odd).
+ *   W device fp32 [N, K]; q4 device uint8 [N, K/2]; gs device fp32 [N, K/G].
+ *   G in {32, 64, 128, 256} and K % G == 0. */
+q8_status q8_quantize_weight_q4gs(const float* W, int64_t N, int64_t K, int G,
+                                  uint8_t* q4, float* gs, void* stream);
+
+/* -------------------------------------------------------------------- linears */
+
+/* W8A16: bf16 activations times int8 weights, the scale applied after the sum
+ * ([tiny-llm] factorisation identity y_j = s_j sum_i x_i q_ji; Int8Linear.forward):
+ *     y[m,n] = s_w[n] * sum_k x[m,k] * q[n,k]      (fp32 accumulation, one rounding to yt)
+ *   x device bf16 [M, K]; q device int8 [N, K]; s_w device fp32 [N];
+ *   y device [M, N] of type yt (Q8_BF16 or Q8_F32).
+ * Decode-sized M (1..16) runs as an HBM-streaming GEMV on the tensor cores; larger M
+ * is computed in blocks of 16 rows (correct, not tuned for prefill). */
+q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w,
+                          void* y, q8_dtype yt, int64_t M, int64_t N, int64_t K,
+                          void* stream);
+
+/* W8A8: static per-tensor int8 activations times per-channel int8 weights
+ * ([SmolVLM-Q8] Q8Linear.forward; the delegated op takes weight_sums):
+ *     acc1[m,n] = sum_k xq1[m,k] q[n,k]     (int32, exact)
+ *     y[m,n]    = s_w[n] * s1 * (acc1 - z1 * wsum[n])
+ * and with second != NULL (two-pass residual, same int8 weight, module docstring):
+ *     y[m,n]   += s_w[n] * s2 * (acc2 - z2 * wsum[n]),  acc2 = sum_k xq2 q
+ * with xq1 / xq2 the codes of q8_quantize_static.  fp32 epilogue.
+ *   x device fp32 [M, K]; q device int8 [N, K]; wsum device int32 [N] (as written by
+ *   q8_quantize_weight); s_w device fp32 [N]; y device fp32 [M, N].
+ *   workspace: device scratch of at least q8_workspace_bytes(Q8_OP_LINEAR_W8A8, M, N,
+ *   K, second != NULL) bytes (may be NULL when that is 0); its contents on entry do not
+ *   matter and are overwritten.
+ * Decode-sized M runs as a GEMV with the activation codes computed in-kernel; larger M
+ * quantizes x into the workspace and runs a tcgen05 int8 GEMM (int32 accumulators in
+ * tensor memory) with the zero-point term and both scales in its epilogue. */
+q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* second,
+                         const int8_t* q, const int32_t* wsum, const float* s_w,
+                         float* y, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/* 8da4w: dynamic per-row int8 activations folded into the 4-bit group-symmetric
+ * weight GEMM ([ET-21229] linear_dq8ca_q4gsw):
+ *     (s, z, xq) = q8_choose_qparams(x)
+ *     y[m,n] = s[m] * sum_g gs[n,g] * sum_{k in g} (xq[m,k] - z[m]) * q4[n,k]
+ * with per-group int32 partial sums and fp32 accumulation across groups.
+ *   x device bf16 [M, K]; q4 device uint8 [N, K/2]; gs device fp32 [N, K/G];
+ *   y device fp32 [M, N]; G in {32, 64, 128, 256}, K % G == 0.
+ *   workspace: at least q8_workspace_bytes(Q8_OP_LINEAR_DQ8CA_Q4GSW, M, N, K, G). */
+q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* gs, int G,
+                                float* y, int64_t M, int64_t N, int64_t K,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Host.  Workspace bytes a linear needs for these sizes (0 if none).  `extra` is
+ * "two-pass" (0/1) for Q8_OP_LINEAR_W8A8 and G for Q8_OP_LINEAR_DQ8CA_Q4GSW.
+ * Returns 0 for invalid arguments as well; the linear then reports the error. */
+size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra);
+
+/* Integer GEMM with int32 output, acc[m,n] = sum_k a[m,k] * b[n,k] (exact): the
+ * tcgen05 int8 MMA path of q8_linear_w8a8 without its epilogue, exported so that the
+ * int32 accumulators can be checked bit for bit.
+ *   a device int8 [M, K]; b device int8 [N, K]; acc device int32 [M, N]. */
+q8_status q8_gemm_s8s8_s32(const int8_t* a, const int8_t* b, int32_t* acc,
+                           int64_t M, int64_t N, int64_t K, void* stream);
+
+/* Host, synchronising.  Reads and clears the device status word that kernels with
+ * bounded waits set when a wait expires (Q8_OK if none did since the last read).
+ * Waits for the given stream first. */
+q8_status q8_last_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* Q8_H */

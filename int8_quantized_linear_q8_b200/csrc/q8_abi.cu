@@ -1,0 +1,286 @@
+// q8_abi.cu -- the C ABI (include/q8.h): argument checks on the host, then kernel
+// launches on the caller's stream.  Nothing here allocates device memory, synchronises
+// (except q8_last_device_status, documented as synchronising) or aborts.
+#include "q8_kernels.cuh"
+
+#include <float.h>
+#include <math.h>
+#include <mutex>
+
+namespace q8 {
+
+// Status word that kernels with bounded waits set when a wait expires (0 = none).
+// Kernels receive its device address as an argument (kernels live in other files).
+__device__ int g_device_status;
+
+static q8_status read_and_clear_device_status() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    if (v == 0) return Q8_OK;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    return Q8_ERR_DEVICE;
+}
+
+// ------------------------------------------------------------------- device checks
+struct DevInfo {
+    int checked = 0;
+    int ok = 0;
+    int num_sms = 0;
+};
+static DevInfo g_dev[128];
+static std::mutex g_dev_mu;
+
+static q8_status current_device(int& num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    if (dev < 0 || dev >= 128) return Q8_ERR_UNSUPPORTED_ARCH;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DevInfo& d = g_dev[dev];
+    if (!d.checked) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return Q8_ERR_LAUNCH;
+        }
+        d.ok = (major == 10 && minor == 0);
+        d.num_sms = sms;
+        d.checked = 1;
+    }
+    num_sms = d.num_sms;
+    return d.ok ? Q8_OK : Q8_ERR_UNSUPPORTED_ARCH;
+}
+
+static inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static inline q8_status check_k(int64_t K) {
+    if (K < 16 || K > 65535 || (K % 16) != 0) return Q8_ERR_SHAPE;
+    return Q8_OK;
+}
+
+static inline q8_status check_qparams(const q8_qparams& p) {
+    if (!(p.scale > 0.0f) || !isfinite(p.scale)) return Q8_ERR_ARG;
+    if (p.zero_point < -128 || p.zero_point > 127) return Q8_ERR_ARG;
+    return Q8_OK;
+}
+
+static inline q8_status launched(cudaError_t e) {
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    return Q8_OK;
+}
+
+#define Q8_TRY(expr)                      \
+    do {                                  \
+        q8_status _s = (expr);            \
+        if (_s != Q8_OK) return _s;       \
+    } while (0)
+
+static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace plans (byte offsets inside the caller's workspace).
+struct W8A8Plan {
+    size_t xq1 = 0, xq2 = 0, bytes = 0;
+};
+static W8A8Plan plan_w8a8(int64_t M, int64_t K, int two) {
+    W8A8Plan p;
+    const size_t codes = align_up((size_t)M * (size_t)K, 256);
+    p.xq1 = 0;
+    p.xq2 = two ? codes : 0;
+    p.bytes = M > 0 ? codes * (two ? 2 : 1) : 0;
+    return p;
+}
+
+}  // namespace q8
+
+using namespace q8;
+
+extern "C" {
+
+const char* q8_status_string(q8_status s) {
+    switch (s) {
+        case Q8_OK: return "ok";
+        case Q8_ERR_NULL: return "a required pointer is NULL";
+        case Q8_ERR_SHAPE: return "a size is out of range";
+        case Q8_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case Q8_ERR_ARG: return "invalid argument";
+        case Q8_ERR_UNSUPPORTED_ARCH: return "the current device is not sm_100 (B200)";
+        case Q8_ERR_LAUNCH: return "a CUDA call failed";
+        case Q8_ERR_WORKSPACE: return "workspace missing or too small";
+        case Q8_ERR_DEVICE: return "a kernel recorded a device-side failure";
+    }
+    return "unknown status";
+}
+
+int q8_version(void) { return 100; }
+
+q8_status q8_quantize_weight(const float* W, int64_t N, int64_t K, int8_t* q, float* s_w,
+                             int32_t* wsum, void* stream) {
+    if (!W || !q || !s_w) return Q8_ERR_NULL;
+    if (N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (!aligned16(W) || !aligned16(q)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_quantize_weight(W, N, (int)K, q, s_w, wsum, (cudaStream_t)stream));
+}
+
+q8_status q8_choose_qparams(const void* x, q8_dtype xt, int64_t M, int64_t K, float* s,
+                            int32_t* z, int8_t* xq, void* stream) {
+    if (xt != Q8_BF16) return Q8_ERR_ARG;
+    if (M < 0 || M > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (M == 0) return Q8_OK;
+    if (!x || !s || !z) return Q8_ERR_NULL;
+    if (!aligned16(x) || (xq && !aligned16(xq))) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_choose_qparams((const uint16_t*)x, M, (int)K, s, z, xq,
+                                          (cudaStream_t)stream));
+}
+
+q8_status q8_quantize_static(const float* x, int64_t M, int64_t K, q8_qparams first,
+                             const q8_qparams* second, int8_t* xq1, int8_t* xq2, void* stream) {
+    if (M < 0) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    Q8_TRY(check_qparams(first));
+    if (second) Q8_TRY(check_qparams(*second));
+    if (M == 0) return Q8_OK;
+    if (!x || !xq1 || (second && !xq2)) return Q8_ERR_NULL;
+    if (!aligned16(x) || !aligned16(xq1) || (second && !aligned16(xq2))) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_quantize_static(x, M, (int)K, first.scale, first.zero_point,
+                                           second != nullptr, second ? second->scale : 1.0f,
+                                           second ? second->zero_point : 0, xq1, xq2,
+                                           (cudaStream_t)stream, sms));
+}
+
+q8_status q8_observe_minmax(const float* x, int64_t n, float* minmax, int reset, void* stream) {
+    if (n < 0) return Q8_ERR_SHAPE;
+    if (!minmax || (n > 0 && !x)) return Q8_ERR_NULL;
+    if (n == 0 && !reset) return Q8_OK;
+    if (x && !aligned16(x)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_observe_minmax(x, n, minmax, reset, (cudaStream_t)stream, sms));
+}
+
+q8_status q8_qparams_from_minmax(float mn, float mx, q8_qparams* out) {
+    if (!out) return Q8_ERR_NULL;
+    if (!isfinite(mn) || !isfinite(mx) || mn > mx) return Q8_ERR_ARG;
+    // Same formula as the device's per-row rule; plain IEEE fp32 host arithmetic.
+    volatile float lo = mn < 0.0f ? mn : 0.0f;
+    volatile float hi = mx > 0.0f ? mx : 0.0f;
+    volatile float range = hi - lo;
+    volatile float s = range / 255.0f;
+    if (s < FLT_EPSILON) s = FLT_EPSILON;
+    volatile float ratio = lo / s;
+    float zf = -128.0f - nearbyintf(ratio);
+    if (zf < -128.0f) zf = -128.0f;
+    if (zf > 127.0f) zf = 127.0f;
+    out->scale = s;
+    out->zero_point = (int32_t)zf;
+    return Q8_OK;
+}
+
+q8_status q8_quantize_weight_q4gs(const float* W, int64_t N, int64_t K, int G, uint8_t* q4,
+                                  float* gs, void* stream) {
+    if (!W || !q4 || !gs) return Q8_ERR_NULL;
+    if (G != 32 && G != 64 && G != 128 && G != 256) return Q8_ERR_ARG;
+    if (N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (K % G) return Q8_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(q4) || !aligned16(gs)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_quantize_weight_q4gs(W, N, (int)K, G, q4, gs, (cudaStream_t)stream));
+}
+
+q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w, void* y,
+                          q8_dtype yt, int64_t M, int64_t N, int64_t K, void* stream) {
+    if (yt != Q8_F32 && yt != Q8_BF16) return Q8_ERR_ARG;
+    if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (M == 0) return Q8_OK;
+    if (!x || !q || !s_w || !y) return Q8_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_w8a16_gemv((const uint16_t*)x, q, s_w, y, yt == Q8_BF16, M, N, (int)K,
+                                      (cudaStream_t)stream, sms));
+}
+
+size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) {
+    if (M < 0 || N < 1 || check_k(K) != Q8_OK) return 0;
+    switch (op) {
+        case Q8_OP_LINEAR_W8A8: return plan_w8a8(M, K, extra != 0).bytes;
+        case Q8_OP_LINEAR_DQ8CA_Q4GSW: return 0;
+    }
+    return 0;
+}
+
+q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* second,
+                         const int8_t* q, const int32_t* wsum, const float* s_w, float* y,
+                         int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes,
+                         void* stream) {
+    if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    Q8_TRY(check_qparams(first));
+    if (second) Q8_TRY(check_qparams(*second));
+    if (M == 0) return Q8_OK;
+    if (!x || !q || !wsum || !s_w || !y) return Q8_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q)) return Q8_ERR_ALIGN;
+    const int two = second != nullptr;
+    const W8A8Plan plan = plan_w8a8(M, K, two);
+    if (plan.bytes > 0 && (!workspace || ws_bytes < plan.bytes)) return Q8_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    cudaStream_t st = (cudaStream_t)stream;
+    int8_t* xq1 = (int8_t*)workspace + plan.xq1;
+    int8_t* xq2 = two ? (int8_t*)workspace + plan.xq2 : nullptr;
+    const float s2 = two ? second->scale : 1.0f;
+    const int z2 = two ? second->zero_point : 0;
+    Q8_TRY(launched(launch_quantize_static(x, M, (int)K, first.scale, first.zero_point, two, s2,
+                                           z2, xq1, xq2, st, sms)));
+    return launched(launch_w8a8_gemv_codes(xq1, xq2, first.scale, first.zero_point, two, s2, z2,
+                                           q, wsum, s_w, y, M, N, (int)K, st));
+}
+
+q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* gs, int G,
+                                float* y, int64_t M, int64_t N, int64_t K, void* workspace,
+                                size_t ws_bytes, void* stream) {
+    (void)x; (void)q4; (void)gs; (void)G; (void)y; (void)M; (void)N; (void)K;
+    (void)workspace; (void)ws_bytes; (void)stream;
+    return Q8_ERR_ARG;
+}
+
+q8_status q8_gemm_s8s8_s32(const int8_t* a, const int8_t* b, int32_t* acc, int64_t M, int64_t N,
+                           int64_t K, void* stream) {
+    (void)a; (void)b; (void)acc; (void)M; (void)N; (void)K; (void)stream;
+    return Q8_ERR_ARG;
+}
+
+q8_status q8_last_device_status(void* stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    return read_and_clear_device_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// q8_kernels.cuh -- launcher declarations and device code shared between kernel files.
+#pragma once
+
+#include "q8_common.cuh"
+
+namespace q8 {
+
+// Sixteen static activation codes (first pass, and the two-pass residual's codes):
+//   c1 = clamp(round(v * (1/s1)) + z1, -128, 127)
+//   r  = v - (c1 - z1) * s1          (fp32 product, then fp32 difference; no FMA)
+//   c2 = clamp(round(r * (1/s2)) + z2, -128, 127)
+// packed four codes per word, lowest k in the lowest byte.
+__device__ __forceinline__ void static_codes16(const float (&v)[16], float s1, float inv1,
+                                               float z1f, int has2, float inv2, float z2f,
+                                               uint32_t (&o1)[4], uint32_t (&o2)[4]) {
+    int c1[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) c1[j] = act_code(v[j], inv1, z1f);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        o1[j] = pack4_s8(c1[4 * j], c1[4 * j + 1], c1[4 * j + 2], c1[4 * j + 3]);
+    if (has2) {
+        int c2[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float d1 = __fmul_rn(__fsub_rn((float)c1[j], z1f), s1);
+            float r = __fsub_rn(v[j], d1);
+            c2[j] = act_code(r, inv2, z2f);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            o2[j] = pack4_s8(c2[4 * j], c2[4 * j + 1], c2[4 * j + 2], c2[4 * j + 3]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o2[j] = 0u;
+    }
+}
+
+// k_quant.cu
+cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int8_t* q, float* s_w,
+                                   int32_t* wsum, cudaStream_t st);
+cudaError_t launch_choose_qparams(const uint16_t* x, int64_t M, int K, float* s, int32_t* z,
+                                  int8_t* xq, cudaStream_t st);
+cudaError_t launch_quantize_static(const float* x, int64_t M, int K, float s1, int z1, int has2,
+                                   float s2, int z2, int8_t* xq1, int8_t* xq2, cudaStream_t st,
+                                   int num_sms);
+cudaError_t launch_observe_minmax(const float* x, int64_t n, float* mm, int reset,
+                                  cudaStream_t st, int num_sms);
+cudaError_t launch_quantize_weight_q4gs(const float* W, int64_t N, int K, int G, uint8_t* q4,
+                                        float* gs, cudaStream_t st);
+
+// k_gemv.cu
+cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
+                              int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,
+                              int num_sms);
+cudaError_t launch_w8a8_gemv_codes(const int8_t* xq1, const int8_t* xq2, float s1, int z1,
+                                   int has2, float s2, int z2, const int8_t* q,
+                                   const int32_t* wsum, const float* s_w, float* y, int64_t M,
+                                   int64_t N, int K, cudaStream_t st);
+
+}  // namespace q8

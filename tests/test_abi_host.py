@@ -1,0 +1,107 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every entry
+point that include/q8.h declares, validates arguments before touching the device, and
+fails loudly (never computes on the CPU) when no sm_100 device is present."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import int8_quantized_linear_q8_b200 as q8
+import oracle
+from int8_quantized_linear_q8_b200 import build as q8build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    q8build.build()
+    return q8.lib()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "q8.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(q8_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declarations_are_exported(L):
+    declared = _declared()
+    assert len(declared) >= 14
+    for name in declared:
+        assert hasattr(L, name), f"{name} declared in include/q8.h but not exported"
+    assert sorted(q8.SYMBOLS) == declared
+
+
+def test_status_strings(L):
+    for code in range(9):
+        assert L.q8_status_string(code)
+    assert L.q8_version() >= 100
+
+
+def test_qparams_from_minmax_host_matches_oracle(L):
+    """The host formula is bit-identical to the oracle's on many ranges."""
+    rng = np.random.default_rng(3)
+    cases = [(-1.0, 3.0), (1.0, 4.0), (-4.0, -1.0), (0.0, 0.0), (-1e-9, 1e-9), (-3000.0, 4.0)]
+    cases += [tuple(sorted(rng.normal(0, 10, 2).astype(np.float32).tolist())) for _ in range(500)]
+    for mn, mx in cases:
+        assert q8.q8_qparams_from_minmax(mn, mx) == oracle.qparams_from_minmax(mn, mx), (mn, mx)
+
+
+def test_qparams_from_minmax_rejects(L):
+    out = q8.q8_qparams()
+    assert L.q8_qparams_from_minmax(1.0, -1.0, ctypes.byref(out)) == q8.Q8_ERR_ARG
+    assert L.q8_qparams_from_minmax(float("nan"), 1.0, ctypes.byref(out)) == q8.Q8_ERR_ARG
+    assert L.q8_qparams_from_minmax(0.0, 1.0, None) == q8.Q8_ERR_NULL
+
+
+def test_workspace_sizes(L):
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 0, 16, 64) == 0
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 4, 16, 64, 0) >= 4 * 64
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 4, 16, 64, 1) >= 2 * 4 * 64
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 4, 16, 63) == 0      # invalid K
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_argument_validation_before_device(L):
+    """Errors are reported from the arguments alone (no device needed)."""
+    good = _p(0x10000)      # never dereferenced: every call below fails validation first
+    odd = _p(0x10001)
+    qp = q8.q8_qparams(0.1, 0)
+    assert L.q8_quantize_weight(None, 4, 64, good, good, None, None) == q8.Q8_ERR_NULL
+    assert L.q8_quantize_weight(good, 4, 60, good, good, None, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_quantize_weight(good, 4, 65536 + 16, good, good, None, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_quantize_weight(good, 0, 64, good, good, None, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_quantize_weight(odd, 4, 64, good, good, None, None) == q8.Q8_ERR_ALIGN
+    assert L.q8_choose_qparams(good, q8.Q8_F32, 4, 64, good, good, None, None) == q8.Q8_ERR_ARG
+    assert L.q8_choose_qparams(good, q8.Q8_BF16, 0, 64, None, None, None, None) == q8.Q8_OK
+    assert L.q8_linear_w8a16(good, good, good, good, 7, 1, 16, 64, None) == q8.Q8_ERR_ARG
+    assert L.q8_linear_w8a16(good, good, good, good, q8.Q8_BF16, 1, 16, 40, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_linear_w8a16(good, good, good, good, q8.Q8_BF16, 0, 16, 64, None) == q8.Q8_OK
+    bad_qp = q8.q8_qparams(0.0, 0)
+    assert L.q8_linear_w8a8(good, bad_qp, None, good, good, good, good, 1, 16, 64, good, 1024,
+                            None) == q8.Q8_ERR_ARG
+    assert L.q8_linear_w8a8(good, q8.q8_qparams(0.1, 200), None, good, good, good, good, 1, 16,
+                            64, good, 1024, None) == q8.Q8_ERR_ARG
+    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 4, 16, 64, None, 0,
+                            None) == q8.Q8_ERR_WORKSPACE
+    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 4, 16, 64, good, 10,
+                            None) == q8.Q8_ERR_WORKSPACE
+    assert L.q8_quantize_weight_q4gs(good, 4, 64, 48, good, good, None) == q8.Q8_ERR_ARG
+    assert L.q8_quantize_weight_q4gs(good, 4, 96, 64, good, good, None) == q8.Q8_ERR_SHAPE
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU failure mode")
+def test_valid_call_without_gpu_fails_loudly(L):
+    good = _p(0x10000)
+    st = L.q8_quantize_weight(good, 4, 64, good, good, None, None)
+    assert st in (q8.Q8_ERR_LAUNCH, q8.Q8_ERR_UNSUPPORTED_ARCH)
+    with pytest.raises((q8.Q8Error, ValueError, RuntimeError)):
+        q8.q8_linear_w8a16(torch.zeros(1, 64, dtype=torch.bfloat16),
+                           torch.zeros(16, 64, dtype=torch.int8), torch.ones(16))

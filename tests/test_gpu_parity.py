@@ -1,0 +1,209 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the CPU oracle on the same
+seeded inputs.  Integer stages (codes, scales, zero points, code sums) must be bit-exact;
+float outputs within the tolerances in tests/tolerance.py."""
+import numpy as np
+import pytest
+import torch
+
+import int8_quantized_linear_q8_b200 as q8
+import oracle
+import q8_workloads as wl
+from int8_quantized_linear_q8_b200 import build as q8build
+from tolerance import check_bf16, check_f32
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    q8build.build()
+    q8.lib()
+    yield
+    assert q8.q8_last_device_status() == q8.Q8_OK
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ------------------------------------------------------------------- weight codes (a1)
+
+
+@pytest.mark.parametrize("N,K,zero_rows", [(256, 512, (7,)), (2560, 960, ()), (33, 16, (0, 32)),
+                                           (11008, 4096, (5,)), (32000, 4096, ())])
+def test_quantize_weight_bit_exact(N, K, zero_rows):
+    W = wl.weight(N, K, seed=100 + N % 97, zero_rows=zero_rows)
+    if N == 33:
+        W[3] *= 1e-30
+        W[4, :] = 0.0
+        W[4, 5] = -2.5
+    q, s, ws = q8.q8_quantize_weight(W.to(DEV))
+    rq, rs, rws = oracle.quantize_weight(W.numpy())
+    assert np.array_equal(q.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(ws.cpu().numpy(), rws)
+
+
+def test_quantize_weight_pr1_zero_row():
+    cfg = wl.PR1
+    W = wl.weight(cfg["N"], cfg["K"], seed=cfg["seed"], zero_rows=cfg["zero_rows"])
+    q, s, ws = q8.q8_quantize_weight(W.to(DEV))
+    assert s[7].item() == 1.0 and not q[7].any().item() and ws[7].item() == 0
+
+
+# ------------------------------------------------------------ activation qparams (a2)
+
+
+def _edge_rows(K):
+    x = wl.normal((8, K), 1.0, seed=200)
+    x[1] = 0.0
+    x[2] = x[2].abs()
+    x[3] = -x[3].abs()
+    x[4] *= 1e4
+    x[5] *= 1e-30
+    x[6, :] = 0.0
+    x[6, 3] = 5.0
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("M,K", [(1, 4096), (64, 4096), (512, 4096), (4096, 4096), (3, 16),
+                                 (8, 48)])
+def test_choose_qparams_bit_exact(M, K):
+    x = wl.normal_bf16((M, K), 1.0, seed=201 + M)
+    if M >= 8:
+        x[:8] = _edge_rows(K)
+    s, z, xq = q8.q8_choose_qparams(x.to(DEV))
+    rs, rz, rxq = oracle.choose_qparams(wl.bf16_bits(x))
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(z.cpu().numpy(), rz)
+    assert np.array_equal(xq.cpu().numpy(), rxq)
+
+
+def test_choose_qparams_without_codes():
+    x = wl.normal_bf16((5, 64), 2.0, seed=202)
+    s, z, xq = q8.q8_choose_qparams(x.to(DEV), want_codes=False)
+    rs, rz, _ = oracle.choose_qparams(wl.bf16_bits(x), want_codes=False)
+    assert xq is None
+    assert np.array_equal(s.cpu().numpy(), rs) and np.array_equal(z.cpu().numpy(), rz)
+
+
+# --------------------------------------------------------- static activation codes (a3)
+
+
+def _w8a8_qparams(K):
+    x, calib = wl.w8a8_inputs(1, K=K)
+    mm = torch.empty(2, device=DEV)
+    q8.q8_observe_minmax(calib.to(DEV), mm, reset=True)
+    mn, mx = mm.cpu().tolist()
+    assert (mn, mx) == oracle.minmax(calib.numpy())
+    first = q8.q8_qparams_from_minmax(mn, mx)
+    assert first == oracle.qparams_from_minmax(mn, mx)
+    second = (float(np.float32(first[0]) / np.float32(255.0)), 0)
+    return first, second
+
+
+@pytest.mark.parametrize("M,K", [(1, 960), (256, 960), (2048, 960), (7, 4096), (4096, 16)])
+@pytest.mark.parametrize("two", [False, True])
+def test_quantize_static_bit_exact(M, K, two):
+    first, second = _w8a8_qparams(K)
+    x, _ = wl.w8a8_inputs(M, K=K)
+    x[0, :4] = torch.tensor([1e30, -1e30, 0.0, -0.0])       # saturation and signed zero
+    xq1, xq2 = q8.q8_quantize_static(x.to(DEV), first, second if two else None)
+    r1, r2 = oracle.static_quant(x.numpy(), first, second if two else None)
+    assert np.array_equal(xq1.cpu().numpy(), r1)
+    if two:
+        assert np.array_equal(xq2.cpu().numpy(), r2)
+
+
+def test_observe_minmax_accumulates():
+    a = wl.normal((1000,), 1.0, seed=203)
+    b = wl.normal((77,), 5.0, seed=204)
+    mm = torch.empty(2, device=DEV)
+    q8.q8_observe_minmax(a.to(DEV), mm, reset=True)
+    q8.q8_observe_minmax(b.to(DEV), mm)
+    both = torch.cat([a, b]).numpy()
+    assert mm.cpu().tolist() == [float(both.min()), float(both.max())]
+
+
+# -------------------------------------------------------------- int4 group codes
+
+
+@pytest.mark.parametrize("N,K,G", [(11008, 4096, 32), (11008, 4096, 128), (19, 256, 64),
+                                   (7, 512, 256)])
+def test_quantize_weight_q4gs_bit_exact(N, K, G):
+    W = wl.weight(N, K, seed=300 + G)
+    W[0, :G] = 0.0                                          # a zero group
+    q4, gs = q8.q8_quantize_weight_q4gs(W.to(DEV), G)
+    rq4, rgs = oracle.quantize_weight_q4gs(W.numpy(), G)
+    assert np.array_equal(q4.cpu().numpy(), rq4)
+    assert np.array_equal(gs.cpu().numpy().view(np.uint32), rgs.view(np.uint32))
+
+
+# ---------------------------------------------------------------------- W8A16 (a4)
+
+
+def _w8a16_case(M, N, K, seed_w, seed_x, out_dtype, zero_rows=()):
+    W = wl.weight(N, K, seed=seed_w, zero_rows=zero_rows)
+    x = wl.normal_bf16((M, K), 1.0, seed=seed_x)
+    q, s, _ = q8.q8_quantize_weight(W.to(DEV), want_wsum=False)
+    y = q8.q8_linear_w8a16(x.to(DEV), q, s, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    rq, rs, _ = oracle.quantize_weight(W.numpy())
+    y64, absum = oracle.linear_w8a16(wl.bf16_bits(x), rq, rs)
+    return y, y64, absum
+
+
+def test_w8a16_pr1_fp32():
+    c = wl.PR1
+    y, y64, absum = _w8a16_case(c["M"], c["N"], c["K"], c["seed"], c["seed"] + 1000,
+                                torch.float32, zero_rows=c["zero_rows"])
+    check_f32(y.cpu().numpy(), y64, absum, "PR1")
+    assert (y[:, 7] == 0).all()
+
+
+@pytest.mark.parametrize("shape", wl.W8A16_SWEEP_SHAPES, ids=lambda s: f"K{s.K}xN{s.N}")
+@pytest.mark.parametrize("M", wl.W8A16_SWEEP_M)
+def test_w8a16_sweep_bf16(shape, M):
+    y, y64, absum = _w8a16_case(M, shape.N, shape.K, wl.W8A16_SWEEP_SEED_W,
+                                wl.W8A16_SWEEP_SEED_X, torch.bfloat16)
+    check_bf16(_bits(y), y64, absum, f"W8A16 M={M} K={shape.K} N={shape.N}")
+
+
+@pytest.mark.parametrize("M,N,K", [(3, 17, 16), (9, 40, 48), (16, 1, 64), (17, 33, 80),
+                                   (40, 130, 1040), (5, 2049, 2000)])
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
+def test_w8a16_ragged(M, N, K, out):
+    y, y64, absum = _w8a16_case(M, N, K, 400 + N, 401 + M, out)
+    if out == torch.float32:
+        check_f32(y.cpu().numpy(), y64, absum, "ragged")
+    else:
+        check_bf16(_bits(y), y64, absum, "ragged")
+
+
+def test_w8a16_empty_m():
+    q = torch.zeros(16, 64, dtype=torch.int8, device=DEV)
+    s = torch.ones(16, device=DEV)
+    y = q8.q8_linear_w8a16(torch.zeros(0, 64, dtype=torch.bfloat16, device=DEV), q, s)
+    assert y.shape == (0, 16)
+
+
+# ----------------------------------------------------------------------- W8A8 (a5/a6)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 37])
+@pytest.mark.parametrize("N", wl.W8A8_N)
+@pytest.mark.parametrize("two", [False, True])
+def test_w8a8_small_m(M, N, two):
+    K = wl.W8A8_K
+    first, second = _w8a8_qparams(K)
+    x, _ = wl.w8a8_inputs(M, K=K)
+    W = wl.weight(N, K, seed=wl.W8A8_SEED_W)
+    q, s, ws = q8.q8_quantize_weight(W.to(DEV))
+    y = q8.q8_linear_w8a8(x.to(DEV), first, q, ws, s, second=second if two else None)
+    torch.cuda.synchronize()
+    rq, rs, _ = oracle.quantize_weight(W.numpy())
+    y64, absum, _, _ = oracle.linear_w8a8(x.numpy(), first, rq, rs,
+                                          second=second if two else None)
+    check_f32(y.cpu().numpy(), y64, absum, f"W8A8 M={M} N={N} two={two}")
