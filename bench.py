@@ -52,6 +52,12 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-paths", action="store_true", help="skip the sub-benchmarks")
+    p.add_argument("--profile", choices=["w8a16", "w8a8"], default=None,
+                   help="run only one kernel case --reps times (for ncu captures), then exit")
+    p.add_argument("--pM", type=int, default=16)
+    p.add_argument("--pN", type=int, default=32000)
+    p.add_argument("--pK", type=int, default=4096)
+    p.add_argument("--reps", type=int, default=3)
     return p.parse_args()
 
 
@@ -251,7 +257,7 @@ def time_graphs(graphs, steps: int, warmup: int, dist: Dist):
     return dist.max(ms), t0, t1
 
 
-def per_case_times(sweep: W8A16Sweep, reps: int = 50):
+def per_case_times(sweep: W8A16Sweep, reps: int = 20):
     """Average device time of each case's kernel, alone, from a graph of `reps` launches
     alternating weight copies (events on the launching stream)."""
     out = []
@@ -269,11 +275,11 @@ def per_case_times(sweep: W8A16Sweep, reps: int = 50):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for _ in range(3):
+        for _ in range(2):
             gr.replay()
         e1.record()
         torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1000.0 / (3 * reps)
+        us = e0.elapsed_time(e1) * 1000.0 / (2 * reps)
         sh = sweep.shapes[i][0]
         b = w8a16_bytes(M, sh.N, sh.K)
         out.append({"K": sh.K, "N": sh.N, "M": M, "us": round(us, 3),
@@ -501,8 +507,36 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_profile(args):
+    """One kernel case, launched --reps times on fresh data (ncu capture target)."""
+    import int8_quantized_linear_q8_b200 as q8
+
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    M, N, K = args.pM, args.pN, args.pK
+    W = torch.randn(N, K, generator=g, device=dev) * 0.02
+    q, s, ws = q8.q8_quantize_weight(W)
+    del W
+    if args.profile == "w8a16":
+        x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        for _ in range(args.reps):
+            q8.q8_linear_w8a16(x, q, s, y=y)
+    else:
+        x = torch.randn(M, K, generator=g, device=dev) * 4
+        y = torch.empty(M, N, device=dev)
+        for _ in range(args.reps):
+            q8.q8_linear_w8a8(x, (0.05, 3), q, ws, s, second=(0.05 / 255, 0), y=y)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "M": M, "N": N, "K": K, "reps": args.reps}))
+
+
 def main():
     args = parse_args()
+    if args.profile:
+        run_profile(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -1,0 +1,396 @@
+// k_gemv_tma.cu -- the decode-sized W8A16 linear as a persistent, TMA-fed HBM stream.
+//
+//   y[m, n] = s_w[n] * sum_k x[m, k] * q[n, k]      (M <= 16 activation rows)
+//
+// The int8 weight q[N, K] is the only large operand: the kernel exists to move it from
+// HBM at full bandwidth and to spend as few instructions as possible per byte.
+//
+// Structure (one CTA per SM, persistent over 16-row groups of q):
+//   * warp 8 (producer): one lane streams the CTA's rows through a ring of shared-memory
+//     stages with 2-D TMA copies.  A stage holds 16 rows x 1024 bytes of K, as 4 boxes of
+//     [16 rows][256 bytes] (boxes 64 bytes wide stream at about half the rate); stage
+//     readiness is an mbarrier with transaction bytes, stage release an mbarrier the
+//     consumer warps arrive on.
+//   * warps 0-7 (consumers): before the first stage they copy the activations x [M, K]
+//     (bf16, at most 128 KB) into shared memory in MMA-fragment order.  Warp w then takes
+//     slabs w and w+8 (64 bytes of K each) of every stage, converts the int8 codes to bf16
+//     in registers (exact, 7 ALU ops per 4 codes) and accumulates with the warp-level bf16
+//     MMA (fp32 accumulate).  After the last stage of a row group the 8 partial sums are
+//     added into a rotating shared-memory slot; the last warp to arrive scales, rounds
+//     once to the output type and writes y.  No barrier is needed between warps.
+//   * partial stages (K not a multiple of 1024) are handled without branches: every box
+//     of a stage is always loaded (columns past K read as zeros) and the staged
+//     activations are zero-padded to a whole number of stages.
+//
+// x fragments are stored as two planes of 16-byte pieces in lane order (conflict-free
+// loads); weight rows are 256 bytes apart, so a 16-byte load phase (2 rows x 4 lanes) has a
+// 2-way bank conflict, well within the shared-memory bandwidth this stream needs.
+#include "q8_kernels.cuh"
+
+namespace q8 {
+
+constexpr int WT_CONSUMERS = 8;                         // consumer warps (2 slabs each)
+constexpr int WT_THREADS = (WT_CONSUMERS + 1) * 32;     // + producer warp
+constexpr int WT_SLABS = 16;                            // 64-byte slabs per stage
+constexpr int WT_BOX = 256;                             // TMA box width (bytes of K)
+constexpr int WT_BOXES = WT_SLABS * 64 / WT_BOX;        // boxes per stage
+constexpr int WT_STAGE_BYTES = 16 * 64 * WT_SLABS;      // 16 KB
+constexpr int WT_MAX_SMEM = 227 * 1024;
+constexpr int WT_SLOTS = 16;                            // rotating partial-sum slots (> stages+1)
+
+struct WtSmem {
+    int stages;
+    size_t ring, xs, red, sws, bars, total;
+};
+
+// Rows of q a CTA may own (its s_w slice is staged in shared memory).
+constexpr int WT_MAX_ROWS = 1024;
+
+static __host__ __device__ inline WtSmem wt_layout(int M, int K, int MT, int stages) {
+    WtSmem L;
+    L.stages = stages;
+    L.ring = 0;
+    L.xs = (size_t)stages * WT_STAGE_BYTES;
+    const int Kpad = (K + WT_SLABS * 64 - 1) / (WT_SLABS * 64) * (WT_SLABS * 64);
+    const size_t xbytes = (size_t)M * Kpad * 2;
+    L.red = L.xs + ((xbytes + 127) / 128) * 128;
+    const size_t redbytes = (size_t)WT_SLOTS * MT * 32 * 4 * sizeof(float);
+    L.sws = L.red + redbytes;
+    L.bars = L.sws + (size_t)WT_MAX_ROWS * sizeof(float);
+    // barriers, slot counters, abort flag
+    L.total = L.bars + (size_t)2 * stages * sizeof(uint64_t) + (WT_SLOTS + 4) * sizeof(int);
+    return L;
+}
+
+// x fragment address: plane h (0/1), chunk c (64 k), activation row m, lane t (0..3):
+// the 16-byte piece x[m][64c + 16t + 8h .. +8].  Kpad = K rounded up to whole stages.
+__device__ __forceinline__ uint32_t xfrag_addr(uint32_t xs, int M, int Kpad, int c, int m,
+                                               int t, int h) {
+    return xs + (uint32_t)h * (uint32_t)(M * Kpad) + (uint32_t)(((c * M + m) * 4 + t) * 16);
+}
+
+template <int MT>
+__global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
+    const __grid_constant__ CUtensorMap wmap, const uint16_t* __restrict__ x,
+    const float* __restrict__ s_w, void* __restrict__ y, int y_bf16, int M, int N, int K,
+    int stages, int* status) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const WtSmem L = wt_layout(M, K, MT, stages);
+    uint8_t* ring = smem + L.ring;
+    float* slots = reinterpret_cast<float*>(smem + L.red);        // [WT_SLOTS][MT][32][4]
+    float* sws = reinterpret_cast<float*>(smem + L.sws);          // s_w of this CTA's rows
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+    uint64_t* empty = full + stages;
+    int* cnt = reinterpret_cast<int*>(empty + stages);               // [WT_SLOTS]
+    volatile int* abort_flag = cnt + WT_SLOTS;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nslab = K >> 6;                              // K % 64 == 0
+    const int nst = (nslab + WT_SLABS - 1) / WT_SLABS;     // stages per row group
+    const int RG = (N + 15) >> 4;
+    const int rg0 = (int)((int64_t)RG * blockIdx.x / gridDim.x);
+    const int rg1 = (int)((int64_t)RG * (blockIdx.x + 1) / gridDim.x);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], WT_CONSUMERS);
+        }
+        for (int i = 0; i < WT_SLOTS; ++i) cnt[i] = 0;
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    for (int i = threadIdx.x; i < WT_SLOTS * MT * 128; i += WT_THREADS) slots[i] = 0.0f;
+    // Programmatic dependent launch: let the next kernel on the stream start its own
+    // set-up now, and wait for the previous one to finish (and its writes to be
+    // visible) before the first global-memory access -- any input may be its output.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    {
+        // The epilogue must not wait on global loads (a stalled warp holds back the ring):
+        // stage this CTA's per-channel scales once.
+        const int row0 = rg0 * 16, rows = min(rg1 * 16, N) - row0;
+        for (int i = threadIdx.x; i < rows; i += WT_THREADS) sws[i] = __ldg(s_w + row0 + i);
+    }
+    __syncthreads();
+
+    if (warp == WT_CONSUMERS) {
+        // ------------------------------------------------------------- producer
+        if (lane == 0) {
+            tma_prefetch_desc(&wmap);
+            int it = 0, s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int rg = rg0; rg < rg1 && ok; ++rg) {
+                for (int st = 0; st < nst; ++st) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int k0 = st * WT_SLABS * 64;
+                    mbar_expect_tx(&full[s], (uint32_t)WT_STAGE_BYTES);
+                    uint8_t* dst = ring + (size_t)s * WT_STAGE_BYTES;
+#pragma unroll
+                    for (int j = 0; j < WT_BOXES; ++j)     // boxes past K read as zeros
+                        tma_load_2d(dst + j * 16 * WT_BOX, &wmap, k0 + j * WT_BOX, rg * 16,
+                                    &full[s]);
+                    ++it;
+                    if (++s == stages) { s = 0; ph ^= 1u; }
+                }
+            }
+            // Do not leave while copies issued here may still be landing in shared memory.
+            for (int i = max(0, it - stages); i < it; ++i)
+                mbar_drain(&full[i % stages], (uint32_t)(i / stages) & 1u);
+        }
+        return;
+    }
+
+    // ----------------------------------------------------------------- consumers
+    const int Kpad = nst * WT_SLABS * 64;
+    const uint32_t xs = smem_u32(smem + L.xs);
+    {
+        // x [M, K] -> fragment order (two planes of 16-byte pieces), element pairs
+        // regrouped to the (even, odd) k pairing of s8x4_to_bf16x2_eo; zero past K.
+        const int units = M * Kpad / 8;
+        const int per_row = Kpad / 8;
+        for (int u = threadIdx.x; u < units; u += WT_CONSUMERS * 32) {
+            const int m = u / per_row, r = u - m * per_row;
+            const int c = r >> 3, t = (r >> 1) & 3, h = r & 1;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (8 * r < K) v = ldg_keep(x + (int64_t)m * K + 8 * r);
+            const uint32_t p0 = __byte_perm(v.x, v.y, 0x5410), p1 = __byte_perm(v.x, v.y, 0x7632);
+            const uint32_t p2 = __byte_perm(v.z, v.w, 0x5410), p3 = __byte_perm(v.z, v.w, 0x7632);
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(
+                             xfrag_addr(xs, M, Kpad, c, m, t, h)),
+                         "r"(p0), "r"(p1), "r"(p2), "r"(p3)
+                         : "memory");
+        }
+    }
+    named_bar_sync(1, WT_CONSUMERS * 32);
+
+    const int g = lane >> 2, t = lane & 3;
+    // This lane's weight bytes in a stage: slab j (j = warp, warp + 8) lives in box j/4,
+    // rows g and g+8, bytes (j%4)*64 + 16t .. +16.  Slab warp+8 is two boxes further.
+    const uint32_t ring_u = smem_u32(ring);
+    const uint32_t w_off = (uint32_t)((warp >> 2) * 16 * WT_BOX + g * WT_BOX + (warp & 3) * 64 +
+                                      t * 16);
+    constexpr uint32_t kSlab2 = 2 * 16 * WT_BOX;            // slab j+8 = 2 boxes on
+    // Activation fragments of chunk c = st*16 + j: plane 0 address; +1024*M bytes per
+    // stage; slab j+8 is 8 chunks (8*M*64 bytes) further.
+    uint32_t x_lane[MT];
+    bool x_live[MT];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int m = mt * 8 + g;
+        x_live[mt] = m < M;
+        x_lane[mt] = xfrag_addr(xs, M, Kpad, warp, x_live[mt] ? m : 0, t, 0);
+    }
+    const uint32_t plane = (uint32_t)(M * Kpad);
+    const uint32_t x_step = (uint32_t)(WT_SLABS * M * 64);
+    const uint32_t x_slab2 = (uint32_t)(8 * M * 64);
+
+    int s = 0, slot = 0;
+    uint32_t ph = 0;
+    uint32_t wst = ring_u + w_off;                           // stage s, this lane
+    // Independent accumulator chains: consecutive MMAs of a warp go to different
+    // accumulators, so they do not wait on each other's results.
+    constexpr int CH = MT == 1 ? 8 : 4;
+    for (int rg = rg0; rg < rg1; ++rg) {
+        float acc[CH][MT][4];
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[c][mt][i] = 0.0f;
+
+        uint32_t xst = 0;                                    // stage offset into x
+        for (int st = 0; st < nst; ++st) {
+            mbar_wait(&full[s], ph, status, abort_flag);   // on expiry: finish with garbage
+            uint4 w[2][2];
+            w[0][0] = lds128(wst);
+            w[0][1] = lds128(wst + 8 * WT_BOX);
+            w[1][0] = lds128(wst + kSlab2);
+            w[1][1] = lds128(wst + kSlab2 + 8 * WT_BOX);
+            uint4 xa[2][MT][2];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    if (x_live[mt]) {
+                        const uint32_t xa_addr = x_lane[mt] + xst + (jj ? x_slab2 : 0u);
+                        xa[jj][mt][0] = lds128(xa_addr);
+                        xa[jj][mt][1] = lds128(xa_addr + plane);
+                    } else {
+                        xa[jj][mt][0] = xa[jj][mt][1] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);           // operands are in registers
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const uint32_t wav[4] = {w[jj][0].x, w[jj][0].y, w[jj][0].z, w[jj][0].w};
+                const uint32_t wbv[4] = {w[jj][1].x, w[jj][1].y, w[jj][1].z, w[jj][1].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t alo, ahi, blo, bhi;       // (even, odd) byte pairs
+                    s8x4_to_bf16x2_eo(wav[q], alo, ahi);
+                    s8x4_to_bf16x2_eo(wbv[q], blo, bhi);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const uint4& xv = xa[jj][mt][q >> 1];
+                        const uint32_t b0 = (q & 1) ? xv.z : xv.x;
+                        const uint32_t b1 = (q & 1) ? xv.w : xv.y;
+                        mma_bf16_16816(acc[(jj * 4 + q) % CH][mt], alo, blo, ahi, bhi, b0, b1);
+                    }
+                }
+            }
+            xst += x_step;
+            wst += WT_STAGE_BYTES;
+            if (++s == stages) { s = 0; ph ^= 1u; wst = ring_u + w_off; }
+        }
+
+        // Add this warp's partial sums into the group's slot; the last warp to arrive
+        // scales, writes y and clears the slot.  Slots rotate, so no barrier is needed:
+        // a warp can run at most `stages` stages (<= WT_SLOTS - 2 groups) ahead of the
+        // slowest one.
+        float* sl = slots + (size_t)slot * MT * 128;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float v = 0.0f;
+#pragma unroll
+                for (int c = 0; c < CH; ++c) v += acc[c][mt][i];
+                atomicAdd(&sl[(mt * 32 + lane) * 4 + i], v);
+            }
+        __threadfence_block();
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) prev = atomicAdd(&cnt[slot], 1);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == WT_CONSUMERS - 1) {
+            // Take the group's sums, clear the slot and release it before any global store.
+            __threadfence_block();
+            float vv[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                volatile float* vp = &sl[(mt * 32 + lane) * 4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) vv[mt][i] = vp[i];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) vp[i] = 0.0f;
+            }
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) atomicExch(&cnt[slot], 0);
+            const int n0 = rg * 16;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int m = mt * 8 + 2 * t + (i & 1);
+                    const int n = n0 + g + 8 * (i >> 1);
+                    if (m < M && n < N) {
+                        const float r = vv[mt][i] * sws[n - rg0 * 16];
+                        if (y_bf16)
+                            reinterpret_cast<__nv_bfloat16*>(y)[(int64_t)m * N + n] =
+                                __float2bfloat16_rn(r);
+                        else
+                            reinterpret_cast<float*>(y)[(int64_t)m * N + n] = r;
+                    }
+                }
+        }
+        if (++slot == WT_SLOTS) slot = 0;
+    }
+}
+
+// ----------------------------------------------------------------------- host side
+
+// Tensor-map encoder from the driver, fetched once through the runtime (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D map over a row-major uint8 matrix [rows, cols] (row stride = cols bytes).
+bool make_tmap_u8_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                     int box_cols, int box_rows, CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Whether the TMA path takes this problem: K % 64 == 0, M <= 16 and the activations fit
+// next to at least 4 ring stages.
+bool w8a16_tma_fits(int64_t M, int64_t K) {
+    if (M < 1 || M > 16 || (K % 64) != 0) return false;
+    const int MT = M <= 8 ? 1 : 2;
+    return wt_layout((int)M, (int)K, MT, 4).total <= (size_t)WT_MAX_SMEM;
+}
+
+template <int MT>
+static cudaError_t launch_wt(const CUtensorMap& map, const uint16_t* x, const float* s_w, void* y,
+                             int y_bf16, int M, int N, int K, cudaStream_t st, int num_sms,
+                             int* status) {
+    int stages = 8;    // must stay <= WT_SLOTS - 2
+    while (stages > 4 && wt_layout(M, K, MT, stages).total > (size_t)WT_MAX_SMEM) --stages;
+    const WtSmem L = wt_layout(M, K, MT, stages);
+    cudaError_t e = cudaFuncSetAttribute(k_w8a16_tma<MT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L.total);
+    if (e != cudaSuccess) return e;
+    const int RG = (N + 15) / 16;
+    int grid = RG < num_sms ? RG : num_sms;
+    const int max_rg = WT_MAX_ROWS / 16;                  // rows a CTA may own
+    if ((RG + grid - 1) / grid > max_rg) grid = (RG + max_rg - 1) / max_rg;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(WT_THREADS);
+    cfg.dynamicSmemBytes = L.total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_w8a16_tma<MT>, map, x, s_w, y, y_bf16, M, N, K, stages,
+                              status);
+}
+
+cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
+                             int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,
+                             int num_sms, int* status) {
+    CUtensorMap map;
+    if (!make_tmap_u8_2d(&map, q, N, K, WT_BOX, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (M <= 8)
+        return launch_wt<1>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms, status);
+    return launch_wt<2>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms, status);
+}
+
+}  // namespace q8

@@ -33,11 +33,12 @@ struct DevInfo {
     int checked = 0;
     int ok = 0;
     int num_sms = 0;
+    int* status = nullptr;     // device address of g_device_status on this device
 };
 static DevInfo g_dev[128];
 static std::mutex g_dev_mu;
 
-static q8_status current_device(int& num_sms) {
+static q8_status current_device(int& num_sms, int** status = nullptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
@@ -56,9 +57,18 @@ static q8_status current_device(int& num_sms) {
         }
         d.ok = (major == 10 && minor == 0);
         d.num_sms = sms;
+        if (d.ok) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+                cudaGetLastError();
+                return Q8_ERR_LAUNCH;
+            }
+            d.status = static_cast<int*>(p);
+        }
         d.checked = 1;
     }
     num_sms = d.num_sms;
+    if (status) *status = d.status;
     return d.ok ? Q8_OK : Q8_ERR_UNSUPPORTED_ARCH;
 }
 
@@ -219,7 +229,11 @@ q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w, void
     if (!x || !q || !s_w || !y) return Q8_ERR_NULL;
     if (!aligned16(x) || !aligned16(q)) return Q8_ERR_ALIGN;
     int sms = 0;
-    Q8_TRY(current_device(sms));
+    int* status = nullptr;
+    Q8_TRY(current_device(sms, &status));
+    if (w8a16_tma_fits(M, K))
+        return launched(launch_w8a16_tma((const uint16_t*)x, q, s_w, y, yt == Q8_BF16, M, N,
+                                         (int)K, (cudaStream_t)stream, sms, status));
     return launched(launch_w8a16_gemv((const uint16_t*)x, q, s_w, y, yt == Q8_BF16, M, N, (int)K,
                                       (cudaStream_t)stream, sms));
 }

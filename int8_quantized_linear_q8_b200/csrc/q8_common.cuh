@@ -108,6 +108,30 @@ __device__ __forceinline__ void s8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_
     hi = __byte_perm(__float_as_uint(a2), __float_as_uint(a3), 0x7632);
 }
 
+// Four int8 codes w = [b0 b1 b2 b3] -> bf16x2 (b0, b2) and (b1, b3), exact, in 7 ALU ops.
+// For a byte b in the low half of a 16-bit lane: bf16 bits 0x4300 | (b & 0x7F) are the value
+// 128 + (b & 0x7F), and 0x4300 | (b & 0x80) is 128 (b >= 0) or 256 (b < 0); their
+// difference is b in both cases and is exact in bf16 (an integer of at most 8 bits).
+// The odd bytes are first shifted into the low halves.  The pairing (even, odd) is a
+// permutation of k that the caller applies to the other MMA operand as well.
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t bits) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(bits));  // (a&b)|c
+    return d;
+}
+__device__ __forceinline__ void s8x4_to_bf16x2_eo(uint32_t w, uint32_t& even, uint32_t& odd) {
+    const uint32_t o = w >> 8;
+    even = bf16x2_sub(lop_and_or(w, 0x007F007Fu, 0x43004300u),
+                      lop_and_or(w, 0x00800080u, 0x43004300u));
+    odd = bf16x2_sub(lop_and_or(o, 0x007F007Fu, 0x43004300u),
+                     lop_and_or(o, 0x00800080u, 0x43004300u));
+}
+
 // ---------------------------------------------------------------- legacy warp MMA
 // D(16x8 fp32) += A(16x16 bf16, row) * B(16x8 bf16, col)
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
@@ -129,6 +153,106 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t 
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+}  // namespace q8
+
+// ============================================================ TMA / mbarrier (sm_90+)
+#include <cuda.h>   // CUtensorMap (type only)
+
+namespace q8 {
+
+// Device status codes written to the caller-visible status word.
+constexpr int kStatusWaitTimeout = 1;
+// Bounded waits give up after this many nanoseconds of %globaltimer (a correct kernel
+// never waits more than microseconds; the limit only turns a logic error into an error
+// status instead of a hang).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for the phase with the given parity to complete.  Returns false, after recording
+// kStatusWaitTimeout in *status and raising the CTA's shared abort flag, if it has not
+// completed within kWaitLimitNs -- or at once if the abort flag is already raised (so
+// that after one expired wait every other wait of the CTA ends quickly too).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
+                                          volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicExch(status, kStatusWaitTimeout);
+                return false;
+            }
+        }
+    }
+}
+// Bounded wait used only on exit paths: waits for a phase without touching flags.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+    }
+}
+// 2-D tiled TMA load of one box into shared memory; completion is signalled on `bar`
+// (transaction bytes).  c0 is the innermost coordinate (bytes for 8-bit elements) and
+// must be a multiple of 16.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
 }
 
 }  // namespace q8

@@ -49,6 +49,14 @@ cudaError_t launch_observe_minmax(const float* x, int64_t n, float* mm, int rese
 cudaError_t launch_quantize_weight_q4gs(const float* W, int64_t N, int K, int G, uint8_t* q4,
                                         float* gs, cudaStream_t st);
 
+// k_gemv_tma.cu
+bool make_tmap_u8_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                     int box_cols, int box_rows, CUtensorMapSwizzle swz);
+bool w8a16_tma_fits(int64_t M, int64_t K);
+cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
+                             int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,
+                             int num_sms, int* status);
+
 // k_gemv.cu
 cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
                               int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,

@@ -171,8 +171,11 @@ def test_w8a16_sweep_bf16(shape, M):
     check_bf16(_bits(y), y64, absum, f"W8A16 M={M} K={shape.K} N={shape.N}")
 
 
-@pytest.mark.parametrize("M,N,K", [(3, 17, 16), (9, 40, 48), (16, 1, 64), (17, 33, 80),
-                                   (40, 130, 1040), (5, 2049, 2000)])
+@pytest.mark.parametrize("M,N,K", [
+    # TMA-streamed path (K % 64 == 0, M <= 16): ragged N, K not a multiple of the 1 KB stage
+    (16, 1, 64), (1, 17, 64), (5, 2049, 1024), (12, 1000, 4160), (9, 33, 128), (2, 300, 11008),
+    # register-streamed fallback (K % 64 != 0, or M > 16)
+    (3, 17, 16), (9, 40, 48), (17, 33, 80), (40, 130, 1040), (5, 2049, 2000)])
 @pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
 def test_w8a16_ragged(M, N, K, out):
     y, y64, absum = _w8a16_case(M, N, K, 400 + N, 401 + M, out)
