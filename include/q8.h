@@ -197,7 +197,8 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra);
 /* Integer GEMM with int32 output, acc[m,n] = sum_k a[m,k] * b[n,k] (exact): the
  * tcgen05 int8 MMA path of q8_linear_w8a8 without its epilogue, exported so that the
  * int32 accumulators can be checked bit for bit.
- *   a device int8 [M, K]; b device int8 [N, K]; acc device int32 [M, N]. */
+ *   a device int8 [M, K]; b device int8 [N, K]; acc device int32 [M, N]; K >= 128
+ *   (Q8_ERR_SHAPE otherwise). */
 q8_status q8_gemm_s8s8_s32(const int8_t* a, const int8_t* b, int32_t* acc,
                            int64_t M, int64_t N, int64_t K, void* stream);
 

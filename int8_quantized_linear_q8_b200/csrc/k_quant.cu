@@ -148,6 +148,8 @@ __global__ __launch_bounds__(256) void k_quantize_static(const float* __restrict
                                                          float s1, float z1f, int8_t* __restrict__ xq1,
                                                          int has2, float s2, float z2f,
                                                          int8_t* __restrict__ xq2) {
+    // the linear launched next may start its set-up (it waits for this kernel's codes)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const float inv1 = __fdiv_rn(1.0f, s1);
     const float inv2 = has2 ? __fdiv_rn(1.0f, s2) : 0.0f;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n16;

@@ -101,6 +101,12 @@ static inline q8_status launched(cudaError_t e) {
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Activation rows up to which the W8A8 linear runs as a GEMV (weights streamed once per
+// 16 rows); above it the tensor-core GEMM takes over.  The tensor-core path loads K in
+// 128-byte steps and needs at least one whole step.
+constexpr int64_t kW8A8GemvMaxM = 16;
+constexpr int64_t kTcMinK = 128;
+
 // Workspace plans (byte offsets inside the caller's workspace).
 struct W8A8Plan {
     size_t xq1 = 0, xq2 = 0, bytes = 0;
@@ -257,13 +263,14 @@ q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* sec
     if (second) Q8_TRY(check_qparams(*second));
     if (M == 0) return Q8_OK;
     if (!x || !q || !wsum || !s_w || !y) return Q8_ERR_NULL;
-    if (!aligned16(x) || !aligned16(q)) return Q8_ERR_ALIGN;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(y)) return Q8_ERR_ALIGN;
     const int two = second != nullptr;
     const W8A8Plan plan = plan_w8a8(M, K, two);
     if (plan.bytes > 0 && (!workspace || ws_bytes < plan.bytes)) return Q8_ERR_WORKSPACE;
     if (!aligned16(workspace)) return Q8_ERR_ALIGN;
     int sms = 0;
-    Q8_TRY(current_device(sms));
+    int* status = nullptr;
+    Q8_TRY(current_device(sms, &status));
     cudaStream_t st = (cudaStream_t)stream;
     int8_t* xq1 = (int8_t*)workspace + plan.xq1;
     int8_t* xq2 = two ? (int8_t*)workspace + plan.xq2 : nullptr;
@@ -271,6 +278,9 @@ q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* sec
     const int z2 = two ? second->zero_point : 0;
     Q8_TRY(launched(launch_quantize_static(x, M, (int)K, first.scale, first.zero_point, two, s2,
                                            z2, xq1, xq2, st, sms)));
+    if (M > kW8A8GemvMaxM && K >= kTcMinK)
+        return launched(launch_w8a8_tc(xq1, xq2, first.scale, first.zero_point, two, s2, z2, q,
+                                       wsum, s_w, y, M, N, (int)K, st, sms, status));
     return launched(launch_w8a8_gemv_codes(xq1, xq2, first.scale, first.zero_point, two, s2, z2,
                                            q, wsum, s_w, y, M, N, (int)K, st));
 }
@@ -285,8 +295,17 @@ q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* g
 
 q8_status q8_gemm_s8s8_s32(const int8_t* a, const int8_t* b, int32_t* acc, int64_t M, int64_t N,
                            int64_t K, void* stream) {
-    (void)a; (void)b; (void)acc; (void)M; (void)N; (void)K; (void)stream;
-    return Q8_ERR_ARG;
+    if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (K < kTcMinK) return Q8_ERR_SHAPE;
+    if (M == 0) return Q8_OK;
+    if (!a || !b || !acc) return Q8_ERR_NULL;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(acc)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    int* status = nullptr;
+    Q8_TRY(current_device(sms, &status));
+    return launched(launch_gemm_s8s8_s32_tc(a, b, acc, M, N, (int)K, (cudaStream_t)stream, sms,
+                                           status));
 }
 
 q8_status q8_last_device_status(void* stream) {

@@ -57,6 +57,14 @@ cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_
                              int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,
                              int num_sms, int* status);
 
+// k_gemm_tc.cu
+cudaError_t launch_gemm_s8s8_s32_tc(const int8_t* a, const int8_t* b, int32_t* acc, int64_t M,
+                                    int64_t N, int K, cudaStream_t st, int num_sms, int* status);
+cudaError_t launch_w8a8_tc(const int8_t* xq1, const int8_t* xq2, float s1, int z1, int has2,
+                           float s2, int z2, const int8_t* q, const int32_t* wsum,
+                           const float* s_w, float* y, int64_t M, int64_t N, int K,
+                           cudaStream_t st, int num_sms, int* status);
+
 // k_gemv.cu
 cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
                               int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,

@@ -210,3 +210,66 @@ def test_w8a8_small_m(M, N, two):
     y64, absum, _, _ = oracle.linear_w8a8(x.numpy(), first, rq, rs,
                                           second=second if two else None)
     check_f32(y.cpu().numpy(), y64, absum, f"W8A8 M={M} N={N} two={two}")
+
+
+@pytest.mark.parametrize("M,N,K,rows", [
+    (128, 256, 128, None), (256, 512, 1024, None), (300, 300, 960, None), (37, 33, 128, None),
+    (17, 2560, 960, None), (1000, 1000, 4096, None),
+    (4096, 4096, 4096, [0, 1, 127, 128, 1000, 2047, 4095]),
+    (4096, 11008, 4096, [0, 129, 4095]), (4096, 4096, 11008, [5, 2100, 4094])])
+def test_gemm_s8s8_s32_bit_exact(M, N, K, rows):
+    """int32 accumulators of the tcgen05 int8 GEMM, bit for bit (sampled rows at full size)."""
+    g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
+    a = torch.randint(-128, 128, (M, K), dtype=torch.int8, generator=g)
+    b = torch.randint(-128, 128, (N, K), dtype=torch.int8, generator=g)
+    acc = q8.q8_gemm_s8s8_s32(a.to(DEV), b.to(DEV)).cpu().numpy()
+    ref = oracle.gemm_s8s8_s32(a.numpy(), b.numpy(), rows=rows)
+    got = acc if rows is None else acc[rows]
+    assert np.array_equal(got, ref)
+
+
+def test_gemm_s8s8_s32_extreme_values():
+    """All-(-128) operands: the largest magnitude sums (K * 2^14) stay exact in int32."""
+    M, N, K = 130, 260, 4096
+    a = torch.full((M, K), -128, dtype=torch.int8)
+    b = torch.full((N, K), -128, dtype=torch.int8)
+    acc = q8.q8_gemm_s8s8_s32(a.to(DEV), b.to(DEV)).cpu().numpy()
+    assert (acc == K * 128 * 128).all()
+
+
+@pytest.mark.parametrize("M", [256, 2048])
+@pytest.mark.parametrize("N", wl.W8A8_N)
+@pytest.mark.parametrize("two", [False, True])
+def test_w8a8_prefill_tensor_core(M, N, two):
+    """Static W8A8 at K = 960 on the tensor-core path (single and two-pass)."""
+    K = wl.W8A8_K
+    first, second = _w8a8_qparams(K)
+    x, _ = wl.w8a8_inputs(M, K=K)
+    W = wl.weight(N, K, seed=wl.W8A8_SEED_W)
+    q, s, ws = q8.q8_quantize_weight(W.to(DEV))
+    y = q8.q8_linear_w8a8(x.to(DEV), first, q, ws, s, second=second if two else None)
+    torch.cuda.synchronize()
+    rq, rs, _ = oracle.quantize_weight(W.numpy())
+    y64, absum, _, _ = oracle.linear_w8a8(x.numpy(), first, rq, rs,
+                                          second=second if two else None)
+    check_f32(y.cpu().numpy(), y64, absum, f"W8A8 TC M={M} N={N} two={two}")
+
+
+@pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 11008), (11008, 4096)])
+@pytest.mark.parametrize("two", [False, True])
+def test_w8a8_llama_prefill_sampled(K, N, two):
+    """Llama-shaped prefill linears at M = 4096 (sampled output rows vs the oracle)."""
+    M = wl.LLAMA_PREFILL_M
+    x = wl.normal((M, K), 1.0, seed=500 + K + N)
+    mm = torch.empty(2, device=DEV)
+    q8.q8_observe_minmax(x.to(DEV), mm, reset=True)
+    first = q8.q8_qparams_from_minmax(*mm.cpu().tolist())
+    second = (float(np.float32(first[0]) / np.float32(255.0)), 0) if two else None
+    W = wl.weight(N, K, seed=600 + K + N)
+    q, s, ws = q8.q8_quantize_weight(W.to(DEV))
+    y = q8.q8_linear_w8a8(x.to(DEV), first, q, ws, s, second=second)
+    torch.cuda.synchronize()
+    rows = [0, 1, 127, 128, 2049, M - 1]
+    rq, rs, _ = oracle.quantize_weight(W.numpy())
+    y64, absum, _, _ = oracle.linear_w8a8(x.numpy(), first, rq, rs, second=second, rows=rows)
+    check_f32(y.cpu().numpy()[rows], y64, absum, f"W8A8 llama K={K} N={N} two={two}")
