@@ -202,6 +202,31 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra);
 q8_status q8_gemm_s8s8_s32(const int8_t* a, const int8_t* b, int32_t* acc,
                            int64_t M, int64_t N, int64_t K, void* stream);
 
+/* Allocation-free W8A8.  The source pages have no counterpart to this call: it exists for
+ * callers that cannot allocate device memory -- a host runtime that has reserved all
+ * device memory for its own pool, a latency-critical loop in which cudaMalloc's implicit
+ * device-wide synchronisation is not acceptable, or a plain C caller with no allocator to
+ * provide q8_linear_w8a8's workspace.  It computes exactly what q8_linear_w8a8 computes,
+ * with the same arguments minus the workspace, using a scratch array built into the
+ * library instead:
+ *   - limit: the scratch holds Q8_NOALLOC_SCRATCH_BYTES (16 MiB); calls whose
+ *     q8_workspace_bytes(Q8_OP_LINEAR_W8A8, M, N, K, second != NULL) exceeds it return
+ *     Q8_ERR_WORKSPACE before anything is enqueued;
+ *   - every GPU on which the library's device code is loaded holds that 16 MiB until the
+ *     process exits;
+ *   - the first call on a device (with that device current) looks up the array's device
+ *     address once; make that first call before any stream capture;
+ *   - all calls share the one array, whose contents carry over from call to call (nothing
+ *     in it needs to start at zero: each call overwrites the part it reads).  Calls that
+ *     may overlap on the GPU (issued on different streams with no ordering between
+ *     them) race on it and give wrong results; order them.  Calls on one stream are
+ *     ordered.
+ *   - nothing here calls cudaMalloc, cudaFree or any allocating routine. */
+#define Q8_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+q8_status q8_linear_w8a8_noalloc(const float* x, q8_qparams first, const q8_qparams* second,
+                                 const int8_t* q, const int32_t* wsum, const float* s_w,
+                                 float* y, int64_t M, int64_t N, int64_t K, void* stream);
+
 /* Host, synchronising.  Reads and clears the device status word that kernels with
  * bounded waits set when a wait expires (Q8_OK if none did since the last read).
  * Waits for the given stream first. */

@@ -32,7 +32,10 @@ SYMBOLS = (
     "q8_quantize_static", "q8_observe_minmax", "q8_qparams_from_minmax",
     "q8_quantize_weight_q4gs", "q8_linear_w8a16", "q8_linear_w8a8", "q8_linear_dq8ca_q4gsw",
     "q8_workspace_bytes", "q8_gemm_s8s8_s32", "q8_last_device_status",
+    "q8_linear_w8a8_noalloc",
 )
+# Built-in scratch of q8_linear_w8a8_noalloc (bytes).
+Q8_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class Q8Error(RuntimeError):
@@ -89,6 +92,9 @@ def _lib() -> ctypes.CDLL:
     L.q8_gemm_s8s8_s32.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp]
     L.q8_last_device_status.restype = st
     L.q8_last_device_status.argtypes = [_vp]
+    L.q8_linear_w8a8_noalloc.restype = st
+    L.q8_linear_w8a8_noalloc.argtypes = [_vp, q8_qparams, ctypes.POINTER(q8_qparams), _vp, _vp,
+                                         _vp, _vp, _i64, _i64, _i64, _vp]
     _LIB = L
     return L
 
@@ -266,6 +272,27 @@ def q8_linear_w8a8(x: torch.Tensor, first, q: torch.Tensor, wsum: torch.Tensor,
     _check(_lib().q8_linear_w8a8(_ptr(x), _qp(first), sec, _ptr(q), _ptr(wsum), _ptr(s_w),
                                  _ptr(y), M, N, K, _ptr(workspace), wsb, _stream(stream)),
            "q8_linear_w8a8")
+    return y
+
+
+def q8_linear_w8a8_noalloc(x: torch.Tensor, first, q: torch.Tensor, wsum: torch.Tensor,
+                           s_w: torch.Tensor, second=None, y=None, stream=None) -> torch.Tensor:
+    """q8_linear_w8a8 without a workspace: for callers that cannot allocate device memory.
+
+    The library uses a 16 MiB scratch array of its own (shared by every call on a device;
+    calls on different streams must not overlap).  Only `y` is allocated here when the
+    caller does not pass it; pass `y` to allocate nothing at all."""
+    M, K = x.shape
+    N = q.shape[0]
+    _need(x, "x", torch.float32, (M, K))
+    _need(q, "q", torch.int8, (N, K))
+    _need(wsum, "wsum", torch.int32, (N,))
+    _need(s_w, "s_w", torch.float32, (N,))
+    y = _out(y, "y", torch.float32, (M, N), x.device)
+    sec = None if second is None else ctypes.byref(_qp(second))
+    _check(_lib().q8_linear_w8a8_noalloc(_ptr(x), _qp(first), sec, _ptr(q), _ptr(wsum),
+                                         _ptr(s_w), _ptr(y), M, N, K, _stream(stream)),
+           "q8_linear_w8a8_noalloc")
     return y
 
 
