@@ -183,8 +183,10 @@ q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* sec
  *     y[m,n] = s[m] * sum_g gs[n,g] * sum_{k in g} (xq[m,k] - z[m]) * q4[n,k]
  * with per-group int32 partial sums and fp32 accumulation across groups.
  *   x device bf16 [M, K]; q4 device uint8 [N, K/2]; gs device fp32 [N, K/G];
- *   y device fp32 [M, N]; G in {32, 64, 128, 256}, K % G == 0.
- *   workspace: at least q8_workspace_bytes(Q8_OP_LINEAR_DQ8CA_Q4GSW, M, N, K, G). */
+ *   y device fp32 [M, N]; G in {32, 64, 128, 256}; K % 128 == 0 and K % G == 0
+ *   (Q8_ERR_SHAPE otherwise).
+ *   workspace: at least q8_workspace_bytes(Q8_OP_LINEAR_DQ8CA_Q4GSW, M, N, K, G) bytes;
+ *   it receives the activation codes, scales and zero points. */
 q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* gs, int G,
                                 float* y, int64_t M, int64_t N, int64_t K,
                                 void* workspace, size_t ws_bytes, void* stream);

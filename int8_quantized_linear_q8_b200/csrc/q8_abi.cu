@@ -120,6 +120,20 @@ static W8A8Plan plan_w8a8(int64_t M, int64_t K, int two) {
     return p;
 }
 
+struct Q4Plan {
+    size_t xq = 0, s = 0, z = 0, bytes = 0;
+};
+static Q4Plan plan_q4(int64_t M, int64_t K) {
+    Q4Plan p;
+    if (M <= 0) return p;
+    p.xq = 0;
+    p.s = align_up((size_t)M * (size_t)K, 256);
+    p.z = p.s + align_up((size_t)M * 4, 256);
+    p.bytes = p.z + align_up((size_t)M * 4, 256);
+    return p;
+}
+static inline bool valid_group(int G) { return G == 32 || G == 64 || G == 128 || G == 256; }
+
 }  // namespace q8
 
 using namespace q8;
@@ -248,7 +262,9 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) 
     if (M < 0 || N < 1 || check_k(K) != Q8_OK) return 0;
     switch (op) {
         case Q8_OP_LINEAR_W8A8: return plan_w8a8(M, K, extra != 0).bytes;
-        case Q8_OP_LINEAR_DQ8CA_Q4GSW: return 0;
+        case Q8_OP_LINEAR_DQ8CA_Q4GSW:
+            if (!valid_group(extra) || K % 128 != 0 || K % extra != 0) return 0;
+            return plan_q4(M, K).bytes;
     }
     return 0;
 }
@@ -288,9 +304,24 @@ q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* sec
 q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* gs, int G,
                                 float* y, int64_t M, int64_t N, int64_t K, void* workspace,
                                 size_t ws_bytes, void* stream) {
-    (void)x; (void)q4; (void)gs; (void)G; (void)y; (void)M; (void)N; (void)K;
-    (void)workspace; (void)ws_bytes; (void)stream;
-    return Q8_ERR_ARG;
+    if (!valid_group(G)) return Q8_ERR_ARG;
+    if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (K % 128 != 0 || K % G != 0) return Q8_ERR_SHAPE;
+    if (M == 0) return Q8_OK;
+    if (!x || !q4 || !gs || !y) return Q8_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q4) || !aligned16(gs) || !aligned16(y)) return Q8_ERR_ALIGN;
+    const Q4Plan plan = plan_q4(M, K);
+    if (!workspace || ws_bytes < plan.bytes) return Q8_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    cudaStream_t st = (cudaStream_t)stream;
+    int8_t* xq = (int8_t*)workspace + plan.xq;
+    float* s = (float*)((uint8_t*)workspace + plan.s);
+    int32_t* z = (int32_t*)((uint8_t*)workspace + plan.z);
+    Q8_TRY(launched(launch_choose_qparams((const uint16_t*)x, M, (int)K, s, z, xq, st)));
+    return launched(launch_q4_gemv(xq, s, z, q4, gs, G, y, M, N, (int)K, st));
 }
 
 q8_status q8_gemm_s8s8_s32(const int8_t* a, const int8_t* b, int32_t* acc, int64_t M, int64_t N,

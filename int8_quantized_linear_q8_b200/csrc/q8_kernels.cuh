@@ -65,6 +65,11 @@ cudaError_t launch_w8a8_tc(const int8_t* xq1, const int8_t* xq2, float s1, int z
                            const float* s_w, float* y, int64_t M, int64_t N, int K,
                            cudaStream_t st, int num_sms, int* status);
 
+// k_q4.cu
+cudaError_t launch_q4_gemv(const int8_t* xq, const float* s, const int32_t* z, const uint8_t* q4,
+                           const float* gs, int G, float* y, int64_t M, int64_t N, int K,
+                           cudaStream_t st);
+
 // k_gemv.cu
 cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
                               int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,

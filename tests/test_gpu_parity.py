@@ -273,3 +273,40 @@ def test_w8a8_llama_prefill_sampled(K, N, two):
     rq, rs, _ = oracle.quantize_weight(W.numpy())
     y64, absum, _, _ = oracle.linear_w8a8(x.numpy(), first, rq, rs, second=second, rows=rows)
     check_f32(y.cpu().numpy()[rows], y64, absum, f"W8A8 llama K={K} N={N} two={two}")
+
+
+# ----------------------------------------------------------------------- 8da4w (a7)
+
+
+def _q4_case(M, N, K, G, seed_x, seed_w, zero_x_rows=()):
+    x = wl.normal_bf16((M, K), 1.0, seed=seed_x)
+    for r in zero_x_rows:
+        x[r] = 0
+    W = wl.weight(N, K, seed=seed_w)
+    q4, gs = q8.q8_quantize_weight_q4gs(W.to(DEV), G)
+    y = q8.q8_linear_dq8ca_q4gsw(x.to(DEV), q4, gs, G)
+    torch.cuda.synchronize()
+    return x, q4.cpu().numpy(), gs.cpu().numpy(), y.cpu().numpy()
+
+
+@pytest.mark.parametrize("M", wl.Q4_M)
+@pytest.mark.parametrize("G", wl.Q4_G)
+def test_dq8ca_q4gsw_config(M, G):
+    """8da4w at K = 4096, N = 11008 (sampled rows for the large M)."""
+    K, N = wl.Q4_K, wl.Q4_N
+    x, q4, gs, y = _q4_case(M, N, K, G, wl.Q4_SEED_X, wl.Q4_SEED_W, zero_x_rows=(0,))
+    rows = None if M <= 64 else [0, 1, 63, 64, M // 2, M - 1]
+    s, z, xq = oracle.choose_qparams(wl.bf16_bits(x))
+    y64, absum = oracle.linear_dq8ca_q4gsw(xq, s, z, q4, gs, G, rows=rows)
+    got = y if rows is None else y[rows]
+    check_f32(got, y64, absum, f"8da4w M={M} G={G}")
+    assert (y[0] == 0).all()                    # an all-zero activation row gives 0 exactly
+
+
+@pytest.mark.parametrize("M,N,K,G", [(3, 17, 128, 32), (9, 40, 256, 64), (17, 33, 512, 128),
+                                     (5, 300, 1024, 256), (1, 1, 128, 128), (70, 129, 384, 32)])
+def test_dq8ca_q4gsw_ragged(M, N, K, G):
+    x, q4, gs, y = _q4_case(M, N, K, G, 900 + M, 901 + N)
+    s, z, xq = oracle.choose_qparams(wl.bf16_bits(x))
+    y64, absum = oracle.linear_dq8ca_q4gsw(xq, s, z, q4, gs, G)
+    check_f32(y, y64, absum, f"8da4w ragged M={M} N={N} K={K} G={G}")
