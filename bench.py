@@ -52,7 +52,10 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-paths", action="store_true", help="skip the sub-benchmarks")
-    p.add_argument("--profile", choices=["w8a16", "w8a8"], default=None,
+    p.add_argument("--eager", action="store_true",
+                   help="launch the timed steps one by one instead of replaying CUDA graphs "
+                        "(for profilers that cannot replay graph-captured launches)")
+    p.add_argument("--profile", choices=["w8a16", "w8a8", "q4"], default=None,
                    help="run only one kernel case --reps times (for ncu captures), then exit")
     p.add_argument("--pM", type=int, default=16)
     p.add_argument("--pN", type=int, default=32000)
@@ -237,6 +240,16 @@ class W8A16Sweep:
         return out
 
 
+class _EagerStep:
+    """Stands in for a captured step graph: replay() launches the step's kernels directly."""
+
+    def __init__(self, sweep, copy):
+        self.sweep, self.copy = sweep, copy
+
+    def replay(self):
+        self.sweep.step(self.copy)
+
+
 def time_graphs(graphs, steps: int, warmup: int, dist: Dist):
     for i in range(warmup):
         graphs[i % len(graphs)].replay()
@@ -378,6 +391,173 @@ def bench_w8a8_paths(dev, reps=30):
     return out
 
 
+def int8_peak_tops(peaks) -> float:
+    """Dense int8 tensor peak: the measured bf16 peak times NVIDIA's nominal int8:bf16
+    dense ratio (2:1, the fp8 = int8 rate)."""
+    return 2.0 * peaks["bf16_tflops"]
+
+
+def bench_w8a8_prefill(dev, peaks, reps=5):
+    """W8A8 (static per-tensor activations) at M = 4096 on the Llama-shaped linears
+    (tcgen05 int8 GEMM incl. its activation-code pre-kernel), one and two passes."""
+    import int8_quantized_linear_q8_b200 as q8
+
+    out = []
+    M = wl.LLAMA_PREFILL_M
+    g = torch.Generator(device=dev)
+    for (K, N) in [(4096, 4096), (4096, 11008), (11008, 4096)]:
+        g.manual_seed(31 * K + N)
+        x = torch.randn(M, K, generator=g, device=dev)
+        W = torch.randn(N, K, generator=g, device=dev) * 0.02
+        q, s, ws = q8.q8_quantize_weight(W)
+        del W
+        mm = torch.empty(2, device=dev)
+        q8.q8_observe_minmax(x, mm, reset=True)
+        first = q8.q8_qparams_from_minmax(*mm.cpu().tolist())
+        second = (float(np.float32(first[0]) / np.float32(255.0)), 0)
+        y = torch.empty(M, N, device=dev)
+        for two in (False, True):
+            sec = second if two else None
+            nb = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, M, N, K, int(two))
+            work = torch.empty(nb, dtype=torch.uint8, device=dev)
+            fn = lambda: q8.q8_linear_w8a8(x, first, q, ws, s, second=sec, y=y, workspace=work)
+            us = _graph_time(fn, reps)
+            ops = 2.0 * M * N * K * (2 if two else 1)
+            tops = ops / us / 1e6
+            out.append({"M": M, "K": K, "N": N, "two_pass": two, "us": round(us, 1),
+                        "TOPS": round(tops, 1),
+                        "frac_int8_peak": round(tops / int8_peak_tops(peaks), 4)})
+        del x, q, s, ws, y, work
+    return out
+
+
+def bench_q4(dev, peaks, reps=5):
+    """8da4w: x bf16 [M, 4096] (M in 1, 64, 512, 4096), int4 weights [11008, 4096] with
+    fp32 group scales (G in 32, 128); incl. the per-row qparams pre-kernel."""
+    import int8_quantized_linear_q8_b200 as q8
+
+    out = []
+    K, N = wl.Q4_K, wl.Q4_N
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.Q4_SEED_W)
+    W = torch.randn(N, K, generator=g, device=dev) * 0.02
+    for G in wl.Q4_G:
+        q4, gs = q8.q8_quantize_weight_q4gs(W, G)
+        for M in wl.Q4_M:
+            g.manual_seed(wl.Q4_SEED_X + M)
+            x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+            y = torch.empty(M, N, device=dev)
+            nb = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_DQ8CA_Q4GSW, M, N, K, G)
+            work = torch.empty(nb, dtype=torch.uint8, device=dev)
+            fn = lambda: q8.q8_linear_dq8ca_q4gsw(x, q4, gs, G, y=y, workspace=work)
+            us = _graph_time(fn, reps if M >= 512 else 4 * reps)
+            ops = 2.0 * M * N * K
+            byts = N * K // 2 + 4 * N * (K // G) + 2 * M * K + 4 * M * N
+            out.append({"M": M, "G": G, "us": round(us, 2), "TOPS": round(ops / us / 1e6, 2),
+                        "GBps": round(byts / us / 1e3, 1),
+                        "frac_int8_peak": round(ops / us / 1e6 / int8_peak_tops(peaks), 4),
+                        "frac_hbm": round(byts / us / 1e3 / peaks["hbm_gbs"], 4)})
+    return out
+
+
+def bench_quantizers(dev, peaks, reps=5):
+    """The quantizers as HBM streams: weight codes (fp32 32000x4096 in), per-row activation
+    qparams + codes (bf16 4096x4096), static activation codes with the residual pass
+    (fp32 4096x4096)."""
+    import int8_quantized_linear_q8_b200 as q8
+
+    g = torch.Generator(device=dev)
+    g.manual_seed(77)
+    out = []
+    W = torch.randn(32000, 4096, generator=g, device=dev) * 0.02
+    q = torch.empty(32000, 4096, dtype=torch.int8, device=dev)
+    sw = torch.empty(32000, device=dev)
+    ws = torch.empty(32000, dtype=torch.int32, device=dev)
+    us = _graph_time(lambda: q8.q8_quantize_weight(W, q=q, s_w=sw, wsum=ws), reps)
+    b = 32000 * 4096 * 5 + 32000 * 8
+    out.append({"op": "quantize_weight", "shape": [32000, 4096], "us": round(us, 1),
+                "GBps": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / peaks["hbm_gbs"], 4)})
+    del W, q
+    xb = torch.randn(4096, 4096, generator=g, device=dev).to(torch.bfloat16)
+    s = torch.empty(4096, device=dev)
+    z = torch.empty(4096, dtype=torch.int32, device=dev)
+    xq = torch.empty(4096, 4096, dtype=torch.int8, device=dev)
+    us = _graph_time(lambda: q8.q8_choose_qparams(xb, s=s, z=z, xq=xq), reps)
+    b = 4096 * 4096 * 3 + 4096 * 8
+    out.append({"op": "choose_qparams", "shape": [4096, 4096], "us": round(us, 1),
+                "GBps": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / peaks["hbm_gbs"], 4)})
+    xf = torch.randn(4096, 4096, generator=g, device=dev) * 4
+    xq2 = torch.empty(4096, 4096, dtype=torch.int8, device=dev)
+    us = _graph_time(lambda: q8.q8_quantize_static(xf, (0.05, 3), (0.05 / 255, 0), xq1=xq, xq2=xq2),
+                     reps)
+    b = 4096 * 4096 * 6
+    out.append({"op": "quantize_static_two_pass", "shape": [4096, 4096], "us": round(us, 1),
+                "GBps": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / peaks["hbm_gbs"], 4)})
+    return out
+
+
+def bench_llama_stack(dev, peaks, prefill=True):
+    """Llama-shaped stack, 32 layers x (q, k, v, o 4096x4096; gate, up 4096->11008; down
+    11008->4096): decode at M = 1 through the W8A16 GEMV (6.5 GB of int8 weights per pass,
+    one CUDA graph of 224 launches) and prefill at M = 4096 through the W8A8 GEMM."""
+    import int8_quantized_linear_q8_b200 as q8
+
+    g = torch.Generator(device=dev)
+    layers = []
+    for li in range(wl.LLAMA_LAYERS):
+        lin = []
+        for j, (name, K, N) in enumerate(wl.LLAMA_LINEARS):
+            g.manual_seed(8 + li * 16 + j)
+            W = torch.randn(N, K, generator=g, device=dev) * 0.02
+            q, s, ws = q8.q8_quantize_weight(W)
+            del W
+            lin.append((K, N, q, s, ws))
+        layers.append(lin)
+    wbytes = sum(K * N for lin in layers for (K, N, _, _, _) in lin)
+    res = {"layers": wl.LLAMA_LAYERS, "weight_bytes": wbytes}
+    # decode
+    xs = {K: torch.randn(1, K, generator=g, device=dev).to(torch.bfloat16) for K in (4096, 11008)}
+    ys = {N: torch.empty(1, N, dtype=torch.bfloat16, device=dev) for N in (4096, 11008)}
+
+    def decode():
+        for lin in layers:
+            for (K, N, q, s, ws) in lin:
+                q8.q8_linear_w8a16(xs[K], q, s, y=ys[N])
+
+    us = _graph_time(decode, 1)
+    byts = sum(K * N + 4 * N + 2 * K + 2 * N for lin in layers for (K, N, _, _, _) in lin)
+    res["decode"] = {"M": 1, "us_per_pass": round(us, 1), "GBps": round(byts / us / 1e3, 1),
+                     "frac_hbm": round(byts / us / 1e3 / peaks["hbm_gbs"], 4),
+                     "launches": 7 * wl.LLAMA_LAYERS}
+    if prefill:
+        M = wl.LLAMA_PREFILL_M
+        xf = {K: torch.randn(M, K, generator=g, device=dev) for K in (4096, 11008)}
+        qp = {}
+        mm = torch.empty(2, device=dev)
+        for K, x in xf.items():
+            q8.q8_observe_minmax(x, mm, reset=True)
+            qp[K] = q8.q8_qparams_from_minmax(*mm.cpu().tolist())
+        yf = {N: torch.empty(M, N, device=dev) for N in (4096, 11008)}
+        work = torch.empty(q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, M, 4096, 11008, 0),
+                           dtype=torch.uint8, device=dev)
+
+        def pre():
+            for lin in layers:
+                for (K, N, q, s, ws) in lin:
+                    q8.q8_linear_w8a8(xf[K], qp[K], q, ws, s, y=yf[N], workspace=work)
+
+        us = _graph_time(pre, 1)
+        ops = sum(2.0 * M * N * K for lin in layers for (K, N, _, _, _) in lin)
+        res["prefill"] = {"M": M, "ms_per_pass": round(us / 1e3, 2),
+                          "TOPS": round(ops / us / 1e6, 1),
+                          "frac_int8_peak": round(ops / us / 1e6 / int8_peak_tops(peaks), 4),
+                          "launches": 2 * 7 * wl.LLAMA_LAYERS}
+        del xf, yf, work
+    del layers
+    torch.cuda.empty_cache()
+    return res
+
+
 def _graph_time(fn, reps):
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -415,7 +595,10 @@ def run_ours(args):
     q8.lib()
 
     sweep = W8A16Sweep(dev)
-    graphs = sweep.graphs()
+    if args.eager:
+        graphs = [_EagerStep(sweep, c) for c in range(sweep.COPIES)]
+    else:
+        graphs = sweep.graphs()
     clk = ClockSampler(dist.local)
     clk.start()
     ms, t0, t1 = time_graphs(graphs, args.steps, args.warmup, dist)
@@ -436,7 +619,8 @@ def run_ours(args):
         "config": {"workload": "W8A16 decode sweep: bf16 x [M,K] (M in 1,4,16) times int8 "
                                "W [N,K], (K,N) in (960,2560),(2048,8192),(4096,11008),"
                                "(4096,32000); bf16 out",
-                   "step": "12 GEMV launches (every shape x M), one CUDA graph",
+                   "step": "12 GEMV launches (every shape x M), " +
+                           ("launched eagerly" if args.eager else "one CUDA graph"),
                    "bytes_per_step": sweep.step_bytes,
                    "l2": f"inputs larger than L2: {sweep.COPIES} rotating weight copies "
                          f"({sweep.weight_bytes / 1e6:.0f} MB) vs 126 MB L2; M-major order",
@@ -449,13 +633,19 @@ def run_ours(args):
         "gpu_launches": args.steps * len(sweep.cases),
         "clocks": clocks,
     }
-    if dist.rank == 0:
+    if dist.rank == 0 and not args.eager:
         result["cases"] = per_case_times(sweep)
     result["e2e"] = e2e_w8a16(sweep, max(10, min(args.steps // 10, 200)), 3, dist)
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline_w8a16(sweep)
     if dist.rank == 0 and not args.no_paths:
-        result["paths"] = {"w8a8_static_k960": bench_w8a8_paths(dev)}
+        result["paths"] = {
+            "w8a8_static_k960": bench_w8a8_paths(dev),
+            "w8a8_prefill_m4096": bench_w8a8_prefill(dev, peaks),
+            "dq8ca_q4gsw": bench_q4(dev, peaks),
+            "quantizers": bench_quantizers(dev, peaks),
+            "llama_stack": bench_llama_stack(dev, peaks),
+        }
     dist.barrier()
     if dist.rank == 0:
         print(json.dumps(result), flush=True)
@@ -523,11 +713,19 @@ def run_profile(args):
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         for _ in range(args.reps):
             q8.q8_linear_w8a16(x, q, s, y=y)
-    else:
+    elif args.profile == "w8a8":
         x = torch.randn(M, K, generator=g, device=dev) * 4
         y = torch.empty(M, N, device=dev)
         for _ in range(args.reps):
             q8.q8_linear_w8a8(x, (0.05, 3), q, ws, s, second=(0.05 / 255, 0), y=y)
+    else:
+        W = torch.randn(N, K, generator=g, device=dev) * 0.02
+        q4, gs = q8.q8_quantize_weight_q4gs(W, 32)
+        del W
+        x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(M, N, device=dev)
+        for _ in range(args.reps):
+            q8.q8_linear_dq8ca_q4gsw(x, q4, gs, 32, y=y)
     torch.cuda.synchronize()
     print(json.dumps({"profile": args.profile, "M": M, "N": N, "K": K, "reps": args.reps}))
 

@@ -1,0 +1,354 @@
+// k_q4_tc.cu -- the 8da4w linear for prefill-sized M on the tcgen05 tensor cores.
+//
+//   y[m, n] = s[m] * sum_g gs[n, g] * T_g[m, n],   T_g = sum_{k in g} (xq[m,k] - z[m]) q4[n,k]
+//
+// The group scale gs[n, g] multiplies every group partial, so the integer sums must leave
+// the tensor core once per group.  Doing that from an int8 MMA would cost three ALU
+// operations per output element per group (zero-point term, conversion, scale); here the
+// operands enter a bf16 MMA as exact small integers instead -- the codes q4 in [-8, 7] and
+// the shifted activation codes (xq - z) in [-255, 255] -- so every product is exact and
+// each group partial is an integer below 2^24 (|T_g| <= 256 * 255 * 8), exact in the fp32
+// accumulator.  The epilogue then needs one fp32 multiply-add per element and group.
+//
+// Operands (prepared by the two kernels below, into the caller's workspace):
+//   A = weights  bf16 [N, K]  (each int4 code as a bf16 integer)
+//   B = acts     bf16 [M, K]  (xq - z per row, from k_choose_qparams_shifted)
+// Swapped roles: the MMA's M dimension is the weight row n (tensor-memory lane), its N
+// dimension the activation row m, so an epilogue thread owns one weight row and its
+// group scales are per-thread scalars.
+//
+// Structure (persistent, one CTA per SM, 6 warps): warp 0 TMA producer (128-byte swizzle,
+// 6-stage ring of 32 KB: 128 weight rows + 128 activation rows x 64 K elements);
+// warp 1 tensor-memory allocator and MMA issuer (kind::f16, M = 128, N = BN, K = 16) --
+// one group's MMAs go into one of two accumulator buffers, tcgen05.commit hands it to
+// the epilogue; warps 2-5 epilogue: tcgen05.ld of the group partials, fp32 multiply-add
+// with the group scale into per-thread registers, at the end of a tile y = s[m] * acc.
+#include "q8_kernels.cuh"
+
+namespace q8 {
+
+// ------------------------------------------------------------- operand preparation
+
+// Packed int4 codes [N, K/2] -> bf16 integers [N, K] (16 codes per thread step).
+__global__ __launch_bounds__(256) void k_q4_expand_bf16(const uint8_t* __restrict__ q4,
+                                                         int64_t n8, uint16_t* __restrict__ wb) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint2 p = __ldg(reinterpret_cast<const uint2*>(q4) + i);   // 16 codes
+        const uint32_t w[2] = {p.x, p.y};
+        uint32_t o[8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int byte = (int)((w[h] >> (8 * b)) & 0xFFu);
+                const int lo = (byte & 0x8) ? (byte & 0xF) - 16 : (byte & 0xF);
+                const int hi = (byte & 0x80) ? ((byte >> 4) & 0xF) - 16 : ((byte >> 4) & 0xF);
+                const uint32_t blo = __float_as_uint((float)lo) >> 16;   // exact in bf16
+                const uint32_t bhi = __float_as_uint((float)hi) >> 16;
+                o[h * 4 + b] = blo | (bhi << 16);
+            }
+        uint4* dst = reinterpret_cast<uint4*>(wb) + 2 * i;
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+// ----------------------------------------------------------------- the GEMM kernel
+constexpr int QT_BM = 128;             // weight rows per tile (tensor-memory lanes)
+constexpr int QT_BK = 64;              // bf16 K elements per stage (128 bytes)
+constexpr int QT_UK = 16;              // K per tcgen05.mma.kind::f16
+constexpr int QT_STAGES = 6;
+constexpr int QT_THREADS = 192;
+
+template <int BN>
+struct QtCfg {
+    static constexpr int A_BYTES = QT_BM * QT_BK * 2;      // 16 KB
+    static constexpr int B_BYTES = BN * QT_BK * 2;
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+    static constexpr size_t SMEM = (size_t)QT_STAGES * STAGE + 4096;
+};
+
+__host__ __device__ constexpr uint32_t qt_idesc_bf16(int M, int N) {
+    // kind::f16: fp32 accumulator (bit 4), A and B bf16 (bits 7 and 10), both K-major
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint64_t qt_desc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+__device__ __forceinline__ void qt_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    const uint32_t z = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z),
+        "r"(z), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void qt_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void qt_ld32(uint32_t taddr, float (&r)[32]) {
+    uint32_t u[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+          "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
+          "=r"(u[13]), "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]),
+          "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]),
+          "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]),
+          "=r"(u[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
+}
+
+template <int BN>
+__global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
+    const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+    const float* __restrict__ gs, const float* __restrict__ s, float* __restrict__ y, int G,
+    int M, int N, int K, int* status) {
+    using C = QtCfg<BN>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* ctrl = smem + (size_t)QT_STAGES * C::STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
+    uint64_t* empty = full + QT_STAGES;
+    uint64_t* tfull = empty + QT_STAGES;     // [2] group accumulator ready
+    uint64_t* tempty = tfull + 2;            // [2] group accumulator drained
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* s_tile = reinterpret_cast<float*>(ctrl + 512);      // [BN] activation-row scales
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_n = (N + QT_BM - 1) / QT_BM;                  // weight-row tiles
+    const int num_m = (M + BN - 1) / BN;                        // activation-row tiles
+    const int tiles = num_n * num_m;
+    const int nk = K / QT_BK;                                   // K % 128 == 0
+    const int steps_per_group = G / QT_UK;
+    const int ngroups = K / G;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < QT_STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem_base = *tmem_slot;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            tma_prefetch_desc(&amap);
+            tma_prefetch_desc(&bmap);
+            int st = 0, it = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int n0 = (t / num_m) * QT_BM, m0 = (t % num_m) * BN;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&empty[st], ph ^ 1u, status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* base = smem + (size_t)st * C::STAGE;
+                    mbar_expect_tx(&full[st], (uint32_t)C::STAGE);
+                    // the tensor maps view the bf16 matrices as bytes: K offset in bytes
+                    tma_load_2d(base, &amap, kb * QT_BK * 2, n0, &full[st]);
+                    tma_load_2d(base + C::A_BYTES, &bmap, kb * QT_BK * 2, m0, &full[st]);
+                    ++it;
+                    if (++st == QT_STAGES) { st = 0; ph ^= 1u; }
+                }
+            }
+            for (int i = max(0, it - QT_STAGES); i < it; ++i)
+                mbar_drain(&full[i % QT_STAGES], (uint32_t)(i / QT_STAGES) & 1u);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = qt_idesc_bf16(QT_BM, BN);
+            int st = 0, buf = 0;
+            uint32_t ph = 0, bph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                int step = 0;                                   // MMA step within the tile
+                for (int kb = 0; kb < nk && ok; ++kb) {
+                    if (!mbar_wait(&full[st], ph, status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const uint32_t base = smem_u32(smem + (size_t)st * C::STAGE);
+                    const uint64_t a = qt_desc_sw128(base);
+                    const uint64_t b = qt_desc_sw128(base + C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < QT_BK / QT_UK; ++k, ++step) {
+                        const int in_group = step % steps_per_group;
+                        if (in_group == 0) {
+                            // a new group: wait until the epilogue has drained this buffer
+                            if (!mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                        }
+                        qt_mma_f16(tmem_base + (uint32_t)(buf * BN), a + 2 * k, b + 2 * k, idesc,
+                                   in_group != 0);
+                        if (in_group == steps_per_group - 1) {
+                            qt_commit(&tfull[buf]);             // group partial ready
+                            if (++buf == 2) { buf = 0; bph ^= 1u; }
+                        }
+                    }
+                    qt_commit(&empty[st]);                      // stage free after these MMAs
+                    if (++st == QT_STAGES) { st = 0; ph ^= 1u; }
+                }
+            }
+            qt_commit(mma_done);
+            mbar_drain(mma_done, 0);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int q = warp & 3;                 // tensor-memory lane quarter
+        const int et = threadIdx.x - 64;        // 0..127
+        int buf = 0;
+        uint32_t bph = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+            const int n0 = (t / num_m) * QT_BM, m0 = (t % num_m) * BN;
+            const int n = n0 + q * 32 + lane;   // this thread's weight row
+            for (int j = et; j < BN; j += 128) s_tile[j] = (m0 + j < M) ? __ldg(s + m0 + j) : 0.f;
+            const float* gsr = gs + (int64_t)(n < N ? n : 0) * ngroups;
+            float acc[BN];
+#pragma unroll
+            for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
+            bool live = true;
+            float gnext = __ldg(gsr);
+            for (int gi = 0; gi < ngroups; ++gi) {
+                const float gcur = gnext;
+                if (gi + 1 < ngroups) gnext = __ldg(gsr + gi + 1);   // overlap with the MMA
+                const bool okw = mbar_wait(&tfull[buf], bph, status, abort_flag);
+                live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                if (live) {
+                    const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c) {
+                        float r[32];
+                        qt_ld32(taddr + c * 32, r);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(gcur, r[j], acc[c * 32 + j]);
+                    }
+                }
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+                if (++buf == 2) { buf = 0; bph ^= 1u; }
+            }
+            named_bar_sync(2, 128);             // s_tile written by all epilogue threads
+            if (live && n < N) {
+#pragma unroll
+                for (int j = 0; j < BN; ++j)
+                    if (m0 + j < M) y[(int64_t)(m0 + j) * N + n] = s_tile[j] * acc[j];
+            }
+            named_bar_sync(2, 128);             // before s_tile is rewritten
+        }
+    }
+
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ----------------------------------------------------------------------- host side
+static bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                              int box_cols, int box_rows) {
+    // a bf16 [rows, cols] matrix is a uint8 [rows, 2*cols] matrix for the TMA unit
+    return make_tmap_u8_2d(map, base, rows, cols * 2, box_cols * 2, box_rows,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int BN>
+static cudaError_t launch_qt(const uint16_t* wb, const uint16_t* xz, const float* gs,
+                             const float* s, float* y, int G, int M, int N, int K,
+                             cudaStream_t st, int num_sms, int* status) {
+    using C = QtCfg<BN>;
+    CUtensorMap ma, mb;
+    if (!make_tmap_bf16_2d(&ma, wb, N, K, QT_BK, QT_BM)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&mb, xz, M, K, QT_BK, BN)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(k_q4_gemm_tc<BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(C::SMEM + 1024));
+    if (e != cudaSuccess) return e;
+    const int tiles = ((N + QT_BM - 1) / QT_BM) * ((M + BN - 1) / BN);
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(QT_THREADS);
+    cfg.dynamicSmemBytes = C::SMEM + 1024;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_q4_gemm_tc<BN>, ma, mb, gs, s, y, G, M, N, K, status);
+}
+
+cudaError_t launch_q4_expand_bf16(const uint8_t* q4, int64_t N, int K, uint16_t* wb,
+                                  cudaStream_t st, int num_sms) {
+    const int64_t n8 = N * (int64_t)K / 16;       // 8-byte groups of packed codes
+    int64_t blocks = (n8 + 255) / 256;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    k_q4_expand_bf16<<<(unsigned)blocks, 256, 0, st>>>(q4, n8, wb);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const float* gs,
+                              const float* s, float* y, int G, int64_t M, int64_t N, int K,
+                              cudaStream_t st, int num_sms, int* status) {
+    if (M <= 64)
+        return launch_qt<64>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
+    return launch_qt<128>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
+}
+
+}  // namespace q8

@@ -142,6 +142,52 @@ __global__ __launch_bounds__(CQ_THREADS) void k_choose_qparams(const uint16_t* _
     }
 }
 
+// Same qparams, but the codes leave as bf16 integers (xq - z) in [-255, 255] -- the
+// activation operand of the tensor-core 8da4w linear (exact in bf16).
+__global__ __launch_bounds__(CQ_THREADS) void k_choose_qparams_shifted(
+    const uint16_t* __restrict__ x, int K, float* __restrict__ s_out, int32_t* __restrict__ z_out,
+    uint16_t* __restrict__ xz) {
+    __shared__ float red[CQ_THREADS / 32];
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int64_t m = blockIdx.x;
+    const uint16_t* row = x + m * (int64_t)K;
+    const int K8 = K >> 3;
+    float mn = 0.0f, mx = 0.0f;
+    for (int i = threadIdx.x; i < K8; i += CQ_THREADS) {
+        uint4 v = ldg_keep(row + 8 * i);
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float a = bf16lo(w[j]), b = bf16hi(w[j]);
+            mn = fminf(mn, fminf(a, b));
+            mx = fmaxf(mx, fmaxf(a, b));
+        }
+    }
+    mn = block_min<CQ_THREADS>(mn, red);
+    mx = block_max<CQ_THREADS>(mx, red);
+    float s, zf;
+    qparams_from_range(mn, mx, s, zf);
+    if (threadIdx.x == 0) {
+        s_out[m] = s;
+        z_out[m] = __float2int_rn(zf);
+    }
+    const float inv = __fdiv_rn(1.0f, s);
+    const int zi = __float2int_rn(zf);
+    uint4* orow = reinterpret_cast<uint4*>(xz + m * (int64_t)K);
+    for (int i = threadIdx.x; i < K8; i += CQ_THREADS) {
+        uint4 v = ldg_keep(row + 8 * i);
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c0 = act_code(bf16lo(w[j]), inv, zf) - zi;
+            const int c1 = act_code(bf16hi(w[j]), inv, zf) - zi;
+            o[j] = (__float_as_uint((float)c0) >> 16) | (__float_as_uint((float)c1) & 0xFFFF0000u);
+        }
+        orow[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
 // ---------------------------------------------------- static activation codes (a3)
 // Elementwise over M*K values (16 per thread per step).
 __global__ __launch_bounds__(256) void k_quantize_static(const float* __restrict__ x, int64_t n16,
@@ -272,6 +318,12 @@ cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int8_t* q, 
 cudaError_t launch_choose_qparams(const uint16_t* x, int64_t M, int K, float* s, int32_t* z,
                                   int8_t* xq, cudaStream_t st) {
     k_choose_qparams<<<(unsigned)M, CQ_THREADS, 0, st>>>(x, K, s, z, xq);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_choose_qparams_shifted(const uint16_t* x, int64_t M, int K, float* s,
+                                          int32_t* z, uint16_t* xz, cudaStream_t st) {
+    k_choose_qparams_shifted<<<(unsigned)M, CQ_THREADS, 0, st>>>(x, K, s, z, xz);
     return cudaGetLastError();
 }
 

@@ -120,16 +120,26 @@ static W8A8Plan plan_w8a8(int64_t M, int64_t K, int two) {
     return p;
 }
 
+// Activation rows up to which the 8da4w linear runs as a GEMV on the packed int4 weights;
+// above it the weights are expanded once per call to bf16 integers and the tensor-core
+// GEMM runs (see k_q4_tc.cu).
+constexpr int64_t kQ4GemvMaxM = 16;
+
 struct Q4Plan {
-    size_t xq = 0, s = 0, z = 0, bytes = 0;
+    bool tc = false;
+    size_t xq = 0, s = 0, z = 0, wb = 0, bytes = 0;
 };
-static Q4Plan plan_q4(int64_t M, int64_t K) {
+static Q4Plan plan_q4(int64_t M, int64_t N, int64_t K) {
     Q4Plan p;
     if (M <= 0) return p;
+    p.tc = M > kQ4GemvMaxM;
+    // GEMV path: int8 codes [M, K]; tensor-core path: bf16 (xq - z) [M, K] + bf16 weights
+    const size_t codes = (size_t)M * (size_t)K * (p.tc ? 2 : 1);
     p.xq = 0;
-    p.s = align_up((size_t)M * (size_t)K, 256);
+    p.s = align_up(codes, 256);
     p.z = p.s + align_up((size_t)M * 4, 256);
-    p.bytes = p.z + align_up((size_t)M * 4, 256);
+    p.wb = p.z + align_up((size_t)M * 4, 256);
+    p.bytes = p.wb + (p.tc ? align_up((size_t)N * (size_t)K * 2, 256) : 0);
     return p;
 }
 static inline bool valid_group(int G) { return G == 32 || G == 64 || G == 128 || G == 256; }
@@ -264,7 +274,7 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) 
         case Q8_OP_LINEAR_W8A8: return plan_w8a8(M, K, extra != 0).bytes;
         case Q8_OP_LINEAR_DQ8CA_Q4GSW:
             if (!valid_group(extra) || K % 128 != 0 || K % extra != 0) return 0;
-            return plan_q4(M, K).bytes;
+            return plan_q4(M, N, K).bytes;
     }
     return 0;
 }
@@ -311,15 +321,24 @@ q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* g
     if (M == 0) return Q8_OK;
     if (!x || !q4 || !gs || !y) return Q8_ERR_NULL;
     if (!aligned16(x) || !aligned16(q4) || !aligned16(gs) || !aligned16(y)) return Q8_ERR_ALIGN;
-    const Q4Plan plan = plan_q4(M, K);
+    const Q4Plan plan = plan_q4(M, N, K);
     if (!workspace || ws_bytes < plan.bytes) return Q8_ERR_WORKSPACE;
     if (!aligned16(workspace)) return Q8_ERR_ALIGN;
     int sms = 0;
-    Q8_TRY(current_device(sms));
+    int* status = nullptr;
+    Q8_TRY(current_device(sms, &status));
     cudaStream_t st = (cudaStream_t)stream;
-    int8_t* xq = (int8_t*)workspace + plan.xq;
-    float* s = (float*)((uint8_t*)workspace + plan.s);
-    int32_t* z = (int32_t*)((uint8_t*)workspace + plan.z);
+    uint8_t* ws = (uint8_t*)workspace;
+    float* s = (float*)(ws + plan.s);
+    int32_t* z = (int32_t*)(ws + plan.z);
+    if (plan.tc) {
+        uint16_t* xz = (uint16_t*)(ws + plan.xq);
+        uint16_t* wb = (uint16_t*)(ws + plan.wb);
+        Q8_TRY(launched(launch_q4_expand_bf16(q4, N, (int)K, wb, st, sms)));
+        Q8_TRY(launched(launch_choose_qparams_shifted((const uint16_t*)x, M, (int)K, s, z, xz, st)));
+        return launched(launch_q4_gemm_tc(wb, xz, gs, s, y, G, M, N, (int)K, st, sms, status));
+    }
+    int8_t* xq = (int8_t*)(ws + plan.xq);
     Q8_TRY(launched(launch_choose_qparams((const uint16_t*)x, M, (int)K, s, z, xq, st)));
     return launched(launch_q4_gemv(xq, s, z, q4, gs, G, y, M, N, (int)K, st));
 }

@@ -41,6 +41,8 @@ cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int8_t* q, 
                                    int32_t* wsum, cudaStream_t st);
 cudaError_t launch_choose_qparams(const uint16_t* x, int64_t M, int K, float* s, int32_t* z,
                                   int8_t* xq, cudaStream_t st);
+cudaError_t launch_choose_qparams_shifted(const uint16_t* x, int64_t M, int K, float* s,
+                                          int32_t* z, uint16_t* xz, cudaStream_t st);
 cudaError_t launch_quantize_static(const float* x, int64_t M, int K, float s1, int z1, int has2,
                                    float s2, int z2, int8_t* xq1, int8_t* xq2, cudaStream_t st,
                                    int num_sms);
@@ -69,6 +71,13 @@ cudaError_t launch_w8a8_tc(const int8_t* xq1, const int8_t* xq2, float s1, int z
 cudaError_t launch_q4_gemv(const int8_t* xq, const float* s, const int32_t* z, const uint8_t* q4,
                            const float* gs, int G, float* y, int64_t M, int64_t N, int K,
                            cudaStream_t st);
+
+// k_q4_tc.cu
+cudaError_t launch_q4_expand_bf16(const uint8_t* q4, int64_t N, int K, uint16_t* wb,
+                                  cudaStream_t st, int num_sms);
+cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const float* gs,
+                              const float* s, float* y, int G, int64_t M, int64_t N, int K,
+                              cudaStream_t st, int num_sms, int* status);
 
 // k_gemv.cu
 cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w, void* y,

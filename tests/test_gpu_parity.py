@@ -310,3 +310,24 @@ def test_dq8ca_q4gsw_ragged(M, N, K, G):
     s, z, xq = oracle.choose_qparams(wl.bf16_bits(x))
     y64, absum = oracle.linear_dq8ca_q4gsw(xq, s, z, q4, gs, G)
     check_f32(y, y64, absum, f"8da4w ragged M={M} N={N} K={K} G={G}")
+
+
+def test_dq8ca_tensor_core_group_partials_exact():
+    """One group (G = K = 256) with unit group scales: y / s must be the exact integer
+    sum_k (xq - z) q4 -- the bf16 tensor-core path keeps every group partial exact."""
+    M, N, K, G = 300, 200, 256, 256
+    g = torch.Generator().manual_seed(4242)
+    x = wl.normal_bf16((M, K), 1.0, seed=4243)
+    q4 = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, generator=g)   # any nibbles
+    gs = torch.ones(N, K // G)
+    y = q8.q8_linear_dq8ca_q4gsw(x.to(DEV), q4.to(DEV), gs.to(DEV), G).cpu().numpy()
+    s, z, xq = oracle.choose_qparams(wl.bf16_bits(x))
+    lo = (q4.numpy() & 0xF).astype(np.int64)
+    hi = (q4.numpy() >> 4).astype(np.int64)
+    codes = np.empty((N, K), np.int64)
+    codes[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+    codes[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+    T = (xq.astype(np.int64) - z[:, None]) @ codes.T
+    assert np.abs(T).max() < 2 ** 24
+    want = s.astype(np.float32)[:, None] * T.astype(np.float32)      # one fp32 rounding
+    assert np.array_equal(y, want)
