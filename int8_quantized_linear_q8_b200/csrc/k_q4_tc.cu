@@ -60,16 +60,30 @@ constexpr int QT_BM = 128;             // weight rows per tile (tensor-memory la
 constexpr int QT_BK = 64;              // bf16 K elements per stage (128 bytes)
 constexpr int QT_UK = 16;              // K per tcgen05.mma.kind::f16
 constexpr int QT_STAGES = 6;
-constexpr int QT_THREADS = 192;
+constexpr int QT_EPI_WARPS = 8;       // two per tensor-memory lane quarter (column halves)
+constexpr int QT_THREADS = (2 + QT_EPI_WARPS) * 32;
+constexpr int QT_NBUF_MAX = 4;        // group accumulator buffers in tensor memory (<= 512 cols)
 
 template <int BN>
 struct QtCfg {
     static constexpr int A_BYTES = QT_BM * QT_BK * 2;      // 16 KB
     static constexpr int B_BYTES = BN * QT_BK * 2;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+    static constexpr int NBUF = 512 / BN < QT_NBUF_MAX ? 512 / BN : QT_NBUF_MAX;
+    static constexpr int TMEM_COLS = NBUF * BN < 32 ? 32 : NBUF * BN;
+    static_assert(NBUF >= 2 && NBUF * BN <= 512, "tensor memory");
+    static constexpr int HALF = BN / 2;                    // columns per epilogue warp
     static constexpr size_t SMEM = (size_t)QT_STAGES * STAGE + 4096;
 };
+
+// acc.xy += g * r.xy as one packed fp32x2 multiply-add
+__device__ __forceinline__ void ffma2(float& ax, float& ay, float g, float rx, float ry) {
+    asm("{\n\t.reg .b64 p, q, c;\n\t"
+        "mov.b64 p, {%2, %2};\n\tmov.b64 q, {%3, %4};\n\tmov.b64 c, {%0, %1};\n\t"
+        "fma.rn.f32x2 c, p, q, c;\n\tmov.b64 {%0, %1}, c;\n\t}"
+        : "+f"(ax), "+f"(ay)
+        : "f"(g), "f"(rx), "f"(ry));
+}
 
 __host__ __device__ constexpr uint32_t qt_idesc_bf16(int M, int N) {
     // kind::f16: fp32 accumulator (bit 4), A and B bf16 (bits 7 and 10), both K-major
@@ -97,6 +111,20 @@ __device__ __forceinline__ void qt_commit(uint64_t* bar) {
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_u32(bar))
         : "memory");
+}
+// Issue a 32-column tensor-memory load; the caller waits once for a batch of them.
+__device__ __forceinline__ void qt_ld32_nowait(uint32_t taddr, uint32_t (&u)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+          "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
+          "=r"(u[13]), "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]),
+          "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]),
+          "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]),
+          "=r"(u[31])
+        : "r"(taddr));
 }
 __device__ __forceinline__ void qt_ld32(uint32_t taddr, float (&r)[32]) {
     uint32_t u[32];
@@ -127,12 +155,13 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
     uint8_t* ctrl = smem + (size_t)QT_STAGES * C::STAGE;
     uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
     uint64_t* empty = full + QT_STAGES;
-    uint64_t* tfull = empty + QT_STAGES;     // [2] group accumulator ready
-    uint64_t* tempty = tfull + 2;            // [2] group accumulator drained
-    uint64_t* mma_done = tempty + 2;
+    uint64_t* tfull = empty + QT_STAGES;     // [NBUF] group accumulator ready
+    uint64_t* tempty = tfull + C::NBUF;      // [NBUF] group accumulator drained
+    uint64_t* mma_done = tempty + C::NBUF;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* s_tile = reinterpret_cast<float*>(ctrl + 512);      // [BN] activation-row scales
+    static_assert(512 + 4 * BN <= 4096, "control region");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_n = (N + QT_BM - 1) / QT_BM;                  // weight-row tiles
@@ -147,9 +176,9 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < C::NBUF; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 4);
+            mbar_init(&tempty[a], QT_EPI_WARPS);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -174,6 +203,10 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
         if (lane == 0) {
             tma_prefetch_desc(&amap);
             tma_prefetch_desc(&bmap);
+            // Activation tiles are re-read by every weight tile: keep them in L2; weight
+            // tiles are re-read only by the next few activation tiles; outputs stream out.
+            const uint64_t keep = make_l2_policy_evict_last();
+            const uint64_t drop = make_l2_policy_evict_first();
             int st = 0, it = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -187,8 +220,8 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                     uint8_t* base = smem + (size_t)st * C::STAGE;
                     mbar_expect_tx(&full[st], (uint32_t)C::STAGE);
                     // the tensor maps view the bf16 matrices as bytes: K offset in bytes
-                    tma_load_2d(base, &amap, kb * QT_BK * 2, n0, &full[st]);
-                    tma_load_2d(base + C::A_BYTES, &bmap, kb * QT_BK * 2, m0, &full[st]);
+                    tma_load_2d_hint(base, &amap, kb * QT_BK * 2, n0, &full[st], drop);
+                    tma_load_2d_hint(base + C::A_BYTES, &bmap, kb * QT_BK * 2, m0, &full[st], keep);
                     ++it;
                     if (++st == QT_STAGES) { st = 0; ph ^= 1u; }
                 }
@@ -229,7 +262,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                                    in_group != 0);
                         if (in_group == steps_per_group - 1) {
                             qt_commit(&tfull[buf]);             // group partial ready
-                            if (++buf == 2) { buf = 0; bph ^= 1u; }
+                            if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
                         }
                     }
                     qt_commit(&empty[st]);                      // stage free after these MMAs
@@ -242,48 +275,83 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- epilogue
-        const int q = warp & 3;                 // tensor-memory lane quarter
-        const int et = threadIdx.x - 64;        // 0..127
+        // warp w (2..9): lane quarter (w % 4) of the weight rows, column half (w - 2) / 4
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int et = threadIdx.x - 64;        // 0 .. 32*QT_EPI_WARPS-1
+        constexpr int HC = C::HALF;             // columns owned by this warp
         int buf = 0;
         uint32_t bph = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
             const int n0 = (t / num_m) * QT_BM, m0 = (t % num_m) * BN;
             const int n = n0 + q * 32 + lane;   // this thread's weight row
-            for (int j = et; j < BN; j += 128) s_tile[j] = (m0 + j < M) ? __ldg(s + m0 + j) : 0.f;
+            for (int j = et; j < BN; j += 32 * QT_EPI_WARPS)
+                s_tile[j] = (m0 + j < M) ? __ldg(s + m0 + j) : 0.f;
             const float* gsr = gs + (int64_t)(n < N ? n : 0) * ngroups;
-            float acc[BN];
+            float acc[HC];
 #pragma unroll
-            for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < HC; ++j) acc[j] = 0.0f;
             bool live = true;
-            float gnext = __ldg(gsr);
+            // Group scales stream in chunks of 16 groups, one chunk ahead of their use: a
+            // group's MMAs take ~10^2 cycles, an L2 round trip several hundred.
+            constexpr int GC = 16;
+            float gcur[GC], gnxt[GC];
+            auto load_chunk = [&](float (&dst)[GC], int g0) {
+#pragma unroll
+                for (int i = 0; i < GC; i += 4) {
+                    // rows are 16-byte aligned only when ngroups % 4 == 0
+                    if ((ngroups & 3) == 0 && g0 + i + 3 < ngroups) {
+                        const float4 v = __ldg(reinterpret_cast<const float4*>(gsr + g0 + i));
+                        dst[i] = v.x; dst[i + 1] = v.y; dst[i + 2] = v.z; dst[i + 3] = v.w;
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            dst[i + u] = (g0 + i + u < ngroups) ? __ldg(gsr + g0 + i + u) : 0.f;
+                    }
+                }
+            };
+            load_chunk(gnxt, 0);
             for (int gi = 0; gi < ngroups; ++gi) {
-                const float gcur = gnext;
-                if (gi + 1 < ngroups) gnext = __ldg(gsr + gi + 1);   // overlap with the MMA
+                if (gi % GC == 0) {
+#pragma unroll
+                    for (int i = 0; i < GC; ++i) gcur[i] = gnxt[i];
+                    if (gi + GC < ngroups) load_chunk(gnxt, gi + GC);
+                }
+                float gsel = gcur[0];
+#pragma unroll
+                for (int i = 1; i < GC; ++i) gsel = (gi % GC == i) ? gcur[i] : gsel;
+                const float gcur_v = gsel;
                 const bool okw = mbar_wait(&tfull[buf], bph, status, abort_flag);
                 live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 if (live) {
-                    const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+                    const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
+                                           (uint32_t)(buf * BN + half * HC);
+                    uint32_t u[HC / 32][32];
 #pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) {
-                        float r[32];
-                        qt_ld32(taddr + c * 32, r);
+                    for (int c = 0; c < HC / 32; ++c) qt_ld32_nowait(taddr + c * 32, u[c]);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(gcur, r[j], acc[c * 32 + j]);
-                    }
+                    for (int c = 0; c < HC / 32; ++c)
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2)
+                            ffma2(acc[c * 32 + j], acc[c * 32 + j + 1], gcur_v,
+                                  __uint_as_float(u[c][j]), __uint_as_float(u[c][j + 1]));
                 }
                 asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[buf]);
-                if (++buf == 2) { buf = 0; bph ^= 1u; }
+                if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
             }
-            named_bar_sync(2, 128);             // s_tile written by all epilogue threads
+            named_bar_sync(2, 32 * QT_EPI_WARPS);   // s_tile written by all epilogue threads
             if (live && n < N) {
 #pragma unroll
-                for (int j = 0; j < BN; ++j)
-                    if (m0 + j < M) y[(int64_t)(m0 + j) * N + n] = s_tile[j] * acc[j];
+                for (int j = 0; j < HC; ++j) {
+                    const int m = m0 + half * HC + j;
+                    if (m < M) st_stream_f32(y + (int64_t)m * N + n, s_tile[half * HC + j] * acc[j]);
+                }
             }
-            named_bar_sync(2, 128);             // before s_tile is rewritten
+            named_bar_sync(2, 32 * QT_EPI_WARPS);   // before s_tile is rewritten
         }
     }
 
