@@ -68,19 +68,27 @@ def parse_args():
 
 
 class Dist:
-    def __init__(self, gpus: int):
+    """One process per GPU (replicas: the path has no exchange step).  The process group
+    only carries the barriers around the timed region and the max-over-ranks time; it is
+    NCCL on GPUs and gloo on the host (the multi-rank tests run it on CPU)."""
+
+    def __init__(self, gpus: int, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.dev = torch.device("cuda", self.local) if backend == "nccl" else torch.device("cpu")
         if self.world > 1:
             import torch.distributed as dist
 
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
-                                    device_id=torch.device("cuda", self.local))
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                        device_id=self.dev)
+            else:
+                dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
             self.pg = dist
-        else:
+        elif backend == "nccl":
             torch.cuda.set_device(0)
 
     def barrier(self):
@@ -90,13 +98,18 @@ class Dist:
     def max(self, v: float) -> float:
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device=self.dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def job_throughput(world: int, steps: int, units_per_step: float, max_ms: float) -> float:
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return world * steps * units_per_step / (max_ms * 1e-3)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -623,7 +636,7 @@ def run_ours(args):
     clocks = ClockSampler.summarize(rows, t0, t1) if isinstance(rows, list) else rows
     del graphs
     ms_per_step = ms / args.steps
-    value = dist.world * args.steps * sweep.step_bytes / (ms * 1e-3) / 1e9
+    value = job_throughput(dist.world, args.steps, sweep.step_bytes, ms) / 1e9
     peaks = measured_peaks()
     per_rank_gbps = args.steps * sweep.step_bytes / (ms * 1e-3) / 1e9
 

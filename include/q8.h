@@ -229,6 +229,14 @@ q8_status q8_linear_w8a8_noalloc(const float* x, q8_qparams first, const q8_qpar
                                  const int8_t* q, const int32_t* wsum, const float* s_w,
                                  float* y, int64_t M, int64_t N, int64_t K, void* stream);
 
+/* Self-test of failure detection: launches one CTA that waits on a barrier nothing will
+ * complete, with the given limit (1 us .. 2 s, Q8_ERR_ARG otherwise); the wait gives up,
+ * writes 0 to *result (device int32, 1 would mean the barrier completed) and records the
+ * expiry in the device status word, which q8_last_device_status then returns as
+ * Q8_ERR_DEVICE.  The library's pipelined kernels use the same bounded wait (2 s limit)
+ * on every barrier, so a lost arrival ends a kernel with an error instead of a hang. */
+q8_status q8_selftest_bounded_wait(int64_t limit_ns, int32_t* result, void* stream);
+
 /* Host, synchronising.  Reads and clears the device status word that kernels with
  * bounded waits set when a wait expires (Q8_OK if none did since the last read).
  * Waits for the given stream first. */

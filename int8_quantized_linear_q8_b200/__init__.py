@@ -32,7 +32,7 @@ SYMBOLS = (
     "q8_quantize_static", "q8_observe_minmax", "q8_qparams_from_minmax",
     "q8_quantize_weight_q4gs", "q8_linear_w8a16", "q8_linear_w8a8", "q8_linear_dq8ca_q4gsw",
     "q8_workspace_bytes", "q8_gemm_s8s8_s32", "q8_last_device_status",
-    "q8_linear_w8a8_noalloc",
+    "q8_linear_w8a8_noalloc", "q8_selftest_bounded_wait",
 )
 # Built-in scratch of q8_linear_w8a8_noalloc (bytes).
 Q8_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -92,6 +92,8 @@ def _lib() -> ctypes.CDLL:
     L.q8_gemm_s8s8_s32.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp]
     L.q8_last_device_status.restype = st
     L.q8_last_device_status.argtypes = [_vp]
+    L.q8_selftest_bounded_wait.restype = st
+    L.q8_selftest_bounded_wait.argtypes = [_i64, _vp, _vp]
     L.q8_linear_w8a8_noalloc.restype = st
     L.q8_linear_w8a8_noalloc.argtypes = [_vp, q8_qparams, ctypes.POINTER(q8_qparams), _vp, _vp,
                                          _vp, _vp, _i64, _i64, _i64, _vp]
@@ -323,6 +325,15 @@ def q8_gemm_s8s8_s32(a: torch.Tensor, b: torch.Tensor, acc=None, stream=None) ->
     _check(_lib().q8_gemm_s8s8_s32(_ptr(a), _ptr(b), _ptr(acc), M, N, K, _stream(stream)),
            "q8_gemm_s8s8_s32")
     return acc
+
+
+def q8_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    """Run the bounded-wait self-test kernel; returns the kernel's result flag (0: the
+    wait expired as intended).  Read q8_last_device_status() afterwards."""
+    res = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check(_lib().q8_selftest_bounded_wait(int(limit_ns), _ptr(res), _stream(stream)),
+           "q8_selftest_bounded_wait")
+    return int(res.item())
 
 
 def q8_last_device_status(stream=None) -> int:

@@ -144,6 +144,23 @@ static Q4Plan plan_q4(int64_t M, int64_t N, int64_t K) {
 }
 static inline bool valid_group(int G) { return G == 32 || G == 64 || G == 128 || G == 256; }
 
+// Self-test of the bounded-wait path: one CTA waits on an mbarrier that nothing will ever
+// complete, with a short limit; the wait gives up, records kStatusWaitTimeout in the status
+// word and the kernel returns normally.
+__global__ void k_selftest_bounded_wait(unsigned long long limit_ns, int* status,
+                                        int* result) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const bool ok = mbar_wait_limit(&bar, 0, status, &abort_flag, limit_ns);
+    if (threadIdx.x == 0) *result = ok ? 1 : 0;
+}
+
 }  // namespace q8
 
 using namespace q8;
@@ -356,6 +373,17 @@ q8_status q8_gemm_s8s8_s32(const int8_t* a, const int8_t* b, int32_t* acc, int64
     Q8_TRY(current_device(sms, &status));
     return launched(launch_gemm_s8s8_s32_tc(a, b, acc, M, N, (int)K, (cudaStream_t)stream, sms,
                                            status));
+}
+
+q8_status q8_selftest_bounded_wait(int64_t limit_ns, int32_t* result, void* stream) {
+    if (!result) return Q8_ERR_NULL;
+    if (limit_ns < 1000 || limit_ns > 2000000000LL) return Q8_ERR_ARG;
+    int sms = 0;
+    int* status = nullptr;
+    Q8_TRY(current_device(sms, &status));
+    k_selftest_bounded_wait<<<1, 32, 0, (cudaStream_t)stream>>>((unsigned long long)limit_ns,
+                                                                 status, result);
+    return launched(cudaGetLastError());
 }
 
 q8_status q8_last_device_status(void* stream) {

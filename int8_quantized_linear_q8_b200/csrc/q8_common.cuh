@@ -223,6 +223,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
         }
     }
 }
+// Same bounded wait with a caller-chosen limit (the self-test uses a short one).
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int* status,
+                                                volatile int* abort_flag,
+                                                unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                *abort_flag = 1;
+                atomicExch(status, kStatusWaitTimeout);
+                return false;
+            }
+        }
+    }
+}
 // Bounded wait used only on exit paths: waits for a phase without touching flags.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
     const unsigned long long t0 = globaltimer_ns();

@@ -28,6 +28,24 @@ def _bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
+# ------------------------------------------------------------------ failure detection
+
+
+def test_bounded_wait_reports_and_context_survives():
+    """A barrier nobody completes: the bounded wait gives up after its limit, the host reads
+    Q8_ERR_DEVICE, the status clears, and the next kernel runs normally."""
+    assert q8.q8_last_device_status() == q8.Q8_OK
+    t0 = __import__("time").time()
+    assert q8.q8_selftest_bounded_wait(20_000_000) == 0       # 20 ms limit
+    assert q8.q8_last_device_status() == q8.Q8_ERR_DEVICE
+    assert __import__("time").time() - t0 < 10.0
+    assert q8.q8_last_device_status() == q8.Q8_OK              # read-and-clear
+    W = wl.weight(64, 128, seed=5)
+    q, s, _ = q8.q8_quantize_weight(W.to(DEV))
+    rq, rs, _ = oracle.quantize_weight(W.numpy())
+    assert np.array_equal(q.cpu().numpy(), rq)
+
+
 # ------------------------------------------------------------------- weight codes (a1)
 
 
