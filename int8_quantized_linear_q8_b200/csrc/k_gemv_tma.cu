@@ -11,8 +11,13 @@
 //     [16 rows][256 bytes] (boxes 64 bytes wide stream at about half the rate); stage
 //     readiness is an mbarrier with transaction bytes, stage release an mbarrier the
 //     consumer warps arrive on.
-//   * warps 0-7 (consumers): before the first stage they copy the activations x [M, K]
-//     (bf16, at most 128 KB) into shared memory in MMA-fragment order.  Warp w then takes
+//   * warps 0-7 (consumers): before the first stage they stage the activations x [M, K]
+//     (bf16) in MMA-fragment order, each lane exactly the fragments it will feed to its own
+//     MMAs.  When they fit (32 * stages-per-row-group * ceil(M/8) <= 512 columns) they go
+//     to tensor memory, which this kernel does not otherwise use: warp w owns TMEM lanes
+//     32*(w%4).. and half the columns, and reads its fragments back with tcgen05.ld, so the
+//     shared-memory port carries only the weight stream and the whole ring is free for
+//     stages.  Otherwise they go to shared memory (at most 128 KB).  Warp w then takes
 //     slabs w and w+8 (64 bytes of K each) of every stage, converts the int8 codes to bf16
 //     in registers (exact, 7 ALU ops per 4 codes) and accumulates with the warp-level bf16
 //     MMA (fp32 accumulate).  After the last stage of a row group the 8 partial sums are
@@ -46,18 +51,18 @@ struct WtSmem {
 // Rows of q a CTA may own (its s_w slice is staged in shared memory).
 constexpr int WT_MAX_ROWS = 1024;
 
-static __host__ __device__ inline WtSmem wt_layout(int M, int K, int MT, int stages) {
+static __host__ __device__ inline WtSmem wt_layout(int M, int K, int MT, int stages, bool xt) {
     WtSmem L;
     L.stages = stages;
     L.ring = 0;
     L.xs = (size_t)stages * WT_STAGE_BYTES;
     const int Kpad = (K + WT_SLABS * 64 - 1) / (WT_SLABS * 64) * (WT_SLABS * 64);
-    const size_t xbytes = (size_t)M * Kpad * 2;
+    const size_t xbytes = xt ? 0 : (size_t)M * Kpad * 2;
     L.red = L.xs + ((xbytes + 127) / 128) * 128;
     const size_t redbytes = (size_t)WT_SLOTS * MT * 32 * 4 * sizeof(float);
     L.sws = L.red + redbytes;
     L.bars = L.sws + (size_t)WT_MAX_ROWS * sizeof(float);
-    // barriers, slot counters, abort flag
+    // barriers, slot counters, abort flag, TMEM address
     L.total = L.bars + (size_t)2 * stages * sizeof(uint64_t) + (WT_SLOTS + 4) * sizeof(int);
     return L;
 }
@@ -69,13 +74,39 @@ __device__ __forceinline__ uint32_t xfrag_addr(uint32_t xs, int M, int Kpad, int
     return xs + (uint32_t)h * (uint32_t)(M * Kpad) + (uint32_t)(((c * M + m) * 4 + t) * 16);
 }
 
-template <int MT>
+// Tensor-memory columns the staged activations need: every consumer warp holds 8
+// columns (32 bytes per lane) per chunk it owns (2 per stage) and per 8 activation rows;
+// warps w and w+4 share a lane quarter, so the allocation is twice one warp's share.
+__host__ __device__ inline int wt_tmem_cols(int nst, int MT) { return 32 * nst * MT; }
+constexpr int WT_TMEM_MAX_COLS = 512;
+
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                   "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr));
+}
+// Completes this thread's outstanding tcgen05.ld; the registers are tied to the wait so
+// that no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_wait_ld_x8(uint32_t (&v)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                   "+r"(v[6]), "+r"(v[7])::"memory");
+}
+
+template <int MT, bool XT>
 __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     const __grid_constant__ CUtensorMap wmap, const uint16_t* __restrict__ x,
     const float* __restrict__ s_w, void* __restrict__ y, int y_bf16, int M, int N, int K,
     int stages, int* status) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    const WtSmem L = wt_layout(M, K, MT, stages);
+    const WtSmem L = wt_layout(M, K, MT, stages, XT);
     uint8_t* ring = smem + L.ring;
     float* slots = reinterpret_cast<float*>(smem + L.red);        // [WT_SLOTS][MT][32][4]
     float* sws = reinterpret_cast<float*>(smem + L.sws);          // s_w of this CTA's rows
@@ -83,6 +114,7 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     uint64_t* empty = full + stages;
     int* cnt = reinterpret_cast<int*>(empty + stages);               // [WT_SLOTS]
     volatile int* abort_flag = cnt + WT_SLOTS;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cnt + WT_SLOTS + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nslab = K >> 6;                              // K % 64 == 0
@@ -90,6 +122,10 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     const int RG = (N + 15) >> 4;
     const int rg0 = (int)((int64_t)RG * blockIdx.x / gridDim.x);
     const int rg1 = (int)((int64_t)RG * (blockIdx.x + 1) / gridDim.x);
+    // power-of-two TMEM allocation (>= 32 columns); the launcher checks it is <= 512
+    int tcols = 32;
+    if (XT)
+        while (tcols < wt_tmem_cols(nst, MT)) tcols <<= 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -100,19 +136,25 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (XT && warp == 0) {
+        // One CTA per SM, so the columns are free unless a kernel that ran before this one
+        // still holds them; the allocation waits for it.  Done before the dependent launch
+        // is released, so no kernel that waits on this one can be holding them.
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(tcols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
     for (int i = threadIdx.x; i < WT_SLOTS * MT * 128; i += WT_THREADS) slots[i] = 0.0f;
+    if (XT) asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (XT) asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     // Programmatic dependent launch: let the next kernel on the stream start its own
     // set-up now, and wait for the previous one to finish (and its writes to be
     // visible) before the first global-memory access -- any input may be its output.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    {
-        // The epilogue must not wait on global loads (a stalled warp holds back the ring):
-        // stage this CTA's per-channel scales once.
-        const int row0 = rg0 * 16, rows = min(rg1 * 16, N) - row0;
-        for (int i = threadIdx.x; i < rows; i += WT_THREADS) sws[i] = __ldg(s_w + row0 + i);
-    }
-    __syncthreads();
 
     if (warp == WT_CONSUMERS) {
         // ------------------------------------------------------------- producer
@@ -146,37 +188,97 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     }
 
     // ----------------------------------------------------------------- consumers
+    // The producer starts streaming as soon as the previous kernel is done; the consumers
+    // stage the scales and the activations meanwhile and then meet at barrier 1.
+    {
+        // The epilogue must not wait on global loads (a stalled warp holds back the ring):
+        // stage this CTA's per-channel scales once.
+        const int row0 = rg0 * 16, rows = min(rg1 * 16, N) - row0;
+        for (int i = threadIdx.x; i < rows; i += WT_CONSUMERS * 32) sws[i] = __ldg(s_w + row0 + i);
+    }
+    const int g = lane >> 2, t = lane & 3;
     const int Kpad = nst * WT_SLABS * 64;
     const uint32_t xs = smem_u32(smem + L.xs);
-    {
+    // this warp's TMEM lanes (its quarter) and columns (half h = warp / 4)
+    const uint32_t tm_warp = XT ? *tmem_slot + ((uint32_t)((warp & 3) * 32) << 16) +
+                                      (uint32_t)((warp >> 2) * (wt_tmem_cols(nst, MT) / 2))
+                                : 0u;
+    if (XT) {
+        // Lane (g, t) of warp w feeds, for its local chunk lc (chunk c = 16*(lc/2) + w +
+        // 8*(lc%2), 64 k) and 8-row tile mt, the 16 elements x[m][64c + 16t .. +16] of row
+        // m = 8*mt + g: 8 words in columns (lc*MT + mt)*8 .. +8 of its own lane, element
+        // pairs regrouped to the (even, odd) k pairing of s8x4_to_bf16x2_eo; zero for rows
+        // past M and chunks past K.  The loads of XB stages are issued together, so the
+        // staging costs about nst / XB memory round trips.
+        constexpr int XB = MT == 1 ? 4 : 2;
+        for (int st0 = 0; st0 < nst; st0 += XB) {
+            uint4 v[XB][2][MT][2];
+#pragma unroll
+            for (int b = 0; b < XB; ++b)
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int c = 16 * (st0 + b) + warp + 8 * jj;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const int m = mt * 8 + g;
+                        v[b][jj][mt][0] = v[b][jj][mt][1] = make_uint4(0, 0, 0, 0);
+                        if (m < M && c < nslab) {
+                            const uint16_t* src = x + (int64_t)m * K + 64 * c + 16 * t;
+                            v[b][jj][mt][0] = ldg_keep(src);
+                            v[b][jj][mt][1] = ldg_keep(src + 8);
+                        }
+                    }
+                }
+#pragma unroll
+            for (int b = 0; b < XB; ++b) {
+                if (st0 + b >= nst) break;                   // warp-uniform
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        uint32_t wv[8];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint4 a = v[b][jj][mt][h];
+                            wv[4 * h + 0] = __byte_perm(a.x, a.y, 0x5410);
+                            wv[4 * h + 1] = __byte_perm(a.x, a.y, 0x7632);
+                            wv[4 * h + 2] = __byte_perm(a.z, a.w, 0x5410);
+                            wv[4 * h + 3] = __byte_perm(a.z, a.w, 0x7632);
+                        }
+                        tmem_st_x8(tm_warp + (uint32_t)(((2 * (st0 + b) + jj) * MT + mt) * 8),
+                                   wv);
+                    }
+            }
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    } else {
         // x [M, K] -> fragment order (two planes of 16-byte pieces), element pairs
         // regrouped to the (even, odd) k pairing of s8x4_to_bf16x2_eo; zero past K.
         const int units = M * Kpad / 8;
         const int per_row = Kpad / 8;
         for (int u = threadIdx.x; u < units; u += WT_CONSUMERS * 32) {
             const int m = u / per_row, r = u - m * per_row;
-            const int c = r >> 3, t = (r >> 1) & 3, h = r & 1;
+            const int c = r >> 3, tt = (r >> 1) & 3, h = r & 1;
             uint4 v = make_uint4(0, 0, 0, 0);
             if (8 * r < K) v = ldg_keep(x + (int64_t)m * K + 8 * r);
             const uint32_t p0 = __byte_perm(v.x, v.y, 0x5410), p1 = __byte_perm(v.x, v.y, 0x7632);
             const uint32_t p2 = __byte_perm(v.z, v.w, 0x5410), p3 = __byte_perm(v.z, v.w, 0x7632);
             asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(
-                             xfrag_addr(xs, M, Kpad, c, m, t, h)),
+                             xfrag_addr(xs, M, Kpad, c, m, tt, h)),
                          "r"(p0), "r"(p1), "r"(p2), "r"(p3)
                          : "memory");
         }
     }
     named_bar_sync(1, WT_CONSUMERS * 32);
 
-    const int g = lane >> 2, t = lane & 3;
     // This lane's weight bytes in a stage: slab j (j = warp, warp + 8) lives in box j/4,
     // rows g and g+8, bytes (j%4)*64 + 16t .. +16.  Slab warp+8 is two boxes further.
     const uint32_t ring_u = smem_u32(ring);
     const uint32_t w_off = (uint32_t)((warp >> 2) * 16 * WT_BOX + g * WT_BOX + (warp & 3) * 64 +
                                       t * 16);
     constexpr uint32_t kSlab2 = 2 * 16 * WT_BOX;            // slab j+8 = 2 boxes on
-    // Activation fragments of chunk c = st*16 + j: plane 0 address; +1024*M bytes per
-    // stage; slab j+8 is 8 chunks (8*M*64 bytes) further.
+    // Shared-memory staging: activation fragments of chunk c = st*16 + j, plane 0 address;
+    // +1024*M bytes per stage; slab j+8 is 8 chunks (8*M*64 bytes) further.
     uint32_t x_lane[MT];
     bool x_live[MT];
 #pragma unroll
@@ -186,7 +288,7 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
         x_lane[mt] = xfrag_addr(xs, M, Kpad, warp, x_live[mt] ? m : 0, t, 0);
     }
     const uint32_t plane = (uint32_t)(M * Kpad);
-    const uint32_t x_step = (uint32_t)(WT_SLABS * M * 64);
+    const uint32_t x_step = XT ? (uint32_t)(2 * MT * 8) : (uint32_t)(WT_SLABS * M * 64);
     const uint32_t x_slab2 = (uint32_t)(8 * M * 64);
 
     int s = 0, slot = 0;
@@ -204,27 +306,46 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[c][mt][i] = 0.0f;
 
-        uint32_t xst = 0;                                    // stage offset into x
+        uint32_t xst = 0;                   // stage offset into x (TMEM columns or bytes)
         for (int st = 0; st < nst; ++st) {
+            // xr[jj][mt]: words 0-3 plane 0 (k 16t..16t+7), words 4-7 plane 1 (+8)
+            uint32_t xr[2][MT][8];
+            if (XT) {
+                // the activations do not depend on the stage: read them before waiting
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+                        tmem_ld_x8(tm_warp + xst + (uint32_t)((jj * MT + mt) * 8), xr[jj][mt]);
+            }
             mbar_wait(&full[s], ph, status, abort_flag);   // on expiry: finish with garbage
             uint4 w[2][2];
             w[0][0] = lds128(wst);
             w[0][1] = lds128(wst + 8 * WT_BOX);
             w[1][0] = lds128(wst + kSlab2);
             w[1][1] = lds128(wst + kSlab2 + 8 * WT_BOX);
-            uint4 xa[2][MT][2];
+            if (XT) {
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj)
+                for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    if (x_live[mt]) {
-                        const uint32_t xa_addr = x_lane[mt] + xst + (jj ? x_slab2 : 0u);
-                        xa[jj][mt][0] = lds128(xa_addr);
-                        xa[jj][mt][1] = lds128(xa_addr + plane);
-                    } else {
-                        xa[jj][mt][0] = xa[jj][mt][1] = make_uint4(0, 0, 0, 0);
+                    for (int mt = 0; mt < MT; ++mt) tmem_wait_ld_x8(xr[jj][mt]);
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        uint4 a = make_uint4(0, 0, 0, 0), b = a;
+                        if (x_live[mt]) {
+                            const uint32_t xa_addr = x_lane[mt] + xst + (jj ? x_slab2 : 0u);
+                            a = lds128(xa_addr);
+                            b = lds128(xa_addr + plane);
+                        }
+                        xr[jj][mt][0] = a.x; xr[jj][mt][1] = a.y;
+                        xr[jj][mt][2] = a.z; xr[jj][mt][3] = a.w;
+                        xr[jj][mt][4] = b.x; xr[jj][mt][5] = b.y;
+                        xr[jj][mt][6] = b.z; xr[jj][mt][7] = b.w;
                     }
-                }
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);           // operands are in registers
 #pragma unroll
@@ -237,12 +358,9 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
                     s8x4_to_bf16x2_eo(wav[q], alo, ahi);
                     s8x4_to_bf16x2_eo(wbv[q], blo, bhi);
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        const uint4& xv = xa[jj][mt][q >> 1];
-                        const uint32_t b0 = (q & 1) ? xv.z : xv.x;
-                        const uint32_t b1 = (q & 1) ? xv.w : xv.y;
-                        mma_bf16_16816(acc[(jj * 4 + q) % CH][mt], alo, blo, ahi, bhi, b0, b1);
-                    }
+                    for (int mt = 0; mt < MT; ++mt)
+                        mma_bf16_16816(acc[(jj * 4 + q) % CH][mt], alo, blo, ahi, bhi,
+                                       xr[jj][mt][2 * q], xr[jj][mt][2 * q + 1]);
                 }
             }
             xst += x_step;
@@ -303,6 +421,16 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
         }
         if (++slot == WT_SLOTS) slot = 0;
     }
+    if (XT) {
+        // every tcgen05.ld of every consumer warp has completed (waited on in the loop)
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        named_bar_sync(1, WT_CONSUMERS * 32);
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (warp == 0)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*tmem_slot),
+                         "r"(tcols)
+                         : "memory");
+    }
 }
 
 // ----------------------------------------------------------------------- host side
@@ -345,22 +473,43 @@ bool make_tmap_u8_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t c
     return r == CUDA_SUCCESS;
 }
 
-// Whether the TMA path takes this problem: K % 64 == 0, M <= 16 and the activations fit
-// next to at least 4 ring stages.
-bool w8a16_tma_fits(int64_t M, int64_t K) {
-    if (M < 1 || M > 16 || (K % 64) != 0) return false;
+// Whether the activations go to tensor memory (they need at most 512 columns).  With 9..16
+// rows they always do: in shared memory they would take the room of the ring and double
+// the shared-memory traffic.  With 1..8 rows they do when shared memory cannot hold them
+// next to 8 stages, or when each CTA streams at least 32 stages: setting up tensor memory
+// costs about half a microsecond more per launch (measured on the small shapes), which
+// the lighter shared-memory traffic pays back only on long streams.
+static bool wt_use_tmem(int M, int K, int64_t N, int num_sms) {
     const int MT = M <= 8 ? 1 : 2;
-    return wt_layout((int)M, (int)K, MT, 4).total <= (size_t)WT_MAX_SMEM;
+    const int nst = (K / 64 + WT_SLABS - 1) / WT_SLABS;
+    if (wt_tmem_cols(nst, MT) > WT_TMEM_MAX_COLS) return false;
+    if (MT == 2) return true;
+    if (wt_layout(M, K, 1, 8, false).total > (size_t)WT_MAX_SMEM) return true;
+    const int64_t RG = (N + 15) / 16;
+    const int64_t grid = RG < num_sms ? RG : num_sms;
+    return (RG + grid - 1) / grid * nst >= 32;
 }
 
-template <int MT>
+// Whether the TMA path takes this problem: K % 64 == 0, M <= 16 and the activations fit
+// in tensor memory, or in shared memory next to at least 4 ring stages.
+bool w8a16_tma_fits(int64_t M, int64_t K) {
+    if (M < 1 || M > 16 || (K % 64) != 0 || K > (int64_t)1 << 30) return false;
+    const int MT = M <= 8 ? 1 : 2;
+    const int nst = (int)((K / 64 + WT_SLABS - 1) / WT_SLABS);
+    if (wt_tmem_cols(nst, MT) <= WT_TMEM_MAX_COLS) return true;
+    // (with 9..16 rows, activations too long for tensor memory do not fit shared memory
+    // next to 4 stages either)
+    return MT == 1 && wt_layout((int)M, (int)K, 1, 4, false).total <= (size_t)WT_MAX_SMEM;
+}
+
+template <int MT, bool XT>
 static cudaError_t launch_wt(const CUtensorMap& map, const uint16_t* x, const float* s_w, void* y,
                              int y_bf16, int M, int N, int K, cudaStream_t st, int num_sms,
                              int* status) {
     int stages = 8;    // must stay <= WT_SLOTS - 2
-    while (stages > 4 && wt_layout(M, K, MT, stages).total > (size_t)WT_MAX_SMEM) --stages;
-    const WtSmem L = wt_layout(M, K, MT, stages);
-    cudaError_t e = cudaFuncSetAttribute(k_w8a16_tma<MT>,
+    while (stages > 4 && wt_layout(M, K, MT, stages, XT).total > (size_t)WT_MAX_SMEM) --stages;
+    const WtSmem L = wt_layout(M, K, MT, stages, XT);
+    cudaError_t e = cudaFuncSetAttribute(k_w8a16_tma<MT, XT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L.total);
     if (e != cudaSuccess) return e;
@@ -378,8 +527,8 @@ static cudaError_t launch_wt(const CUtensorMap& map, const uint16_t* x, const fl
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_w8a16_tma<MT>, map, x, s_w, y, y_bf16, M, N, K, stages,
-                              status);
+    return cudaLaunchKernelEx(&cfg, k_w8a16_tma<MT, XT>, map, x, s_w, y, y_bf16, M, N, K,
+                              stages, status);
 }
 
 cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
@@ -388,9 +537,14 @@ cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_
     CUtensorMap map;
     if (!make_tmap_u8_2d(&map, q, N, K, WT_BOX, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
+    const bool xt = wt_use_tmem((int)M, K, N, num_sms);
     if (M <= 8)
-        return launch_wt<1>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms, status);
-    return launch_wt<2>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms, status);
+        return xt ? launch_wt<1, true>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms,
+                                       status)
+                  : launch_wt<1, false>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms,
+                                        status);
+    if (!xt) return cudaErrorInvalidValue;             // excluded by w8a16_tma_fits
+    return launch_wt<2, true>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms, status);
 }
 
 }  // namespace q8
