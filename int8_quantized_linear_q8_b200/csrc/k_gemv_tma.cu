@@ -34,12 +34,20 @@
 
 namespace q8 {
 
-constexpr int WT_CONSUMERS = 8;                         // consumer warps (2 slabs each)
+#ifndef WT_SLABS_DEF
+#define WT_SLABS_DEF 16
+#endif
+constexpr int WT_SLABS = WT_SLABS_DEF;                  // 64-byte slabs per stage
+#ifndef WT_CONSUMERS_DEF
+#define WT_CONSUMERS_DEF 8
+#endif
+constexpr int WT_CONSUMERS = WT_CONSUMERS_DEF;          // consumer warps
+constexpr int WT_SPW = WT_SLABS / WT_CONSUMERS;         // slabs per consumer warp and stage
+static_assert(WT_SPW * WT_CONSUMERS == WT_SLABS && WT_CONSUMERS % 4 == 0, "slab split");
 constexpr int WT_THREADS = (WT_CONSUMERS + 1) * 32;     // + producer warp
-constexpr int WT_SLABS = 16;                            // 64-byte slabs per stage
 constexpr int WT_BOX = 256;                             // TMA box width (bytes of K)
 constexpr int WT_BOXES = WT_SLABS * 64 / WT_BOX;        // boxes per stage
-constexpr int WT_STAGE_BYTES = 16 * 64 * WT_SLABS;      // 16 KB
+constexpr int WT_STAGE_BYTES = 16 * 64 * WT_SLABS;      // 16 rows of WT_SLABS * 64 bytes
 constexpr int WT_MAX_SMEM = 227 * 1024;
 constexpr int WT_SLOTS = 16;                            // rotating partial-sum slots (> stages+1)
 
@@ -77,7 +85,7 @@ __device__ __forceinline__ uint32_t xfrag_addr(uint32_t xs, int M, int Kpad, int
 // Tensor-memory columns the staged activations need: every consumer warp holds 8
 // columns (32 bytes per lane) per chunk it owns (2 per stage) and per 8 activation rows;
 // warps w and w+4 share a lane quarter, so the allocation is twice one warp's share.
-__host__ __device__ inline int wt_tmem_cols(int nst, int MT) { return 32 * nst * MT; }
+__host__ __device__ inline int wt_tmem_cols(int nst, int MT) { return 2 * WT_SLABS * nst * MT; }
 constexpr int WT_TMEM_MAX_COLS = 512;
 
 __device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&v)[8]) {
@@ -199,10 +207,11 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     const int g = lane >> 2, t = lane & 3;
     const int Kpad = nst * WT_SLABS * 64;
     const uint32_t xs = smem_u32(smem + L.xs);
-    // this warp's TMEM lanes (its quarter) and columns (half h = warp / 4)
-    const uint32_t tm_warp = XT ? *tmem_slot + ((uint32_t)((warp & 3) * 32) << 16) +
-                                      (uint32_t)((warp >> 2) * (wt_tmem_cols(nst, MT) / 2))
-                                : 0u;
+    // this warp's TMEM lanes (its quarter) and columns (share warp / 4 of its quarter)
+    const uint32_t tm_warp =
+        XT ? *tmem_slot + ((uint32_t)((warp & 3) * 32) << 16) +
+                 (uint32_t)((warp >> 2) * (wt_tmem_cols(nst, MT) / (WT_CONSUMERS / 4)))
+           : 0u;
     if (XT) {
         // Lane (g, t) of warp w feeds, for its local chunk lc (chunk c = 16*(lc/2) + w +
         // 8*(lc%2), 64 k) and 8-row tile mt, the 16 elements x[m][64c + 16t .. +16] of row
@@ -210,14 +219,14 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
         // pairs regrouped to the (even, odd) k pairing of s8x4_to_bf16x2_eo; zero for rows
         // past M and chunks past K.  The loads of XB stages are issued together, so the
         // staging costs about nst / XB memory round trips.
-        constexpr int XB = MT == 1 ? 4 : 2;
+        constexpr int XB = (MT == 1 ? 8 : 4) / WT_SPW;
         for (int st0 = 0; st0 < nst; st0 += XB) {
-            uint4 v[XB][2][MT][2];
+            uint4 v[XB][WT_SPW][MT][2];
 #pragma unroll
             for (int b = 0; b < XB; ++b)
 #pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {
-                    const int c = 16 * (st0 + b) + warp + 8 * jj;
+                for (int jj = 0; jj < WT_SPW; ++jj) {
+                    const int c = WT_SLABS * (st0 + b) + warp + WT_CONSUMERS * jj;
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
                         const int m = mt * 8 + g;
@@ -233,7 +242,7 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
             for (int b = 0; b < XB; ++b) {
                 if (st0 + b >= nst) break;                   // warp-uniform
 #pragma unroll
-                for (int jj = 0; jj < 2; ++jj)
+                for (int jj = 0; jj < WT_SPW; ++jj)
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
                         uint32_t wv[8];
@@ -245,7 +254,8 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
                             wv[4 * h + 2] = __byte_perm(a.z, a.w, 0x5410);
                             wv[4 * h + 3] = __byte_perm(a.z, a.w, 0x7632);
                         }
-                        tmem_st_x8(tm_warp + (uint32_t)(((2 * (st0 + b) + jj) * MT + mt) * 8),
+                        tmem_st_x8(tm_warp +
+                                       (uint32_t)(((WT_SPW * (st0 + b) + jj) * MT + mt) * 8),
                                    wv);
                     }
             }
@@ -271,12 +281,12 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     }
     named_bar_sync(1, WT_CONSUMERS * 32);
 
-    // This lane's weight bytes in a stage: slab j (j = warp, warp + 8) lives in box j/4,
-    // rows g and g+8, bytes (j%4)*64 + 16t .. +16.  Slab warp+8 is two boxes further.
+    // This lane's weight bytes in a stage: slab j (j = warp + WT_CONSUMERS*jj) lives in
+    // box j/4, rows g and g+8, bytes (j%4)*64 + 16t .. +16.
     const uint32_t ring_u = smem_u32(ring);
     const uint32_t w_off = (uint32_t)((warp >> 2) * 16 * WT_BOX + g * WT_BOX + (warp & 3) * 64 +
                                       t * 16);
-    constexpr uint32_t kSlab2 = 2 * 16 * WT_BOX;            // slab j+8 = 2 boxes on
+    constexpr uint32_t kSlab2 = WT_CONSUMERS / 4 * 16 * WT_BOX;  // slab j+WT_CONSUMERS
     // Shared-memory staging: activation fragments of chunk c = st*16 + j, plane 0 address;
     // +1024*M bytes per stage; slab j+8 is 8 chunks (8*M*64 bytes) further.
     uint32_t x_lane[MT];
@@ -288,15 +298,15 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
         x_lane[mt] = xfrag_addr(xs, M, Kpad, warp, x_live[mt] ? m : 0, t, 0);
     }
     const uint32_t plane = (uint32_t)(M * Kpad);
-    const uint32_t x_step = XT ? (uint32_t)(2 * MT * 8) : (uint32_t)(WT_SLABS * M * 64);
-    const uint32_t x_slab2 = (uint32_t)(8 * M * 64);
+    const uint32_t x_step = XT ? (uint32_t)(WT_SPW * MT * 8) : (uint32_t)(WT_SLABS * M * 64);
+    const uint32_t x_slab2 = (uint32_t)(WT_CONSUMERS * M * 64);
 
     int s = 0, slot = 0;
     uint32_t ph = 0;
     uint32_t wst = ring_u + w_off;                           // stage s, this lane
     // Independent accumulator chains: consecutive MMAs of a warp go to different
     // accumulators, so they do not wait on each other's results.
-    constexpr int CH = MT == 1 ? 8 : 4;
+    constexpr int CH = WT_SPW == 2 && MT == 1 ? 8 : 4;
     for (int rg = rg0; rg < rg1; ++rg) {
         float acc[CH][MT][4];
 #pragma unroll
@@ -309,34 +319,35 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
         uint32_t xst = 0;                   // stage offset into x (TMEM columns or bytes)
         for (int st = 0; st < nst; ++st) {
             // xr[jj][mt]: words 0-3 plane 0 (k 16t..16t+7), words 4-7 plane 1 (+8)
-            uint32_t xr[2][MT][8];
+            uint32_t xr[WT_SPW][MT][8];
             if (XT) {
                 // the activations do not depend on the stage: read them before waiting
 #pragma unroll
-                for (int jj = 0; jj < 2; ++jj)
+                for (int jj = 0; jj < WT_SPW; ++jj)
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt)
                         tmem_ld_x8(tm_warp + xst + (uint32_t)((jj * MT + mt) * 8), xr[jj][mt]);
             }
             mbar_wait(&full[s], ph, status, abort_flag);   // on expiry: finish with garbage
-            uint4 w[2][2];
-            w[0][0] = lds128(wst);
-            w[0][1] = lds128(wst + 8 * WT_BOX);
-            w[1][0] = lds128(wst + kSlab2);
-            w[1][1] = lds128(wst + kSlab2 + 8 * WT_BOX);
+            uint4 w[WT_SPW][2];
+#pragma unroll
+            for (int jj = 0; jj < WT_SPW; ++jj) {
+                w[jj][0] = lds128(wst + jj * kSlab2);
+                w[jj][1] = lds128(wst + jj * kSlab2 + 8 * WT_BOX);
+            }
             if (XT) {
 #pragma unroll
-                for (int jj = 0; jj < 2; ++jj)
+                for (int jj = 0; jj < WT_SPW; ++jj)
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) tmem_wait_ld_x8(xr[jj][mt]);
             } else {
 #pragma unroll
-                for (int jj = 0; jj < 2; ++jj)
+                for (int jj = 0; jj < WT_SPW; ++jj)
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
                         uint4 a = make_uint4(0, 0, 0, 0), b = a;
                         if (x_live[mt]) {
-                            const uint32_t xa_addr = x_lane[mt] + xst + (jj ? x_slab2 : 0u);
+                            const uint32_t xa_addr = x_lane[mt] + xst + (uint32_t)jj * x_slab2;
                             a = lds128(xa_addr);
                             b = lds128(xa_addr + plane);
                         }
@@ -349,7 +360,7 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);           // operands are in registers
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
+            for (int jj = 0; jj < WT_SPW; ++jj) {
                 const uint32_t wav[4] = {w[jj][0].x, w[jj][0].y, w[jj][0].z, w[jj][0].w};
                 const uint32_t wbv[4] = {w[jj][1].x, w[jj][1].y, w[jj][1].z, w[jj][1].w};
 #pragma unroll
@@ -487,7 +498,7 @@ static bool wt_use_tmem(int M, int K, int64_t N, int num_sms) {
     if (wt_layout(M, K, 1, 8, false).total > (size_t)WT_MAX_SMEM) return true;
     const int64_t RG = (N + 15) / 16;
     const int64_t grid = RG < num_sms ? RG : num_sms;
-    return (RG + grid - 1) / grid * nst >= 32;
+    return (RG + grid - 1) / grid * nst * WT_STAGE_BYTES >= ((int64_t)512 << 10);
 }
 
 // Whether the TMA path takes this problem: K % 64 == 0, M <= 16 and the activations fit
