@@ -69,7 +69,11 @@ typedef struct {
 } q8_qparams;
 
 /* Which call a workspace is sized for (q8_workspace_bytes). */
-typedef enum { Q8_OP_LINEAR_W8A8 = 0, Q8_OP_LINEAR_DQ8CA_Q4GSW = 1 } q8_op;
+typedef enum {
+    Q8_OP_LINEAR_W8A8 = 0,
+    Q8_OP_LINEAR_DQ8CA_Q4GSW = 1,
+    Q8_OP_LINEAR_W8A16 = 2          /* q8_linear_w8a16_ws */
+} q8_op;
 
 /* Host.  Human-readable name of a status code (static string). */
 const char* q8_status_string(q8_status s);
@@ -157,6 +161,27 @@ q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w,
                           void* y, q8_dtype yt, int64_t M, int64_t N, int64_t K,
                           void* stream);
 
+/* W8A16, same definition and arguments as q8_linear_w8a16, computed on the int8 tensor
+ * cores for decode-sized M (1..16): the bf16 activations are rewritten once per call as
+ * exact int8 digit planes (per row: base-128 digits of the values on a common power of
+ * two), every plane is multiplied with the int8 weight by tcgen05.mma.kind::i8 (exact
+ * int32), and the planes are recombined in fp64 before the scale -- the dot product is
+ * rounded about once, so the result meets the same bound as q8_linear_w8a16 with room
+ * to spare.  A row whose values span more than the plane budget (jcap planes of 7 bits:
+ * 80 for M = 1, 20 for M = 4, 10 for M = 16) keeps its smallest elements, and any
+ * non-finite ones, out of the planes and adds their products in the epilogue (slower,
+ * same accuracy; infinities and NaNs propagate as in IEEE arithmetic).
+ *   workspace: device memory of at least q8_workspace_bytes(Q8_OP_LINEAR_W8A16, M, N, K, 0)
+ *   bytes, 16-byte aligned, ZERO-FILLED before its first use and then left to this
+ *   function (it keeps per-call flags there); one workspace must not be used by two calls
+ *   that may run at the same time.  The kernel keeps one CTA per SM resident and its
+ *   CTAs wait on each other (bounded): it must not share the GPU with a limit on SMs.
+ *   Q8_ERR_WORKSPACE if the workspace is NULL or too small.  M > 16 (workspace size 0)
+ *   runs q8_linear_w8a16. */
+q8_status q8_linear_w8a16_ws(const void* x, const int8_t* q, const float* s_w,
+                             void* y, q8_dtype yt, int64_t M, int64_t N, int64_t K,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* W8A8: static per-tensor int8 activations times per-channel int8 weights
  * ([SmolVLM-Q8] Q8Linear.forward; the delegated op takes weight_sums):
  *     acc1[m,n] = sum_k xq1[m,k] q[n,k]     (int32, exact)
@@ -192,7 +217,8 @@ q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* g
                                 void* workspace, size_t ws_bytes, void* stream);
 
 /* Host.  Workspace bytes a linear needs for these sizes (0 if none).  `extra` is
- * "two-pass" (0/1) for Q8_OP_LINEAR_W8A8 and G for Q8_OP_LINEAR_DQ8CA_Q4GSW.
+ * "two-pass" (0/1) for Q8_OP_LINEAR_W8A8, G for Q8_OP_LINEAR_DQ8CA_Q4GSW and unused (0)
+ * for Q8_OP_LINEAR_W8A16 (whose size also depends on the current device's SM count).
  * Returns 0 for invalid arguments as well; the linear then reports the error. */
 size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra);
 

@@ -285,9 +285,34 @@ q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w, void
                                       (cudaStream_t)stream, sms));
 }
 
+q8_status q8_linear_w8a16_ws(const void* x, const int8_t* q, const float* s_w, void* y,
+                             q8_dtype yt, int64_t M, int64_t N, int64_t K, void* workspace,
+                             size_t ws_bytes, void* stream) {
+    if (yt != Q8_F32 && yt != Q8_BF16) return Q8_ERR_ARG;
+    if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (M == 0) return Q8_OK;
+    if (!x || !q || !s_w || !y) return Q8_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    int* status = nullptr;
+    Q8_TRY(current_device(sms, &status));
+    const size_t need = w8a16_tc_workspace_bytes(M, K, sms);
+    if (need == 0) return q8_linear_w8a16(x, q, s_w, y, yt, M, N, K, stream);
+    if (!workspace || ws_bytes < need) return Q8_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return Q8_ERR_ALIGN;
+    return launched(launch_w8a16_tc((const uint16_t*)x, q, s_w, y, yt == Q8_BF16, M, N, (int)K,
+                                    workspace, (cudaStream_t)stream, sms, status));
+}
+
 size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) {
     if (M < 0 || N < 1 || check_k(K) != Q8_OK) return 0;
     switch (op) {
+        case Q8_OP_LINEAR_W8A16: {
+            int sms = 0;
+            if (current_device(sms) != Q8_OK) return 0;
+            return w8a16_tc_workspace_bytes(M, K, sms);
+        }
         case Q8_OP_LINEAR_W8A8: return plan_w8a8(M, K, extra != 0).bytes;
         case Q8_OP_LINEAR_DQ8CA_Q4GSW:
             if (!valid_group(extra) || K % 128 != 0 || K % extra != 0) return 0;

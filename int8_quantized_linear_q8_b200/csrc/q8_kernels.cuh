@@ -59,6 +59,12 @@ cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_
                              int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,
                              int num_sms, int* status);
 
+// k_w8a16_tc.cu
+size_t w8a16_tc_workspace_bytes(int64_t M, int64_t K, int num_sms);
+cudaError_t launch_w8a16_tc(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
+                            int y_bf16, int64_t M, int64_t N, int K, void* ws,
+                            cudaStream_t st, int num_sms, int* status);
+
 // k_gemm_tc.cu
 cudaError_t launch_gemm_s8s8_s32_tc(const int8_t* a, const int8_t* b, int32_t* acc, int64_t M,
                                     int64_t N, int K, cudaStream_t st, int num_sms, int* status);
