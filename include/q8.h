@@ -72,7 +72,7 @@ typedef struct {
 typedef enum {
     Q8_OP_LINEAR_W8A8 = 0,
     Q8_OP_LINEAR_DQ8CA_Q4GSW = 1,
-    Q8_OP_LINEAR_W8A16 = 2          /* q8_linear_w8a16_ws */
+    Q8_OP_LINEAR_W8A16_PLANES = 2   /* q8_linear_w8a16_planes */
 } q8_op;
 
 /* Host.  Human-readable name of a status code (static string). */
@@ -170,17 +170,20 @@ q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w,
  * to spare.  A row whose values span more than the plane budget (jcap planes of 7 bits:
  * 80 for M = 1, 20 for M = 4, 10 for M = 16) keeps its smallest elements, and any
  * non-finite ones, out of the planes and adds their products in the epilogue (slower,
- * same accuracy; infinities and NaNs propagate as in IEEE arithmetic).
- *   workspace: device memory of at least q8_workspace_bytes(Q8_OP_LINEAR_W8A16, M, N, K, 0)
- *   bytes, 16-byte aligned, ZERO-FILLED before its first use and then left to this
- *   function (it keeps per-call flags there); one workspace must not be used by two calls
- *   that may run at the same time.  The kernel keeps one CTA per SM resident and its
- *   CTAs wait on each other (bounded): it must not share the GPU with a limit on SMs.
+ * same accuracy; infinities and NaNs propagate as in IEEE arithmetic).  Its weight stream
+ * is conversion-free, but building the planes costs a grid-wide handshake per call, so
+ * q8_linear_w8a16 is faster at the sizes measured; this form is for callers that want
+ * the tighter rounding.
+ *   workspace: at least q8_workspace_bytes(Q8_OP_LINEAR_W8A16_PLANES, M, N, K, 0) bytes,
+ *   16-byte aligned, ZERO-FILLED before its first use and then left to this function (it
+ *   keeps per-call flags there); one workspace must not serve two calls that may run at
+ *   the same time.  The kernel keeps one CTA per SM resident and its CTAs wait on each
+ *   other (bounded): it must not share the GPU with a limit on SMs.
  *   Q8_ERR_WORKSPACE if the workspace is NULL or too small.  M > 16 (workspace size 0)
  *   runs q8_linear_w8a16. */
-q8_status q8_linear_w8a16_ws(const void* x, const int8_t* q, const float* s_w,
-                             void* y, q8_dtype yt, int64_t M, int64_t N, int64_t K,
-                             void* workspace, size_t ws_bytes, void* stream);
+q8_status q8_linear_w8a16_planes(const void* x, const int8_t* q, const float* s_w,
+                                 void* y, q8_dtype yt, int64_t M, int64_t N, int64_t K,
+                                 void* workspace, size_t ws_bytes, void* stream);
 
 /* W8A8: static per-tensor int8 activations times per-channel int8 weights
  * ([SmolVLM-Q8] Q8Linear.forward; the delegated op takes weight_sums):
@@ -218,7 +221,8 @@ q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* g
 
 /* Host.  Workspace bytes a linear needs for these sizes (0 if none).  `extra` is
  * "two-pass" (0/1) for Q8_OP_LINEAR_W8A8, G for Q8_OP_LINEAR_DQ8CA_Q4GSW and unused (0)
- * for Q8_OP_LINEAR_W8A16 (whose size also depends on the current device's SM count).
+ * for Q8_OP_LINEAR_W8A16_PLANES (whose size also depends on the current device's SM
+ * count).
  * Returns 0 for invalid arguments as well; the linear then reports the error. */
 size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra);
 

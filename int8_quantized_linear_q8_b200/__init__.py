@@ -24,7 +24,7 @@ Q8_OK = 0
 Q8_ERR_NULL, Q8_ERR_SHAPE, Q8_ERR_ALIGN, Q8_ERR_ARG = 1, 2, 3, 4
 Q8_ERR_UNSUPPORTED_ARCH, Q8_ERR_LAUNCH, Q8_ERR_WORKSPACE, Q8_ERR_DEVICE = 5, 6, 7, 8
 Q8_F32, Q8_BF16 = 0, 1
-Q8_OP_LINEAR_W8A8, Q8_OP_LINEAR_DQ8CA_Q4GSW, Q8_OP_LINEAR_W8A16 = 0, 1, 2
+Q8_OP_LINEAR_W8A8, Q8_OP_LINEAR_DQ8CA_Q4GSW, Q8_OP_LINEAR_W8A16_PLANES = 0, 1, 2
 
 # Every entry point of include/q8.h, for export checks.
 SYMBOLS = (
@@ -32,7 +32,7 @@ SYMBOLS = (
     "q8_quantize_static", "q8_observe_minmax", "q8_qparams_from_minmax",
     "q8_quantize_weight_q4gs", "q8_linear_w8a16", "q8_linear_w8a8", "q8_linear_dq8ca_q4gsw",
     "q8_workspace_bytes", "q8_gemm_s8s8_s32", "q8_last_device_status",
-    "q8_linear_w8a8_noalloc", "q8_selftest_bounded_wait", "q8_linear_w8a16_ws",
+    "q8_linear_w8a8_noalloc", "q8_selftest_bounded_wait", "q8_linear_w8a16_planes",
 )
 # Built-in scratch of q8_linear_w8a8_noalloc (bytes).
 Q8_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -81,8 +81,9 @@ def _lib() -> ctypes.CDLL:
     L.q8_quantize_weight_q4gs.argtypes = [_vp, _i64, _i64, st, _vp, _vp, _vp]
     L.q8_linear_w8a16.restype = st
     L.q8_linear_w8a16.argtypes = [_vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp]
-    L.q8_linear_w8a16_ws.restype = st
-    L.q8_linear_w8a16_ws.argtypes = [_vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp, _sz, _vp]
+    L.q8_linear_w8a16_planes.restype = st
+    L.q8_linear_w8a16_planes.argtypes = [_vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp, _sz,
+                                         _vp]
     L.q8_linear_w8a8.restype = st
     L.q8_linear_w8a8.argtypes = [_vp, q8_qparams, ctypes.POINTER(q8_qparams), _vp, _vp, _vp,
                                  _vp, _i64, _i64, _i64, _vp, _sz, _vp]
@@ -259,20 +260,20 @@ def q8_linear_w8a16(x: torch.Tensor, q: torch.Tensor, s_w: torch.Tensor, y=None,
     return y
 
 
-def q8_w8a16_workspace(M: int, N: int, K: int, device=None) -> Optional[torch.Tensor]:
-    """A zero-filled workspace for q8_linear_w8a16_ws (None when the sizes need none).
+def q8_w8a16_planes_workspace(M: int, N: int, K: int, device=None) -> Optional[torch.Tensor]:
+    """A zero-filled workspace for q8_linear_w8a16_planes (None when the sizes need none).
     Keep one per stream: the call leaves per-call flags in it."""
-    nbytes = q8_workspace_bytes(Q8_OP_LINEAR_W8A16, M, N, K)
+    nbytes = q8_workspace_bytes(Q8_OP_LINEAR_W8A16_PLANES, M, N, K)
     if nbytes == 0:
         return None
     return torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
 
-def q8_linear_w8a16_ws(x: torch.Tensor, q: torch.Tensor, s_w: torch.Tensor, workspace,
-                       y=None, out_dtype: torch.dtype = torch.bfloat16,
-                       stream=None) -> torch.Tensor:
-    """q8_linear_w8a16 on the int8 tensor cores (exact digit planes of x); `workspace` from
-    q8_w8a16_workspace (zero-filled once, not shared by concurrent calls)."""
+def q8_linear_w8a16_planes(x: torch.Tensor, q: torch.Tensor, s_w: torch.Tensor, workspace,
+                           y=None, out_dtype: torch.dtype = torch.bfloat16,
+                           stream=None) -> torch.Tensor:
+    """q8_linear_w8a16 on the int8 tensor cores over exact digit planes of x; `workspace`
+    from q8_w8a16_planes_workspace (zero-filled once, not shared by concurrent calls)."""
     M, K = x.shape
     N = q.shape[0]
     _need(x, "x", torch.bfloat16, (M, K))
@@ -283,9 +284,9 @@ def q8_linear_w8a16_ws(x: torch.Tensor, q: torch.Tensor, s_w: torch.Tensor, work
     y = _out(y, "y", out_dtype, (M, N), x.device)
     yt = Q8_BF16 if y.dtype == torch.bfloat16 else Q8_F32
     wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_lib().q8_linear_w8a16_ws(_ptr(x), _ptr(q), _ptr(s_w), _ptr(y), yt, M, N, K,
-                                     _ptr(workspace), wsb, _stream(stream)),
-           "q8_linear_w8a16_ws")
+    _check(_lib().q8_linear_w8a16_planes(_ptr(x), _ptr(q), _ptr(s_w), _ptr(y), yt, M, N, K,
+                                         _ptr(workspace), wsb, _stream(stream)),
+           "q8_linear_w8a16_planes")
     return y
 
 

@@ -190,7 +190,7 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
                 }
             }
             for (int i = max(0, it - TC_STAGES); i < it; ++i)
-                mbar_drain(&full[i % TC_STAGES], (uint32_t)(i / TC_STAGES) & 1u);
+                mbar_drain(&full[i % TC_STAGES], (uint32_t)(i / TC_STAGES) & 1u, status);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -229,7 +229,7 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
             }
             // all MMAs issued here are complete before tensor memory is released
             tc_commit(mma_done);
-            mbar_drain(mma_done, 0);
+            mbar_drain(mma_done, 0, status);
         }
         __syncwarp();
     } else {

@@ -168,6 +168,9 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
         // ------------------------------------------------------------- producer
         if (lane == 0) {
             tma_prefetch_desc(&wmap);
+            // the weight is read once: let it leave L2 first, so that the activations and
+            // scales (of this call and the next ones) stay there
+            const uint64_t pol = make_l2_policy_evict_first();
             int it = 0, s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -182,15 +185,15 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
                     uint8_t* dst = ring + (size_t)s * WT_STAGE_BYTES;
 #pragma unroll
                     for (int j = 0; j < WT_BOXES; ++j)     // boxes past K read as zeros
-                        tma_load_2d(dst + j * 16 * WT_BOX, &wmap, k0 + j * WT_BOX, rg * 16,
-                                    &full[s]);
+                        tma_load_2d_hint(dst + j * 16 * WT_BOX, &wmap, k0 + j * WT_BOX, rg * 16,
+                                         &full[s], pol);
                     ++it;
                     if (++s == stages) { s = 0; ph ^= 1u; }
                 }
             }
             // Do not leave while copies issued here may still be landing in shared memory.
             for (int i = max(0, it - stages); i < it; ++i)
-                mbar_drain(&full[i % stages], (uint32_t)(i / stages) & 1u);
+                mbar_drain(&full[i % stages], (uint32_t)(i / stages) & 1u, status);
         }
         return;
     }

@@ -227,7 +227,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                 }
             }
             for (int i = max(0, it - QT_STAGES); i < it; ++i)
-                mbar_drain(&full[i % QT_STAGES], (uint32_t)(i / QT_STAGES) & 1u);
+                mbar_drain(&full[i % QT_STAGES], (uint32_t)(i / QT_STAGES) & 1u, status);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
@@ -270,7 +270,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                 }
             }
             qt_commit(mma_done);
-            mbar_drain(mma_done, 0);
+            mbar_drain(mma_done, 0, status);
         }
         __syncwarp();
     } else {

@@ -533,7 +533,7 @@ __global__ __launch_bounds__(WC_THREADS, 1) void k_w8a16_tc(
             }
             // do not leave while copies issued here may still be landing
             for (long long i = issued > S ? issued - S : 0; i < issued; ++i)
-                mbar_drain(&full[i % S], (uint32_t)(i / S) & 1u);
+                mbar_drain(&full[i % S], (uint32_t)(i / S) & 1u, a.status);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -570,7 +570,7 @@ __global__ __launch_bounds__(WC_THREADS, 1) void k_w8a16_tc(
             }
             // every MMA issued here completes before tensor memory is released
             wc_commit(mma_done);
-            mbar_drain(mma_done, 0);
+            mbar_drain(mma_done, 0, a.status);
         }
         __syncwarp();
     } else {

@@ -285,9 +285,9 @@ q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w, void
                                       (cudaStream_t)stream, sms));
 }
 
-q8_status q8_linear_w8a16_ws(const void* x, const int8_t* q, const float* s_w, void* y,
-                             q8_dtype yt, int64_t M, int64_t N, int64_t K, void* workspace,
-                             size_t ws_bytes, void* stream) {
+q8_status q8_linear_w8a16_planes(const void* x, const int8_t* q, const float* s_w, void* y,
+                                 q8_dtype yt, int64_t M, int64_t N, int64_t K, void* workspace,
+                                 size_t ws_bytes, void* stream) {
     if (yt != Q8_F32 && yt != Q8_BF16) return Q8_ERR_ARG;
     if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
     Q8_TRY(check_k(K));
@@ -308,7 +308,7 @@ q8_status q8_linear_w8a16_ws(const void* x, const int8_t* q, const float* s_w, v
 size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) {
     if (M < 0 || N < 1 || check_k(K) != Q8_OK) return 0;
     switch (op) {
-        case Q8_OP_LINEAR_W8A16: {
+        case Q8_OP_LINEAR_W8A16_PLANES: {
             int sms = 0;
             if (current_device(sms) != Q8_OK) return 0;
             return w8a16_tc_workspace_bytes(M, K, sms);

@@ -241,11 +241,16 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, 
         }
     }
 }
-// Bounded wait used only on exit paths: waits for a phase without touching flags.
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+// Bounded wait used only on exit paths: waits for a phase without touching the abort flag.
+// A drain that runs out of time means a logic error; it is recorded in *status if given.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity,
+                                           int* status = nullptr) {
     const unsigned long long t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (status) atomicExch(status, kStatusWaitTimeout);
+            return;
+        }
     }
 }
 // 2-D tiled TMA load of one box into shared memory; completion is signalled on `bar`

@@ -205,6 +205,69 @@ def test_w8a16_ragged(M, N, K, out):
         check_bf16(_bits(y), y64, absum, "ragged")
 
 
+def _w8a16_direct(x_bf16, W, out_dtype=torch.float32):
+    q, s, _ = q8.q8_quantize_weight(W.to(DEV), want_wsum=False)
+    y = q8.q8_linear_w8a16(x_bf16.to(DEV), q, s, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    rq, rs, _ = oracle.quantize_weight(W.numpy())
+    y64, absum = oracle.linear_w8a16(wl.bf16_bits(x_bf16), rq, rs)
+    return y.cpu().numpy(), y64, absum
+
+
+def _range_edge_rows(M, K, e_small, seed):
+    """Row 0..M-1: x[:, 0] = 2^10 with an all-zero weight column (so it only sets the row's
+    exponent range), every other element +-(1 + j/128) * 2^e_small.  The output is then the
+    sum of the small elements alone, and the tolerance is relative to it."""
+    g = torch.Generator().manual_seed(seed)
+    sign = torch.where(torch.rand(M, K, generator=g) < 0.5, -1.0, 1.0)
+    frac = 1.0 + torch.randint(0, 128, (M, K), generator=g).to(torch.float32) / 128.0
+    x = sign * frac * 2.0 ** e_small
+    x[:, 0] = 1024.0
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("M,N", [(16, 2000), (4, 32000)])
+@pytest.mark.parametrize("e_small", [-22, -23])
+def test_w8a16_fp16_range_boundary(M, N, e_small):
+    """2^10 and 2^-22 are 32 binades apart -- the widest range the fp16 path takes (its
+    smallest elements land exactly on the fp16 subnormal grid); at 2^-23 the kernel must
+    fall back to bf16.  Either way the small elements' sum must be exact to fp32 rounding."""
+    K = 4096
+    x = _range_edge_rows(M, K, e_small, seed=90 + M)
+    W = wl.weight(N, K, seed=91)
+    W[:, 0] = 0.0
+    y, y64, absum = _w8a16_direct(x, W)
+    check_f32(y, y64, absum, f"range boundary 2^{e_small}")
+
+
+@pytest.mark.parametrize("M,N", [(16, 1000), (4, 32000)])
+@pytest.mark.parametrize("kind", ["wide", "tiny", "inf"])
+def test_w8a16_activation_ranges(M, N, kind):
+    """Rows the fp16 path cannot take (exponents spread over 2^-120..2^60, inf/NaN) and rows
+    it takes with a large scale (all values near the bf16 subnormal range)."""
+    K = 4096
+    g = torch.Generator().manual_seed(95)
+    x = torch.randn(M, K, generator=g, dtype=torch.float64)
+    if kind == "wide":
+        x = x * torch.pow(2.0, torch.randint(-120, 61, (M, K), generator=g).to(torch.float64))
+    elif kind == "tiny":
+        x = x * 2.0 ** -128
+    x = x.to(torch.float32).to(torch.bfloat16)
+    if kind == "inf":
+        x[0, 3] = float("inf")
+        x[1, 7] = float("nan")
+    W = wl.weight(N, K, seed=96)
+    y, y64, absum = _w8a16_direct(x, W)
+    if kind == "inf":
+        y = y.astype(np.float64)
+        assert np.array_equal(np.isnan(y), np.isnan(y64))
+        assert np.array_equal(np.isinf(y), np.isinf(y64))
+        fin = np.isfinite(y64)
+        check_f32(y[fin], y64[fin], absum[fin], "finite rows")
+    else:
+        check_f32(y, y64, absum, kind)
+
+
 def test_w8a16_empty_m():
     q = torch.zeros(16, 64, dtype=torch.int8, device=DEV)
     s = torch.ones(16, device=DEV)

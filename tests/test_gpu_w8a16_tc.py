@@ -1,4 +1,4 @@
-"""GPU parity of q8_linear_w8a16_ws -- W8A16 on the int8 tensor cores over exact digit planes
+"""GPU parity of q8_linear_w8a16_planes -- W8A16 on the int8 tensor cores over exact digit planes
 of the activations -- against the oracle.  Besides the contract tolerances of tests/tolerance.py,
 fp32 outputs are held to about one rounding of the exact dot product, which is what the
 digit-plane recombination gives."""
@@ -30,7 +30,7 @@ _WS = {}
 
 def _ws(M, N, K):
     """One zero-filled workspace for the module, grown as needed (flags persist across calls)."""
-    n = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A16, M, N, K)
+    n = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A16_PLANES, M, N, K)
     if n == 0:
         return None
     if "ws" not in _WS or _WS["ws"].numel() < n:
@@ -58,7 +58,7 @@ def _case(x_bf16, W, out_dtype):
     M, K = x_bf16.shape
     N = W.shape[0]
     q, s, _ = q8.q8_quantize_weight(W.to(DEV), want_wsum=False)
-    y = q8.q8_linear_w8a16_ws(x_bf16.to(DEV), q, s, _ws(M, N, K), out_dtype=out_dtype)
+    y = q8.q8_linear_w8a16_planes(x_bf16.to(DEV), q, s, _ws(M, N, K), out_dtype=out_dtype)
     torch.cuda.synchronize()
     rq, rs, _ = oracle.quantize_weight(W.numpy())
     y64, absum = oracle.linear_w8a16(wl.bf16_bits(x_bf16), rq, rs)
@@ -163,19 +163,19 @@ def test_w8a16_tc_workspace_checks():
     W = wl.weight(N, K, seed=60)
     q, s, _ = q8.q8_quantize_weight(W.to(DEV), want_wsum=False)
     x = wl.normal_bf16((M, K), 1.0, seed=61).to(DEV)
-    need = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A16, M, N, K)
+    need = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A16_PLANES, M, N, K)
     assert need > 0
     small = torch.zeros(need - 1024, dtype=torch.uint8, device=DEV)
     with pytest.raises(q8.Q8Error) as ei:
-        q8.q8_linear_w8a16_ws(x, q, s, small)
+        q8.q8_linear_w8a16_planes(x, q, s, small)
     assert ei.value.status == q8.Q8_ERR_WORKSPACE
     with pytest.raises(q8.Q8Error) as ei:
-        q8.q8_linear_w8a16_ws(x, q, s, None)
+        q8.q8_linear_w8a16_planes(x, q, s, None)
     assert ei.value.status == q8.Q8_ERR_WORKSPACE
     # more than 16 rows needs no workspace and runs the workspace-free path
-    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A16, 17, N, K) == 0
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A16_PLANES, 17, N, K) == 0
     x17 = wl.normal_bf16((17, K), 1.0, seed=62)
-    y = q8.q8_linear_w8a16_ws(x17.to(DEV), q, s, None, out_dtype=torch.float32)
+    y = q8.q8_linear_w8a16_planes(x17.to(DEV), q, s, None, out_dtype=torch.float32)
     rq, rs, _ = oracle.quantize_weight(W.numpy())
     y64, absum = oracle.linear_w8a16(wl.bf16_bits(x17), rq, rs)
     check_f32(y.cpu().numpy(), y64, absum, "M=17 fallback")
