@@ -34,20 +34,22 @@
 
 namespace q8 {
 
-#ifndef WT_SLABS_DEF
-#define WT_SLABS_DEF 16
-#endif
-constexpr int WT_SLABS = WT_SLABS_DEF;                  // 64-byte slabs per stage
 #ifndef WT_CONSUMERS_DEF
 #define WT_CONSUMERS_DEF 8
 #endif
 constexpr int WT_CONSUMERS = WT_CONSUMERS_DEF;          // consumer warps
-constexpr int WT_SPW = WT_SLABS / WT_CONSUMERS;         // slabs per consumer warp and stage
-static_assert(WT_SPW * WT_CONSUMERS == WT_SLABS && WT_CONSUMERS % 4 == 0, "slab split");
 constexpr int WT_THREADS = (WT_CONSUMERS + 1) * 32;     // + producer warp
 constexpr int WT_BOX = 256;                             // TMA box width (bytes of K)
-constexpr int WT_BOXES = WT_SLABS * 64 / WT_BOX;        // boxes per stage
-constexpr int WT_STAGE_BYTES = 16 * 64 * WT_SLABS;      // 16 rows of WT_SLABS * 64 bytes
+// Stage geometry: a stage is 16 rows x SL slabs of 64 bytes of K (SL = 16 or 32).
+#define WT_GEOMETRY(SL_)                                                                   \
+    constexpr int WT_SLABS = (SL_);                    /* 64-byte slabs per stage */      \
+    constexpr int WT_SPW = WT_SLABS / WT_CONSUMERS;    /* slabs per consumer warp */      \
+    constexpr int WT_BOXES = WT_SLABS * 64 / WT_BOX;   /* TMA boxes per stage */          \
+    constexpr int WT_STAGE_BYTES = 16 * 64 * WT_SLABS;                                    \
+    static_assert(WT_SPW * WT_CONSUMERS == WT_SLABS && WT_CONSUMERS % 4 == 0, "slab split"); \
+    (void)WT_SPW;                                                                          \
+    (void)WT_BOXES;                                                                        \
+    (void)WT_STAGE_BYTES
 constexpr int WT_MAX_SMEM = 227 * 1024;
 constexpr int WT_SLOTS = 16;                            // rotating partial-sum slots (> stages+1)
 
@@ -59,7 +61,9 @@ struct WtSmem {
 // Rows of q a CTA may own (its s_w slice is staged in shared memory).
 constexpr int WT_MAX_ROWS = 1024;
 
+template <int SL>
 static __host__ __device__ inline WtSmem wt_layout(int M, int K, int MT, int stages, bool xt) {
+    WT_GEOMETRY(SL);
     WtSmem L;
     L.stages = stages;
     L.ring = 0;
@@ -85,7 +89,8 @@ __device__ __forceinline__ uint32_t xfrag_addr(uint32_t xs, int M, int Kpad, int
 // Tensor-memory columns the staged activations need: every consumer warp holds 8
 // columns (32 bytes per lane) per chunk it owns (2 per stage) and per 8 activation rows;
 // warps w and w+4 share a lane quarter, so the allocation is twice one warp's share.
-__host__ __device__ inline int wt_tmem_cols(int nst, int MT) { return 2 * WT_SLABS * nst * MT; }
+template <int SL>
+__host__ __device__ inline int wt_tmem_cols(int nst, int MT) { return 2 * SL * nst * MT; }
 constexpr int WT_TMEM_MAX_COLS = 512;
 
 __device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&v)[8]) {
@@ -108,13 +113,14 @@ __device__ __forceinline__ void tmem_wait_ld_x8(uint32_t (&v)[8]) {
                    "+r"(v[6]), "+r"(v[7])::"memory");
 }
 
-template <int MT, bool XT>
+template <int MT, bool XT, int SL>
 __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     const __grid_constant__ CUtensorMap wmap, const uint16_t* __restrict__ x,
     const float* __restrict__ s_w, void* __restrict__ y, int y_bf16, int M, int N, int K,
     int stages, int* status) {
+    WT_GEOMETRY(SL);
     extern __shared__ __align__(1024) uint8_t smem[];
-    const WtSmem L = wt_layout(M, K, MT, stages, XT);
+    const WtSmem L = wt_layout<SL>(M, K, MT, stages, XT);
     uint8_t* ring = smem + L.ring;
     float* slots = reinterpret_cast<float*>(smem + L.red);        // [WT_SLOTS][MT][32][4]
     float* sws = reinterpret_cast<float*>(smem + L.sws);          // s_w of this CTA's rows
@@ -133,7 +139,7 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     // power-of-two TMEM allocation (>= 32 columns); the launcher checks it is <= 512
     int tcols = 32;
     if (XT)
-        while (tcols < wt_tmem_cols(nst, MT)) tcols <<= 1;
+        while (tcols < wt_tmem_cols<SL>(nst, MT)) tcols <<= 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -213,7 +219,7 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     // this warp's TMEM lanes (its quarter) and columns (share warp / 4 of its quarter)
     const uint32_t tm_warp =
         XT ? *tmem_slot + ((uint32_t)((warp & 3) * 32) << 16) +
-                 (uint32_t)((warp >> 2) * (wt_tmem_cols(nst, MT) / (WT_CONSUMERS / 4)))
+                 (uint32_t)((warp >> 2) * (wt_tmem_cols<SL>(nst, MT) / (WT_CONSUMERS / 4)))
            : 0u;
     if (XT) {
         // Lane (g, t) of warp w feeds, for its local chunk lc (chunk c = 16*(lc/2) + w +
@@ -487,43 +493,59 @@ bool make_tmap_u8_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t c
     return r == CUDA_SUCCESS;
 }
 
-// Whether the activations go to tensor memory (they need at most 512 columns).  With 9..16
-// rows they always do: in shared memory they would take the room of the ring and double
-// the shared-memory traffic.  With 1..8 rows they do when shared memory cannot hold them
-// next to 8 stages, or when each CTA streams at least 32 stages: setting up tensor memory
-// costs about half a microsecond more per launch (measured on the small shapes), which
-// the lighter shared-memory traffic pays back only on long streams.
+// Whether the activations go to tensor memory (they need at most 512 columns), for
+// stages of 16 slabs.  With 9..16 rows they always do: in shared memory they would take
+// the room of the ring and double the shared-memory traffic.  With 1..8 rows they do when
+// shared memory cannot hold them next to 8 stages, or when each CTA streams at least 512 KB:
+// setting up tensor memory costs about half a microsecond more per launch (measured on the
+// small shapes), which the lighter shared-memory traffic pays back only on long streams.
 static bool wt_use_tmem(int M, int K, int64_t N, int num_sms) {
+    WT_GEOMETRY(16);
     const int MT = M <= 8 ? 1 : 2;
     const int nst = (K / 64 + WT_SLABS - 1) / WT_SLABS;
-    if (wt_tmem_cols(nst, MT) > WT_TMEM_MAX_COLS) return false;
+    if (wt_tmem_cols<16>(nst, MT) > WT_TMEM_MAX_COLS) return false;
     if (MT == 2) return true;
-    if (wt_layout(M, K, 1, 8, false).total > (size_t)WT_MAX_SMEM) return true;
+    if (wt_layout<16>(M, K, 1, 8, false).total > (size_t)WT_MAX_SMEM) return true;
     const int64_t RG = (N + 15) / 16;
     const int64_t grid = RG < num_sms ? RG : num_sms;
     return (RG + grid - 1) / grid * nst * WT_STAGE_BYTES >= ((int64_t)512 << 10);
 }
 
+// Stages of 32 slabs (2 KB of K, 6 in the ring, activations in tensor memory) halve the
+// per-stage overhead of the consumers; they pay on long streams (each CTA at least 256 KB)
+// when K is a whole number of them, and cost latency on short ones (measured: 4096 x 32000
+// -8%, 4096 x 11008 -4%, 2048 x 8192 +3%).
+static bool wt_use_wide(int M, int K, int64_t N, int num_sms) {
+    const int MT = M <= 8 ? 1 : 2;
+    if (K % 2048 != 0 || wt_tmem_cols<32>(K / 2048, MT) > WT_TMEM_MAX_COLS) return false;
+    const int64_t RG = (N + 15) / 16;
+    const int64_t grid = RG < num_sms ? RG : num_sms;
+    return (RG + grid - 1) / grid * 16 * (int64_t)K >= ((int64_t)256 << 10);
+}
+
 // Whether the TMA path takes this problem: K % 64 == 0, M <= 16 and the activations fit
-// in tensor memory, or in shared memory next to at least 4 ring stages.
+// in tensor memory, or in shared memory next to at least 4 ring stages (16-slab stages;
+// 32-slab stages are only chosen where they fit too).
 bool w8a16_tma_fits(int64_t M, int64_t K) {
+    WT_GEOMETRY(16);
     if (M < 1 || M > 16 || (K % 64) != 0 || K > (int64_t)1 << 30) return false;
     const int MT = M <= 8 ? 1 : 2;
     const int nst = (int)((K / 64 + WT_SLABS - 1) / WT_SLABS);
-    if (wt_tmem_cols(nst, MT) <= WT_TMEM_MAX_COLS) return true;
+    if (wt_tmem_cols<16>(nst, MT) <= WT_TMEM_MAX_COLS) return true;
     // (with 9..16 rows, activations too long for tensor memory do not fit shared memory
     // next to 4 stages either)
-    return MT == 1 && wt_layout((int)M, (int)K, 1, 4, false).total <= (size_t)WT_MAX_SMEM;
+    return MT == 1 && wt_layout<16>((int)M, (int)K, 1, 4, false).total <= (size_t)WT_MAX_SMEM;
 }
 
-template <int MT, bool XT>
+template <int MT, bool XT, int SL>
 static cudaError_t launch_wt(const CUtensorMap& map, const uint16_t* x, const float* s_w, void* y,
                              int y_bf16, int M, int N, int K, cudaStream_t st, int num_sms,
                              int* status) {
     int stages = 8;    // must stay <= WT_SLOTS - 2
-    while (stages > 4 && wt_layout(M, K, MT, stages, XT).total > (size_t)WT_MAX_SMEM) --stages;
-    const WtSmem L = wt_layout(M, K, MT, stages, XT);
-    cudaError_t e = cudaFuncSetAttribute(k_w8a16_tma<MT, XT>,
+    while (stages > 4 && wt_layout<SL>(M, K, MT, stages, XT).total > (size_t)WT_MAX_SMEM)
+        --stages;
+    const WtSmem L = wt_layout<SL>(M, K, MT, stages, XT);
+    cudaError_t e = cudaFuncSetAttribute(k_w8a16_tma<MT, XT, SL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L.total);
     if (e != cudaSuccess) return e;
@@ -541,7 +563,7 @@ static cudaError_t launch_wt(const CUtensorMap& map, const uint16_t* x, const fl
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_w8a16_tma<MT, XT>, map, x, s_w, y, y_bf16, M, N, K,
+    return cudaLaunchKernelEx(&cfg, k_w8a16_tma<MT, XT, SL>, map, x, s_w, y, y_bf16, M, N, K,
                               stages, status);
 }
 
@@ -551,14 +573,16 @@ cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_
     CUtensorMap map;
     if (!make_tmap_u8_2d(&map, q, N, K, WT_BOX, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    const bool xt = wt_use_tmem((int)M, K, N, num_sms);
+    const int m = (int)M, n = (int)N;
+    if (wt_use_wide(m, K, N, num_sms))
+        return M <= 8 ? launch_wt<1, true, 32>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status)
+                      : launch_wt<2, true, 32>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status);
+    const bool xt = wt_use_tmem(m, K, N, num_sms);
     if (M <= 8)
-        return xt ? launch_wt<1, true>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms,
-                                       status)
-                  : launch_wt<1, false>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms,
-                                        status);
+        return xt ? launch_wt<1, true, 16>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status)
+                  : launch_wt<1, false, 16>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status);
     if (!xt) return cudaErrorInvalidValue;             // excluded by w8a16_tma_fits
-    return launch_wt<2, true>(map, x, s_w, y, y_bf16, (int)M, (int)N, K, st, num_sms, status);
+    return launch_wt<2, true, 16>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status);
 }
 
 }  // namespace q8

@@ -194,6 +194,8 @@ def test_w8a16_sweep_bf16(shape, M):
     (16, 1, 64), (1, 17, 64), (5, 2049, 1024), (12, 1000, 4160), (9, 33, 128), (2, 300, 11008),
     # ... activations at the tensor-memory limit (512 columns), and past it in shared memory
     (16, 100, 8192), (8, 50, 16384), (1, 70, 16448), (3, 33, 17472),
+    # ... 2 KB stages (K % 2048 == 0, long streams per CTA), ragged N
+    (3, 9000, 4096), (16, 20000, 6144), (1, 40000, 8192),
     # register-streamed fallback (K % 64 != 0, or M > 16)
     (3, 17, 16), (9, 40, 48), (17, 33, 80), (40, 130, 1040), (5, 2049, 2000)])
 @pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
