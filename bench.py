@@ -60,6 +60,7 @@ def parse_args():
     p.add_argument("--pM", type=int, default=16)
     p.add_argument("--pN", type=int, default=32000)
     p.add_argument("--pK", type=int, default=4096)
+    p.add_argument("--pG", type=int, default=32, help="8da4w group size (--profile q4)")
     p.add_argument("--reps", type=int, default=3)
     return p.parse_args()
 
@@ -752,12 +753,12 @@ def run_profile(args):
             q8.q8_linear_w8a8(x, (0.05, 3), q, ws, s, second=(0.05 / 255, 0), y=y)
     else:
         W = torch.randn(N, K, generator=g, device=dev) * 0.02
-        q4, gs = q8.q8_quantize_weight_q4gs(W, 32)
+        q4, gs = q8.q8_quantize_weight_q4gs(W, args.pG)
         del W
         x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
         y = torch.empty(M, N, device=dev)
         for _ in range(args.reps):
-            q8.q8_linear_dq8ca_q4gsw(x, q4, gs, 32, y=y)
+            q8.q8_linear_dq8ca_q4gsw(x, q4, gs, args.pG, y=y)
     torch.cuda.synchronize()
     print(json.dumps({"profile": args.profile, "M": M, "N": N, "K": K, "reps": args.reps}))
 

@@ -103,23 +103,56 @@ __global__ __launch_bounds__(CQ_THREADS) void k_choose_qparams(const uint16_t* _
                                                                int K, float* __restrict__ s_out,
                                                                int32_t* __restrict__ z_out,
                                                                int8_t* __restrict__ xq) {
-    __shared__ float red[CQ_THREADS / 32];
+    // A dependent kernel launched with programmatic serialisation (the 8da4w stream) may
+    // start now: it waits for this grid before it reads the codes, scales or zero points.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // One CTA per row.  Rows of up to CQ_REG * 8 * CQ_THREADS values stay in registers
+    // between the range pass and the code pass, and all their loads are in flight at once
+    // (the kernel is latency-bound: one row is a few KB); longer rows are read twice.
+    constexpr int CQ_REG = 4;
+    __shared__ float red[2][CQ_THREADS / 32];
     const int64_t m = blockIdx.x;
     const uint16_t* row = x + m * (int64_t)K;
     const int K8 = K >> 3;
-    float mn = 0.0f, mx = 0.0f;
-    for (int i = threadIdx.x; i < K8; i += CQ_THREADS) {
-        uint4 v = ldg_keep(row + 8 * i);
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const bool in_regs = K8 <= CQ_REG * CQ_THREADS;
+    uint4 v[CQ_REG];
+    float mn = 0.0f, mx = 0.0f;                  // the range always includes 0
+    auto range = [&](const uint4& u) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            float a = bf16lo(w[j]), b = bf16hi(w[j]);
+            const float a = bf16lo(w[j]), b = bf16hi(w[j]);
             mn = fminf(mn, fminf(a, b));
             mx = fmaxf(mx, fmaxf(a, b));
         }
+    };
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < CQ_REG; ++r) {
+            const int i = threadIdx.x + r * CQ_THREADS;
+            v[r] = i < K8 ? ldg_keep(row + 8 * i) : make_uint4(0, 0, 0, 0);   // zeros: no effect
+        }
+#pragma unroll
+        for (int r = 0; r < CQ_REG; ++r) range(v[r]);
+    } else {
+        for (int i = threadIdx.x; i < K8; i += CQ_THREADS) range(ldg_keep(row + 8 * i));
     }
-    mn = block_min<CQ_THREADS>(mn, red);
-    mx = block_max<CQ_THREADS>(mx, red);
+    // min and max over the CTA, one barrier
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        red[0][threadIdx.x >> 5] = mn;
+        red[1][threadIdx.x >> 5] = mx;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < CQ_THREADS / 32; ++w) {
+        mn = fminf(mn, red[0][w]);
+        mx = fmaxf(mx, red[1][w]);
+    }
     float s, zf;
     qparams_from_range(mn, mx, s, zf);
     if (threadIdx.x == 0) {
@@ -129,9 +162,8 @@ __global__ __launch_bounds__(CQ_THREADS) void k_choose_qparams(const uint16_t* _
     if (xq == nullptr) return;
     const float inv = __fdiv_rn(1.0f, s);
     uint2* qrow = reinterpret_cast<uint2*>(xq + m * (int64_t)K);
-    for (int i = threadIdx.x; i < K8; i += CQ_THREADS) {
-        uint4 v = ldg_keep(row + 8 * i);
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    auto codes = [&](const uint4& u, int i) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
         int c[8];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -139,6 +171,15 @@ __global__ __launch_bounds__(CQ_THREADS) void k_choose_qparams(const uint16_t* _
             c[2 * j + 1] = act_code(bf16hi(w[j]), inv, zf);
         }
         qrow[i] = make_uint2(pack4_s8(c[0], c[1], c[2], c[3]), pack4_s8(c[4], c[5], c[6], c[7]));
+    };
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < CQ_REG; ++r) {
+            const int i = threadIdx.x + r * CQ_THREADS;
+            if (i < K8) codes(v[r], i);
+        }
+    } else {
+        for (int i = threadIdx.x; i < K8; i += CQ_THREADS) codes(ldg_keep(row + 8 * i), i);
     }
 }
 

@@ -389,7 +389,10 @@ def test_dq8ca_q4gsw_config(M, G):
 
 
 @pytest.mark.parametrize("M,N,K,G", [(3, 17, 128, 32), (9, 40, 256, 64), (17, 33, 512, 128),
-                                     (5, 300, 1024, 256), (1, 1, 128, 128), (70, 129, 384, 32)])
+                                     (5, 300, 1024, 256), (1, 1, 128, 128), (70, 129, 384, 32),
+                                     # the TMA stream: partial last stage, ragged N, 9..16 rows
+                                     (2, 1000, 2176, 32), (16, 4097, 4096, 128),
+                                     (8, 2000, 6144, 64), (12, 700, 4224, 32), (4, 11008, 4096, 256)])
 def test_dq8ca_q4gsw_ragged(M, N, K, G):
     x, q4, gs, y = _q4_case(M, N, K, G, 900 + M, 901 + N)
     s, z, xq = oracle.choose_qparams(wl.bf16_bits(x))
