@@ -51,10 +51,11 @@ constexpr int WT_BOX = 256;                             // TMA box width (bytes 
     (void)WT_BOXES;                                                                        \
     (void)WT_STAGE_BYTES
 constexpr int WT_MAX_SMEM = 227 * 1024;
-constexpr int WT_SLOTS = 16;                            // rotating partial-sum slots (> stages+1)
+constexpr int WT_SLOTS = 16;                            // most partial-sum slots in flight
 
 struct WtSmem {
     int stages;
+    int nslots;                        // partial-sum slots (row groups in flight)
     size_t ring, xs, red, sws, bars, total;
 };
 
@@ -71,7 +72,13 @@ static __host__ __device__ inline WtSmem wt_layout(int M, int K, int MT, int sta
     const int Kpad = (K + WT_SLABS * 64 - 1) / (WT_SLABS * 64) * (WT_SLABS * 64);
     const size_t xbytes = xt ? 0 : (size_t)M * Kpad * 2;
     L.red = L.xs + ((xbytes + 127) / 128) * 128;
-    const size_t redbytes = (size_t)WT_SLOTS * MT * 32 * 4 * sizeof(float);
+    // A warp runs at most `stages` stages ahead of the slowest one, so at most
+    // ceil(stages / nst) + 2 row groups (nst stages each) have partial sums in flight;
+    // each warp keeps its own partial of a group.
+    const int nst = Kpad / (WT_SLABS * 64);
+    L.nslots = (stages + nst - 1) / nst + 2;
+    if (L.nslots > WT_SLOTS) L.nslots = WT_SLOTS;
+    const size_t redbytes = (size_t)L.nslots * WT_CONSUMERS * MT * 32 * 4 * sizeof(float);
     L.sws = L.red + redbytes;
     L.bars = L.sws + (size_t)WT_MAX_ROWS * sizeof(float);
     // barriers, slot counters, abort flag, TMEM address
@@ -122,7 +129,7 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     extern __shared__ __align__(1024) uint8_t smem[];
     const WtSmem L = wt_layout<SL>(M, K, MT, stages, XT);
     uint8_t* ring = smem + L.ring;
-    float* slots = reinterpret_cast<float*>(smem + L.red);        // [WT_SLOTS][MT][32][4]
+    float* slots = reinterpret_cast<float*>(smem + L.red);  // [nslots][WT_CONSUMERS][MT][32][4]
     float* sws = reinterpret_cast<float*>(smem + L.sws);          // s_w of this CTA's rows
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint64_t* empty = full + stages;
@@ -160,7 +167,6 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    for (int i = threadIdx.x; i < WT_SLOTS * MT * 128; i += WT_THREADS) slots[i] = 0.0f;
     if (XT) asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (XT) asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -388,38 +394,43 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
             if (++s == stages) { s = 0; ph ^= 1u; wst = ring_u + w_off; }
         }
 
-        // Add this warp's partial sums into the group's slot; the last warp to arrive
-        // scales, writes y and clears the slot.  Slots rotate, so no barrier is needed:
-        // a warp can run at most `stages` stages (<= WT_SLOTS - 2 groups) ahead of the
-        // slowest one.
-        float* sl = slots + (size_t)slot * MT * 128;
+        // Store this warp's partial sums in the group's slot; the last warp to arrive adds
+        // the WT_CONSUMERS partials in warp order (no float atomics, so the sum is the same
+        // on every run), scales and writes y.  Slots rotate, so no barrier is needed: a
+        // warp can run at most `stages` stages (nslots - 2 groups) ahead of the slowest one.
+        float* sl = slots + (size_t)slot * WT_CONSUMERS * MT * 128;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+        for (int mt = 0; mt < MT; ++mt) {
+            float v[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                float v = 0.0f;
+                v[i] = 0.0f;
 #pragma unroll
-                for (int c = 0; c < CH; ++c) v += acc[c][mt][i];
-                atomicAdd(&sl[(mt * 32 + lane) * 4 + i], v);
+                for (int c = 0; c < CH; ++c) v[i] += acc[c][mt][i];
             }
+            *reinterpret_cast<float4*>(&sl[((size_t)warp * MT + mt) * 128 + lane * 4]) =
+                make_float4(v[0], v[1], v[2], v[3]);
+        }
         __threadfence_block();
         __syncwarp();
         int prev = 0;
         if (lane == 0) prev = atomicAdd(&cnt[slot], 1);
         prev = __shfl_sync(0xffffffffu, prev, 0);
         if (prev == WT_CONSUMERS - 1) {
-            // Take the group's sums, clear the slot and release it before any global store.
             __threadfence_block();
             float vv[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                volatile float* vp = &sl[(mt * 32 + lane) * 4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) vv[mt][i] = vp[i];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) vp[i] = 0.0f;
+                for (int i = 0; i < 4; ++i) vv[mt][i] = 0.0f;
+                for (int w = 0; w < WT_CONSUMERS; ++w) {
+                    float4 u;
+                    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                                 : "=f"(u.x), "=f"(u.y), "=f"(u.z), "=f"(u.w)
+                                 : "r"(smem_u32(&sl[((size_t)w * MT + mt) * 128 + lane * 4])));
+                    vv[mt][0] += u.x; vv[mt][1] += u.y; vv[mt][2] += u.z; vv[mt][3] += u.w;
+                }
             }
-            __threadfence_block();
             __syncwarp();
             if (lane == 0) atomicExch(&cnt[slot], 0);
             const int n0 = rg * 16;
@@ -439,7 +450,7 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
                     }
                 }
         }
-        if (++slot == WT_SLOTS) slot = 0;
+        if (++slot == L.nslots) slot = 0;
     }
     if (XT) {
         // every tcgen05.ld of every consumer warp has completed (waited on in the loop)

@@ -90,15 +90,6 @@ __global__ __launch_bounds__(QW_THREADS) void k_quantize_weight(const float* __r
 // ------------------------------------------------- per-row activation qparams (a2)
 constexpr int CQ_THREADS = 256;
 
-__device__ __forceinline__ void qparams_from_range(float mn, float mx, float& s, float& zf) {
-    mn = fminf(mn, 0.0f);
-    mx = fmaxf(mx, 0.0f);
-    s = __fdiv_rn(__fsub_rn(mx, mn), 255.0f);
-    if (s < FLT_EPSILON) s = FLT_EPSILON;
-    zf = __fsub_rn(-128.0f, rintf(__fdiv_rn(mn, s)));
-    zf = fminf(fmaxf(zf, -128.0f), 127.0f);
-}
-
 __global__ __launch_bounds__(CQ_THREADS) void k_choose_qparams(const uint16_t* __restrict__ x,
                                                                int K, float* __restrict__ s_out,
                                                                int32_t* __restrict__ z_out,

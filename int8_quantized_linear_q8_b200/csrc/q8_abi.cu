@@ -381,9 +381,12 @@ q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* g
         return launched(launch_q4_gemm_tc(wb, xz, gs, s, y, G, M, N, (int)K, st, sms, status));
     }
     int8_t* xq = (int8_t*)(ws + plan.xq);
-    Q8_TRY(launched(launch_choose_qparams((const uint16_t*)x, M, (int)K, s, z, xq, st)));
-    if (q4_tma_fits(M, K, G))
-        return launched(launch_q4_tma(xq, s, z, q4, gs, G, y, M, N, (int)K, st, sms, status));
+    const bool tma = q4_tma_fits(M, K, G);
+    const bool qp = tma && q4_tma_quantizes(M);      // one kernel: qparams + weight stream
+    if (!qp) Q8_TRY(launched(launch_choose_qparams((const uint16_t*)x, M, (int)K, s, z, xq, st)));
+    if (tma)
+        return launched(launch_q4_tma((const uint16_t*)x, xq, s, z, qp, q4, gs, G, y, M, N,
+                                      (int)K, st, sms, status));
     return launched(launch_q4_gemv(xq, s, z, q4, gs, G, y, M, N, (int)K, st));
 }
 

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <float.h>
 #include <stdint.h>
 
 #include "../../include/q8.h"
@@ -25,6 +26,18 @@ __device__ __forceinline__ int act_code(float v, float inv, float zf) {
     float r = __fadd_rn(rintf(t), zf);
     r = fminf(fmaxf(r, -128.0f), 127.0f);
     return __float2int_rn(r);
+}
+
+// Asymmetric int8 parameters of a row whose values span [mn, mx] (choose_qparams_affine
+// of the executorch 8da4w operator): the range is widened to include 0, s = (mx - mn) / 255
+// (at least FLT_EPSILON) and z = -128 - round(mn / s), clamped to [-128, 127].
+__device__ __forceinline__ void qparams_from_range(float mn, float mx, float& s, float& zf) {
+    mn = fminf(mn, 0.0f);
+    mx = fmaxf(mx, 0.0f);
+    s = __fdiv_rn(__fsub_rn(mx, mn), 255.0f);
+    if (s < FLT_EPSILON) s = FLT_EPSILON;
+    zf = __fsub_rn(-128.0f, rintf(__fdiv_rn(mn, s)));
+    zf = fminf(fmaxf(zf, -128.0f), 127.0f);
 }
 
 // Weight code: clamp(round(w / s), -lim, lim) with a true IEEE division.

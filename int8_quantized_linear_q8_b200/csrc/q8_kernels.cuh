@@ -80,9 +80,12 @@ cudaError_t launch_q4_gemv(const int8_t* xq, const float* s, const int32_t* z, c
 
 // k_q4_tma.cu
 bool q4_tma_fits(int64_t M, int64_t K, int G);
-cudaError_t launch_q4_tma(const int8_t* xq, const float* s, const int32_t* z, const uint8_t* q4,
-                          const float* gs, int G, float* y, int64_t M, int64_t N, int K,
-                          cudaStream_t st, int num_sms, int* status);
+bool q4_tma_quantizes(int64_t M);
+// qp: x bf16 [M, K] is quantized in the kernel and xq / s / z receive the codes and
+// qparams; otherwise xq / s / z are the qparams kernel's output and x is unused.
+cudaError_t launch_q4_tma(const uint16_t* x, int8_t* xq, float* s, int32_t* z, bool qp,
+                          const uint8_t* q4, const float* gs, int G, float* y, int64_t M,
+                          int64_t N, int K, cudaStream_t st, int num_sms, int* status);
 
 // k_q4_tc.cu
 cudaError_t launch_q4_expand_bf16(const uint8_t* q4, int64_t N, int K, uint16_t* wb,

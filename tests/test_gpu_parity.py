@@ -392,7 +392,9 @@ def test_dq8ca_q4gsw_config(M, G):
                                      (5, 300, 1024, 256), (1, 1, 128, 128), (70, 129, 384, 32),
                                      # the TMA stream: partial last stage, ragged N, 9..16 rows
                                      (2, 1000, 2176, 32), (16, 4097, 4096, 128),
-                                     (8, 2000, 6144, 64), (12, 700, 4224, 32), (4, 11008, 4096, 256)])
+                                     (8, 2000, 6144, 64), (12, 700, 4224, 32), (4, 11008, 4096, 256),
+                                     # rows longer than the stream keeps in registers
+                                     (1, 300, 12288, 64), (3, 500, 10240, 128)])
 def test_dq8ca_q4gsw_ragged(M, N, K, G):
     x, q4, gs, y = _q4_case(M, N, K, G, 900 + M, 901 + N)
     s, z, xq = oracle.choose_qparams(wl.bf16_bits(x))
@@ -400,12 +402,41 @@ def test_dq8ca_q4gsw_ragged(M, N, K, G):
     check_f32(y, y64, absum, f"8da4w ragged M={M} N={N} K={K} G={G}")
 
 
-def test_dq8ca_tensor_core_group_partials_exact():
-    """One group (G = K = 256) with unit group scales: y / s must be the exact integer
-    sum_k (xq - z) q4 -- the bf16 tensor-core path keeps every group partial exact."""
-    M, N, K, G = 300, 200, 256, 256
+@pytest.mark.parametrize("M,K,G", [(1, 4096, 32), (2, 12288, 128), (7, 2176, 64), (16, 4096, 256)])
+def test_dq8ca_decode_workspace_codes(M, K, G):
+    """Up to 16 rows the decode stream quantizes the activations inside the kernel; the
+    workspace still receives them (codes [M, K] at offset 0, then the scales and the zero
+    points, each on a 256-byte boundary) and they are the oracle's choose_qparams bit for
+    bit, including an all-zero row and a row with a single huge value."""
+    N = 300
+    x = wl.normal_bf16((M, K), 1.0, seed=4300 + M)
+    x[0] = 0
+    if M > 1:
+        x[M - 1, K // 3] = 3.0e4
+    W = wl.weight(N, K, seed=4301)
+    q4, gs = q8.q8_quantize_weight_q4gs(W.to(DEV), G)
+    nb = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_DQ8CA_Q4GSW, M, N, K, G)
+    work = torch.full((nb,), 0x5A, dtype=torch.uint8, device=DEV)
+    q8.q8_linear_dq8ca_q4gsw(x.to(DEV), q4, gs, G, workspace=work)
+    torch.cuda.synchronize()
+    w = work.cpu().numpy()
+    rs, rz, rxq = oracle.choose_qparams(wl.bf16_bits(x))
+    off_s = -(-M * K // 256) * 256
+    off_z = off_s + -(-M * 4 // 256) * 256
+    assert np.array_equal(w[:M * K].view(np.int8).reshape(M, K), rxq)
+    assert np.array_equal(w[off_s:off_s + 4 * M].view(np.float32), np.asarray(rs, np.float32))
+    assert np.array_equal(w[off_z:off_z + 4 * M].view(np.int32), np.asarray(rz, np.int32))
+
+
+@pytest.mark.parametrize("M,K", [(300, 256), (5, 256), (16, 4096), (1, 12288), (3, 2304)])
+def test_dq8ca_group_partials_exact(M, K):
+    """Unit group scales: y / s must be the exact integer sum_k (xq - z) q4 (one fp32
+    rounding of s * T).  Above 16 rows this is the bf16 tensor-core path; up to 16 rows the
+    decode stream, whose in-kernel activation codes and zero points must then be the
+    oracle's bit for bit."""
+    N, G = 200, 256
     g = torch.Generator().manual_seed(4242)
-    x = wl.normal_bf16((M, K), 1.0, seed=4243)
+    x = wl.normal_bf16((M, K), 1.0, seed=4243 + M)
     q4 = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, generator=g)   # any nibbles
     gs = torch.ones(N, K // G)
     y = q8.q8_linear_dq8ca_q4gsw(x.to(DEV), q4.to(DEV), gs.to(DEV), G).cpu().numpy()
