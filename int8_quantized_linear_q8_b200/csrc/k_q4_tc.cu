@@ -237,7 +237,10 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
             uint32_t ph = 0, bph = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                int step = 0;                                   // MMA step within the tile
+                // MMA step within the current group (a running counter: this thread issues
+                // every MMA of the CTA, so its loop must stay short -- a modulo per step
+                // made the issue loop, not the tensor core, the limit)
+                int in_group = 0;
                 for (int kb = 0; kb < nk && ok; ++kb) {
                     if (!mbar_wait(&full[st], ph, status, abort_flag)) {
                         ok = false;
@@ -248,8 +251,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                     const uint64_t a = qt_desc_sw128(base);
                     const uint64_t b = qt_desc_sw128(base + C::A_BYTES);
 #pragma unroll
-                    for (int k = 0; k < QT_BK / QT_UK; ++k, ++step) {
-                        const int in_group = step % steps_per_group;
+                    for (int k = 0; k < QT_BK / QT_UK; ++k) {
                         if (in_group == 0) {
                             // a new group: wait until the epilogue has drained this buffer
                             if (!mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag)) {
@@ -260,7 +262,8 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                         }
                         qt_mma_f16(tmem_base + (uint32_t)(buf * BN), a + 2 * k, b + 2 * k, idesc,
                                    in_group != 0);
-                        if (in_group == steps_per_group - 1) {
+                        if (++in_group == steps_per_group) {
+                            in_group = 0;
                             qt_commit(&tfull[buf]);             // group partial ready
                             if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
                         }

@@ -216,17 +216,50 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Non-blocking test of the same phase.  Measured on B200: a try_wait on an already completed
+// phase still costs the issuing thread ~260 cycles, test_wait ~60 -- between the MMAs of a
+// single issuing thread that difference halved the tensor-core rate -- so every wait starts
+// with test_wait and only falls back to the suspending form.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// The same test, but a thread whose phase is not complete is suspended until it completes
+// or `hint_ns` nanoseconds pass.  Waiting threads then take no issue slots from the warps
+// that share their scheduler (a hot spin on try_wait slowed a lone MMA-issuing thread
+// several-fold), and a completed phase still wakes them at once.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+constexpr uint32_t kWaitSleepNs = 20000;        // longest single suspension of a waiter
+
 // Wait for the phase with the given parity to complete.  Returns false, after recording
 // kStatusWaitTimeout in *status and raising the CTA's shared abort flag, if it has not
 // completed within kWaitLimitNs -- or at once if the abort flag is already raised (so
 // that after one expired wait every other wait of the CTA ends quickly too).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
                                           volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
+        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+        if ((i & 7u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 *abort_flag = 1;
@@ -240,11 +273,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int* status,
                                                 volatile int* abort_flag,
                                                 unsigned long long limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
+        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+        if ((i & 7u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
@@ -258,8 +291,9 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, 
 // A drain that runs out of time means a logic error; it is recorded in *status if given.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity,
                                            int* status = nullptr) {
+    if (mbar_test_wait(bar, parity)) return;
     const unsigned long long t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             if (status) atomicExch(status, kStatusWaitTimeout);
             return;
