@@ -17,12 +17,16 @@
 // dimension the activation row m, so an epilogue thread owns one weight row and its
 // group scales are per-thread scalars.
 //
-// Structure (persistent, one CTA per SM, 6 warps): warp 0 TMA producer (128-byte swizzle,
-// 6-stage ring of 32 KB: 128 weight rows + 128 activation rows x 64 K elements);
+// Structure (persistent, one CTA per SM, 10 warps): warp 0 TMA producer (128-byte swizzle;
+// a ring of 6 boxes of 64 K elements per operand, 128 weight rows and BN activation rows:
+// 3 stages of two boxes for G >= 64, so that one barrier round covers 8 MMAs -- a wait
+// between MMAs leaves the tensor pipe idle for a few hundred cycles -- or 6 stages of one
+// box for G = 32, where a group hand-off comes every 2 MMAs anyway);
 // warp 1 tensor-memory allocator and MMA issuer (kind::f16, M = 128, N = BN, K = 16) --
-// one group's MMAs go into one of two accumulator buffers, tcgen05.commit hands it to
-// the epilogue; warps 2-5 epilogue: tcgen05.ld of the group partials, fp32 multiply-add
-// with the group scale into per-thread registers, at the end of a tile y = s[m] * acc.
+// one group's MMAs go into one of NBUF accumulator buffers, tcgen05.commit hands it to
+// the epilogue; warps 2-9 epilogue (two per tensor-memory lane quarter): tcgen05.ld of the
+// group partials, fp32 multiply-add with the group scale into per-thread registers, at
+// the end of a tile y = s[m] * acc.
 #include "q8_kernels.cuh"
 
 namespace q8 {
@@ -57,23 +61,31 @@ __global__ __launch_bounds__(256) void k_q4_expand_bf16(const uint8_t* __restric
 
 // ----------------------------------------------------------------- the GEMM kernel
 constexpr int QT_BM = 128;             // weight rows per tile (tensor-memory lanes)
-constexpr int QT_BK = 64;              // bf16 K elements per stage (128 bytes)
+constexpr int QT_BOXK = 64;            // bf16 K elements per TMA box (one 128-byte swizzle row)
+constexpr int QT_RING = 6;             // TMA boxes per operand in flight (the ring's depth)
 constexpr int QT_UK = 16;              // K per tcgen05.mma.kind::f16
-constexpr int QT_STAGES = 6;
 constexpr int QT_EPI_WARPS = 8;       // two per tensor-memory lane quarter (column halves)
 constexpr int QT_THREADS = (2 + QT_EPI_WARPS) * 32;
 constexpr int QT_NBUF_MAX = 4;        // group accumulator buffers in tensor memory (<= 512 cols)
 
-template <int BN>
+// KB boxes per operand and stage: 2 (8 MMAs per barrier round, 3 stages) where a group
+// spans at least 4 MMAs; with G = 32 a group handshake comes every 2 MMAs anyway and the
+// deeper 6-stage ring of single boxes is faster (measured).
+template <int BN, int KB>
 struct QtCfg {
-    static constexpr int A_BYTES = QT_BM * QT_BK * 2;      // 16 KB
-    static constexpr int B_BYTES = BN * QT_BK * 2;
+    static constexpr int KBOX = KB;
+    static constexpr int BK = QT_BOXK * KB;                // K elements per stage
+    static constexpr int STAGES = QT_RING / KB;
+    static constexpr int A_BOX = QT_BM * QT_BOXK * 2;      // 16 KB
+    static constexpr int B_BOX = BN * QT_BOXK * 2;
+    static constexpr int A_BYTES = A_BOX * KB;
+    static constexpr int B_BYTES = B_BOX * KB;
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int NBUF = 512 / BN < QT_NBUF_MAX ? 512 / BN : QT_NBUF_MAX;
     static constexpr int TMEM_COLS = NBUF * BN < 32 ? 32 : NBUF * BN;
     static_assert(NBUF >= 2 && NBUF * BN <= 512, "tensor memory");
     static constexpr int HALF = BN / 2;                    // columns per epilogue warp
-    static constexpr size_t SMEM = (size_t)QT_STAGES * STAGE + 4096;
+    static constexpr size_t SMEM = (size_t)STAGES * STAGE + 4096;
 };
 
 // acc.xy += g * r.xy as one packed fp32x2 multiply-add
@@ -144,18 +156,18 @@ __device__ __forceinline__ void qt_ld32(uint32_t taddr, float (&r)[32]) {
     for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
 
-template <int BN>
+template <int BN, int KB>
 __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
     const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
     const float* __restrict__ gs, const float* __restrict__ s, float* __restrict__ y, int G,
     int M, int N, int K, int* status) {
-    using C = QtCfg<BN>;
+    using C = QtCfg<BN, KB>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t* ctrl = smem + (size_t)QT_STAGES * C::STAGE;
+    uint8_t* ctrl = smem + (size_t)C::STAGES * C::STAGE;
     uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
-    uint64_t* empty = full + QT_STAGES;
-    uint64_t* tfull = empty + QT_STAGES;     // [NBUF] group accumulator ready
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* tfull = empty + C::STAGES;     // [NBUF] group accumulator ready
     uint64_t* tempty = tfull + C::NBUF;      // [NBUF] group accumulator drained
     uint64_t* mma_done = tempty + C::NBUF;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -167,12 +179,12 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
     const int num_n = (N + QT_BM - 1) / QT_BM;                  // weight-row tiles
     const int num_m = (M + BN - 1) / BN;                        // activation-row tiles
     const int tiles = num_n * num_m;
-    const int nk = K / QT_BK;                                   // K % 128 == 0
+    const int nk = K / C::BK;                                   // K % 128 == 0
     const int steps_per_group = G / QT_UK;
     const int ngroups = K / G;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < QT_STAGES; ++i) {
+        for (int i = 0; i < C::STAGES; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
@@ -220,14 +232,19 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                     uint8_t* base = smem + (size_t)st * C::STAGE;
                     mbar_expect_tx(&full[st], (uint32_t)C::STAGE);
                     // the tensor maps view the bf16 matrices as bytes: K offset in bytes
-                    tma_load_2d_hint(base, &amap, kb * QT_BK * 2, n0, &full[st], drop);
-                    tma_load_2d_hint(base + C::A_BYTES, &bmap, kb * QT_BK * 2, m0, &full[st], keep);
+#pragma unroll
+                    for (int h = 0; h < C::KBOX; ++h) {
+                        const int kx = (kb * C::BK + h * QT_BOXK) * 2;
+                        tma_load_2d_hint(base + h * C::A_BOX, &amap, kx, n0, &full[st], drop);
+                        tma_load_2d_hint(base + C::A_BYTES + h * C::B_BOX, &bmap, kx, m0, &full[st],
+                                         keep);
+                    }
                     ++it;
-                    if (++st == QT_STAGES) { st = 0; ph ^= 1u; }
+                    if (++st == C::STAGES) { st = 0; ph ^= 1u; }
                 }
             }
-            for (int i = max(0, it - QT_STAGES); i < it; ++i)
-                mbar_drain(&full[i % QT_STAGES], (uint32_t)(i / QT_STAGES) & 1u, status);
+            for (int i = max(0, it - C::STAGES); i < it; ++i)
+                mbar_drain(&full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1u, status);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
@@ -248,10 +265,13 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                     }
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                     const uint32_t base = smem_u32(smem + (size_t)st * C::STAGE);
-                    const uint64_t a = qt_desc_sw128(base);
-                    const uint64_t b = qt_desc_sw128(base + C::A_BYTES);
 #pragma unroll
-                    for (int k = 0; k < QT_BK / QT_UK; ++k) {
+                    for (int k = 0; k < C::BK / QT_UK; ++k) {
+                        // box k / 4 of each operand, 32-byte K step k % 4 inside its rows
+                        constexpr int KPB = QT_BOXK / QT_UK;
+                        const uint64_t a = qt_desc_sw128(base + (k / KPB) * C::A_BOX) + 2 * (k % KPB);
+                        const uint64_t b =
+                            qt_desc_sw128(base + C::A_BYTES + (k / KPB) * C::B_BOX) + 2 * (k % KPB);
                         if (in_group == 0) {
                             // a new group: wait until the epilogue has drained this buffer
                             if (!mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag)) {
@@ -260,8 +280,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                             }
                             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                         }
-                        qt_mma_f16(tmem_base + (uint32_t)(buf * BN), a + 2 * k, b + 2 * k, idesc,
-                                   in_group != 0);
+                        qt_mma_f16(tmem_base + (uint32_t)(buf * BN), a, b, idesc, in_group != 0);
                         if (++in_group == steps_per_group) {
                             in_group = 0;
                             qt_commit(&tfull[buf]);             // group partial ready
@@ -269,7 +288,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                         }
                     }
                     qt_commit(&empty[st]);                      // stage free after these MMAs
-                    if (++st == QT_STAGES) { st = 0; ph ^= 1u; }
+                    if (++st == C::STAGES) { st = 0; ph ^= 1u; }
                 }
             }
             qt_commit(mma_done);
@@ -376,15 +395,15 @@ static bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, int64_t rows, 
                            CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <int BN>
+template <int BN, int KB>
 static cudaError_t launch_qt(const uint16_t* wb, const uint16_t* xz, const float* gs,
                              const float* s, float* y, int G, int M, int N, int K,
                              cudaStream_t st, int num_sms, int* status) {
-    using C = QtCfg<BN>;
+    using C = QtCfg<BN, KB>;
     CUtensorMap ma, mb;
-    if (!make_tmap_bf16_2d(&ma, wb, N, K, QT_BK, QT_BM)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_2d(&mb, xz, M, K, QT_BK, BN)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(k_q4_gemm_tc<BN>,
+    if (!make_tmap_bf16_2d(&ma, wb, N, K, QT_BOXK, QT_BM)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&mb, xz, M, K, QT_BOXK, BN)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(k_q4_gemm_tc<BN, KB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(C::SMEM + 1024));
     if (e != cudaSuccess) return e;
@@ -400,7 +419,7 @@ static cudaError_t launch_qt(const uint16_t* wb, const uint16_t* xz, const float
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_q4_gemm_tc<BN>, ma, mb, gs, s, y, G, M, N, K, status);
+    return cudaLaunchKernelEx(&cfg, k_q4_gemm_tc<BN, KB>, ma, mb, gs, s, y, G, M, N, K, status);
 }
 
 cudaError_t launch_q4_expand_bf16(const uint8_t* q4, int64_t N, int K, uint16_t* wb,
@@ -418,8 +437,10 @@ cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const floa
                               const float* s, float* y, int G, int64_t M, int64_t N, int K,
                               cudaStream_t st, int num_sms, int* status) {
     if (M <= 64)
-        return launch_qt<64>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
-    return launch_qt<128>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
+        return G == 32 ? launch_qt<64, 1>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status)
+                       : launch_qt<64, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
+    return G == 32 ? launch_qt<128, 1>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status)
+                   : launch_qt<128, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
 }
 
 }  // namespace q8
