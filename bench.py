@@ -301,20 +301,22 @@ def time_graphs(graphs, steps: int, warmup: int, dist: Dist):
     return dist.max(ms), t0, t1
 
 
-def per_case_times(sweep: W8A16Sweep, reps: int = 20):
+def per_case_times(sweep: W8A16Sweep, reps: int = 20, launch=None):
     """Average device time of each case's kernel, alone, from a graph of `reps` launches
-    alternating weight copies (events on the launching stream)."""
+    alternating weight copies (events on the launching stream).  `launch(i, M, copy)`
+    defaults to the sweep's own q8_linear_w8a16 launch."""
+    launch = launch or sweep.launch
     out = []
     for i, M in sweep.cases:
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            sweep.launch(i, M, 0)
+            launch(i, M, 0)
         torch.cuda.current_stream().wait_stream(s)
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr):
             for r in range(reps):
-                sweep.launch(i, M, r % sweep.COPIES)
+                launch(i, M, r % sweep.COPIES)
         gr.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -460,6 +462,26 @@ def bench_w8a8_prefill(dev, peaks, reps=5):
                         "frac_int8_peak": round(tops / int8_peak_tops(peaks), 4)})
         del x, q, s, ws, y, work
     return out
+
+
+def planes_case_times(sweep: W8A16Sweep):
+    """The sweep's cases through q8_linear_w8a16_planes (int8 tensor cores over exact digit
+    planes of the activations), timed like the headline's per-case times."""
+    q8 = sweep.q8
+    ws = {}
+
+    def launch(i, M, copy):
+        sh, copies, s = sweep.shapes[i]
+        if (i, M) not in ws:
+            n = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A16_PLANES, M, sh.N, sh.K)
+            ws[(i, M)] = torch.zeros(max(n, 16), dtype=torch.uint8, device=copies[0].device)
+        q8.q8_linear_w8a16_planes(sweep.xs[(i, M)], copies[copy], s, ws[(i, M)],
+                                  y=sweep.ys[(i, M)])
+
+    out = per_case_times(sweep, launch=launch)
+    total_b = sum(w8a16_bytes(c["M"], c["N"], c["K"]) for c in out)
+    total_us = sum(c["us"] for c in out)
+    return {"cases": out, "GBps_sum_of_cases": round(total_b / total_us / 1e3, 1)}
 
 
 def bench_q4(dev, peaks, reps=5):
@@ -673,6 +695,7 @@ def run_ours(args):
         result["cpu_baseline"] = cpu_baseline_w8a16(sweep)
     if dist.rank == 0 and not args.no_paths:
         result["paths"] = {
+            "w8a16_planes": planes_case_times(sweep),
             "w8a8_static_k960": bench_w8a8_paths(dev),
             "w8a8_prefill_m4096": bench_w8a8_prefill(dev, peaks),
             "dq8ca_q4gsw": bench_q4(dev, peaks),
