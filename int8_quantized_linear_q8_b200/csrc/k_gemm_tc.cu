@@ -46,7 +46,8 @@ struct TcCfg {
     static constexpr int STAGE_BYTES = A_TILES * A_BYTES + B_BYTES;   // 48 KB
     static constexpr int ACC_COLS = TWO ? 2 * BN : BN;         // per accumulator buffer
     static_assert(2 * ACC_COLS <= TC_TMEM_COLS, "tensor memory");
-    static constexpr size_t SMEM = (size_t)TC_STAGES * STAGE_BYTES + 8192;   // + control
+    // + control (8 KB) + the epilogue's store-transpose tiles (4 warps x 32 x 36 floats)
+    static constexpr size_t SMEM = (size_t)TC_STAGES * STAGE_BYTES + 8192 + 4 * 32 * 36 * 4;
 };
 
 struct TcEpi {
@@ -127,6 +128,7 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* epi_sw = reinterpret_cast<float*>(ctrl + 1024);      // [2][256]
     int* epi_ws = reinterpret_cast<int*>(ctrl + 1024 + 2048);   // [2][256] (ends at 5 KB)
+    float* epi_tile = reinterpret_cast<float*>(ctrl + 8192);     // [4 warps][32][36]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_m = (M + TC_BM - 1) / TC_BM;
@@ -294,18 +296,34 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
                     }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] *= sw[j];
-                    if (m < M) {
-                        float* out = ep.y + (int64_t)m * N + nb;
-                        if (nb + 32 <= N && (N & 3) == 0) {
+                    // Each thread holds one output row; written directly, every store
+                    // instruction would touch 32 rows.  Transpose the warp's 32 x 32 chunk
+                    // through shared memory (rows padded to 36 floats: conflict-free
+                    // 16-byte accesses) so that each store covers 4 rows x 128 bytes.
+                    float* tile = epi_tile + (warp - 2) * (32 * 36);
 #pragma unroll
-                            for (int j = 0; j < 32; j += 4)
-                                *reinterpret_cast<float4*>(out + j) =
-                                    make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-                        } else {
-                            for (int j = 0; j < 32; ++j)
-                                if (nb + j < N) out[j] = v[j];
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(tile + lane * 36 + j) =
+                            make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                    __syncwarp();
+                    const int cc = (lane & 7) * 4;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = 4 * i + (lane >> 3);
+                        const float4 w = *reinterpret_cast<const float4*>(tile + r * 36 + cc);
+                        const int mr = m0 + q * 32 + r;
+                        if (mr < M) {
+                            float* out = ep.y + (int64_t)mr * N + nb + cc;
+                            if (nb + cc + 4 <= N && (N & 3) == 0) {
+                                *reinterpret_cast<float4*>(out) = w;
+                            } else {
+                                const float wv[4] = {w.x, w.y, w.z, w.w};
+                                for (int u = 0; u < 4; ++u)
+                                    if (nb + cc + u < N) out[u] = wv[u];
+                            }
                         }
                     }
+                    __syncwarp();                       // the tile is rewritten next chunk
                 }
             }
             tc_fence_before();
