@@ -63,6 +63,8 @@ __global__ __launch_bounds__(256) void k_q4_expand_bf16(const uint8_t* __restric
 constexpr int QT_BM = 128;             // weight rows per tile (tensor-memory lanes)
 constexpr int QT_BOXK = 64;            // bf16 K elements per TMA box (one 128-byte swizzle row)
 constexpr int QT_RING = 6;             // TMA boxes per operand in flight (the ring's depth)
+constexpr int Q4TC_WIDE_M = 2048;      // activation rows from which tiles are 256 rows wide
+constexpr int Q4TC_WIDE_G = 64;        // ... for groups of at least this many codes
 constexpr int QT_UK = 16;              // K per tcgen05.mma.kind::f16
 constexpr int QT_EPI_WARPS = 8;       // two per tensor-memory lane quarter (column halves)
 constexpr int QT_THREADS = (2 + QT_EPI_WARPS) * 32;
@@ -75,7 +77,10 @@ template <int BN, int KB>
 struct QtCfg {
     static constexpr int KBOX = KB;
     static constexpr int BK = QT_BOXK * KB;                // K elements per stage
-    static constexpr int STAGES = QT_RING / KB;
+    static constexpr int STAGE_SZ = (QT_BM + BN) * QT_BOXK * 2 * KB;
+    // QT_RING / KB stages, as many as fit next to the control region (192 KB of ring)
+    static constexpr int STAGES =
+        (QT_RING / KB) * STAGE_SZ <= 196608 ? QT_RING / KB : 196608 / STAGE_SZ;
     static constexpr int A_BOX = QT_BM * QT_BOXK * 2;      // 16 KB
     static constexpr int B_BOX = BN * QT_BOXK * 2;
     static constexpr int A_BYTES = A_BOX * KB;
@@ -316,7 +321,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
             bool live = true;
             // Group scales stream in chunks of 16 groups, one chunk ahead of their use: a
             // group's MMAs take ~10^2 cycles, an L2 round trip several hundred.
-            constexpr int GC = 16;
+            constexpr int GC = HC > 64 ? 8 : 16;      // (register budget with 128 columns)
             float gcur[GC], gnxt[GC];
             auto load_chunk = [&](float (&dst)[GC], int g0) {
 #pragma unroll
@@ -349,16 +354,23 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                 if (live) {
                     const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
                                            (uint32_t)(buf * BN + half * HC);
-                    uint32_t u[HC / 32][32];
+                    // 32-column chunks, up to two per tensor-memory wait (with 128 columns
+                    // per warp one at a time: 128 fp32 sums already take the registers)
+                    constexpr int NCH = HC / 32;
+                    constexpr int LB = NCH <= 2 ? NCH : 1;
 #pragma unroll
-                    for (int c = 0; c < HC / 32; ++c) qt_ld32_nowait(taddr + c * 32, u[c]);
-                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    for (int c0 = 0; c0 < NCH; c0 += LB) {
+                        uint32_t u[LB][32];
 #pragma unroll
-                    for (int c = 0; c < HC / 32; ++c)
+                        for (int c = 0; c < LB; ++c) qt_ld32_nowait(taddr + (c0 + c) * 32, u[c]);
+                        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2)
-                            ffma2(acc[c * 32 + j], acc[c * 32 + j + 1], gcur_v,
-                                  __uint_as_float(u[c][j]), __uint_as_float(u[c][j + 1]));
+                        for (int c = 0; c < LB; ++c)
+#pragma unroll
+                            for (int j = 0; j < 32; j += 2)
+                                ffma2(acc[(c0 + c) * 32 + j], acc[(c0 + c) * 32 + j + 1], gcur_v,
+                                      __uint_as_float(u[c][j]), __uint_as_float(u[c][j + 1]));
+                    }
                 }
                 asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                 __syncwarp();
@@ -439,6 +451,12 @@ cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const floa
     if (M <= 64)
         return G == 32 ? launch_qt<64, 1>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status)
                        : launch_qt<64, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
+    // 256 activation rows per tile where there are enough of them to keep the tiles
+    // balanced over the SMs: each MMA does twice the work for the same per-group hand-off.
+    // Not for small groups: the epilogue (128 columns per warp, one tensor-memory chunk at
+    // a time, registers short) then falls behind the MMAs (G = 32: 1062 -> 1395 us).
+    if (M >= Q4TC_WIDE_M && G >= Q4TC_WIDE_G)
+        return launch_qt<256, 1>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
     return G == 32 ? launch_qt<128, 1>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status)
                    : launch_qt<128, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
 }

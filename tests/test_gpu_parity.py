@@ -394,7 +394,9 @@ def test_dq8ca_q4gsw_config(M, G):
                                      (2, 1000, 2176, 32), (16, 4097, 4096, 128),
                                      (8, 2000, 6144, 64), (12, 700, 4224, 32), (4, 11008, 4096, 256),
                                      # rows longer than the stream keeps in registers
-                                     (1, 300, 12288, 64), (3, 500, 10240, 128)])
+                                     (1, 300, 12288, 64), (3, 500, 10240, 128),
+                                     # 256-row activation tiles: ragged last tile, odd N
+                                     (2100, 300, 512, 64), (2048, 129, 256, 256)])
 def test_dq8ca_q4gsw_ragged(M, N, K, G):
     x, q4, gs, y = _q4_case(M, N, K, G, 900 + M, 901 + N)
     s, z, xq = oracle.choose_qparams(wl.bf16_bits(x))
