@@ -70,9 +70,11 @@ constexpr int QT_EPI_WARPS = 8;       // two per tensor-memory lane quarter (col
 constexpr int QT_THREADS = (2 + QT_EPI_WARPS) * 32;
 constexpr int QT_NBUF_MAX = 4;        // group accumulator buffers in tensor memory (<= 512 cols)
 
-// KB boxes per operand and stage: 2 (8 MMAs per barrier round, 3 stages) where a group
-// spans at least 4 MMAs; with G = 32 a group handshake comes every 2 MMAs anyway and the
-// deeper 6-stage ring of single boxes is faster (measured).
+// KB boxes per operand and stage: 2 (8 MMAs per barrier round; 3 stages with 128-row
+// tiles, 2 with 256) where a group spans at least 4 MMAs -- even with only two stages
+// that beats 4 stages of one box (measured, 256-row tiles, G = 128: 576 -> 472 us); with
+// G = 32 a group hand-off comes every 2 MMAs anyway and the deeper 6-stage ring of single
+// boxes is faster.
 template <int BN, int KB>
 struct QtCfg {
     static constexpr int KBOX = KB;
@@ -456,7 +458,7 @@ cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const floa
     // Not for small groups: the epilogue (128 columns per warp, one tensor-memory chunk at
     // a time, registers short) then falls behind the MMAs (G = 32: 1062 -> 1395 us).
     if (M >= Q4TC_WIDE_M && G >= Q4TC_WIDE_G)
-        return launch_qt<256, 1>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
+        return launch_qt<256, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
     return G == 32 ? launch_qt<128, 1>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status)
                    : launch_qt<128, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
 }
