@@ -401,6 +401,326 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
     }
 }
 
+// ------------------------------------------------- fused variant for small M (M <= 64)
+//
+// The same GEMM, but the weight operand is built inside the kernel: TMA brings the packed
+// int4 rows (128 rows x 32 bytes per 64-K box, 4x fewer bytes than the bf16 matrix), and
+// four converter warps write them into the 128-byte-swizzled bf16 A tile (thread r owns
+// weight row r).  Each code becomes an exact bf16 integer in three operations per pair:
+// the offset nibble v = nibble ^ 8 (= code + 8) is placed in the mantissa of 0x4300
+// (bf16 128 + v, exact: the unit in the last place of [128, 256) is 1), and a bf16x2
+// subtraction of 136 leaves the code.  The converters fence the async proxy and arrive on
+// the stage's "A ready" barrier; the MMA issuer waits only on that barrier (the converters
+// waited for the stage's TMA bytes, activations included).  No global bf16 weight copy.
+constexpr int QF_CONV_WARPS = 4;
+constexpr int QF_THREADS = (2 + QF_CONV_WARPS + QT_EPI_WARPS) * 32;
+
+template <int BN, int KB>
+struct QfCfg {
+    static constexpr int KBOX = KB;
+    static constexpr int BK = QT_BOXK * KB;
+    static constexpr int A_BOX = QT_BM * QT_BOXK * 2;      // 16 KB of bf16 weight per box
+    static constexpr int B_BOX = BN * QT_BOXK * 2;
+    static constexpr int A_BYTES = A_BOX * KB;
+    static constexpr int B_BYTES = B_BOX * KB;
+    static constexpr int Q_ROW = QT_BOXK / 2 * KB;         // packed bytes per weight row
+    static constexpr int Q_BYTES = QT_BM * Q_ROW;
+    static constexpr int STAGE = A_BYTES + B_BYTES + Q_BYTES;
+    static constexpr int STAGES = 196608 / STAGE < 6 ? 196608 / STAGE : 6;
+    static constexpr int TX = B_BYTES + Q_BYTES;           // bytes the TMA copies deliver
+    static constexpr int NBUF = 512 / BN < QT_NBUF_MAX ? 512 / BN : QT_NBUF_MAX;
+    static constexpr int TMEM_COLS = NBUF * BN < 32 ? 32 : NBUF * BN;
+    static constexpr int HALF = BN / 2;
+    static constexpr size_t SMEM = (size_t)STAGES * STAGE + 4096;
+    static_assert(STAGES >= 2, "ring");
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
+};
+
+// Packed word w (8 codes, low nibble first) -> 4 words of bf16 pairs (codes 2i, 2i+1)
+__device__ __forceinline__ void q4_word_to_bf16(uint32_t w, uint32_t (&o)[4]) {
+    const uint32_t v = w ^ 0x88888888u;                    // code + 8 per nibble
+    const uint32_t lo = v & 0x0F0F0F0Fu, hi = (v >> 4) & 0x0F0F0F0Fu;
+    const __nv_bfloat162 off = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)0x4308),
+                                                  __ushort_as_bfloat16((unsigned short)0x4308));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        // bytes [lo_i, -, hi_i, -] -> (128 + v) in both halves
+        const uint32_t t = (__byte_perm(lo, hi, (uint32_t)(i | (i << 4) | ((4 + i) << 8) |
+                                                            ((4 + i) << 12))) &
+                            0x00FF00FFu) | 0x43004300u;
+        __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&t);
+        b = __hsub2(b, off);
+        o[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+}
+
+template <int BN, int KB>
+__global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap bmap,
+    const float* __restrict__ gs, const float* __restrict__ s, float* __restrict__ y, int G,
+    int M, int N, int K, int* status) {
+    using C = QfCfg<BN, KB>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* ctrl = smem + (size_t)C::STAGES * C::STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);      // TMA bytes (activations, codes)
+    uint64_t* aready = full + C::STAGES;                     // bf16 weight tile written
+    uint64_t* empty = aready + C::STAGES;                    // stage's MMAs complete
+    uint64_t* tfull = empty + C::STAGES;
+    uint64_t* tempty = tfull + C::NBUF;
+    uint64_t* mma_done = tempty + C::NBUF;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* s_tile = reinterpret_cast<float*>(ctrl + 512);
+    static_assert(512 + 4 * BN <= 4096, "control region");
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_n = (N + QT_BM - 1) / QT_BM;
+    const int num_m = (M + BN - 1) / BN;
+    const int tiles = num_n * num_m;
+    const int nk = K / C::BK;                                  // K % 128 == 0
+    const int steps_per_group = G / QT_UK;
+    const int ngroups = K / G;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&aready[i], QF_CONV_WARPS);
+            mbar_init(&empty[i], 1);
+        }
+        for (int a = 0; a < C::NBUF; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], QT_EPI_WARPS);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem_base = *tmem_slot;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            tma_prefetch_desc(&qmap);
+            tma_prefetch_desc(&bmap);
+            const uint64_t keep = make_l2_policy_evict_last();   // activations: re-read
+            const uint64_t drop = make_l2_policy_evict_first();  // weight codes
+            int st = 0, it = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int n0 = (t / num_m) * QT_BM, m0 = (t % num_m) * BN;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&empty[st], ph ^ 1u, status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* base = smem + (size_t)st * C::STAGE;
+                    mbar_expect_tx(&full[st], (uint32_t)C::TX);
+#pragma unroll
+                    for (int h = 0; h < C::KBOX; ++h)
+                        tma_load_2d_hint(base + C::A_BYTES + h * C::B_BOX, &bmap,
+                                         (kb * C::BK + h * QT_BOXK) * 2, m0, &full[st], keep);
+                    tma_load_2d_hint(base + C::A_BYTES + C::B_BYTES, &qmap, kb * C::BK / 2, n0,
+                                     &full[st], drop);
+                    ++it;
+                    if (++st == C::STAGES) { st = 0; ph ^= 1u; }
+                }
+            }
+            for (int i = max(0, it - C::STAGES); i < it; ++i)
+                mbar_drain(&full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1u, status);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = qt_idesc_bf16(QT_BM, BN);
+            int st = 0, buf = 0;
+            uint32_t ph = 0, bph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                int in_group = 0;                  // MMA step within the current group
+                for (int kb = 0; kb < nk && ok; ++kb) {
+                    if (!mbar_wait(&aready[st], ph, status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const uint32_t base = smem_u32(smem + (size_t)st * C::STAGE);
+#pragma unroll
+                    for (int k = 0; k < C::BK / QT_UK; ++k) {
+                        constexpr int KPB = QT_BOXK / QT_UK;
+                        const uint64_t a = qt_desc_sw128(base + (k / KPB) * C::A_BOX) + 2 * (k % KPB);
+                        const uint64_t b = qt_desc_sw128(base + C::A_BYTES + (k / KPB) * C::B_BOX) +
+                                           2 * (k % KPB);
+                        if (in_group == 0) {
+                            if (!mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                        }
+                        qt_mma_f16(tmem_base + (uint32_t)(buf * BN), a, b, idesc, in_group != 0);
+                        if (++in_group == steps_per_group) {
+                            in_group = 0;
+                            qt_commit(&tfull[buf]);
+                            if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
+                        }
+                    }
+                    qt_commit(&empty[st]);
+                    if (++st == C::STAGES) { st = 0; ph ^= 1u; }
+                }
+            }
+            qt_commit(mma_done);
+            mbar_drain(mma_done, 0, status);
+        }
+        __syncwarp();
+    } else if (warp < 2 + QF_CONV_WARPS) {
+        // ---------------------------------------------------------------- converters
+        // thread r: weight row r of the tile, its Q_ROW packed bytes -> 8 * KB 16-byte
+        // chunks of bf16 codes, chunk c of box h at row r, position c ^ (r % 8)
+        const int r = (warp - 2) * 32 + lane;
+        int st = 0;
+        uint32_t ph = 0;
+        bool live = true;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+            for (int kb = 0; kb < nk; ++kb) {
+                const bool okw = mbar_wait(&full[st], ph, status, abort_flag);
+                live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
+                uint8_t* base = smem + (size_t)st * C::STAGE;
+                if (live) {
+                    const uint32_t qrow = smem_u32(base + C::A_BYTES + C::B_BYTES + r * C::Q_ROW);
+#pragma unroll
+                    for (int h = 0; h < C::KBOX; ++h) {
+                        uint4 qw[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u)
+                            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                                         : "=r"(qw[u].x), "=r"(qw[u].y), "=r"(qw[u].z), "=r"(qw[u].w)
+                                         : "r"(qrow + (uint32_t)(h * 32 + u * 16)));
+                        const uint32_t words[8] = {qw[0].x, qw[0].y, qw[0].z, qw[0].w,
+                                                   qw[1].x, qw[1].y, qw[1].z, qw[1].w};
+                        const uint32_t arow = smem_u32(base + h * C::A_BOX + r * 128);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            uint32_t o[4];
+                            q4_word_to_bf16(words[c], o);
+                            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(
+                                             arow + (uint32_t)((c ^ (r & 7)) << 4)),
+                                         "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                                         : "memory");
+                        }
+                    }
+                }
+                // make the generic-proxy writes visible to the tensor core, then hand over
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&aready[st]);
+                if (++st == C::STAGES) { st = 0; ph ^= 1u; }
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        // warp w (6..13): lane quarter w % 4 of the weight rows, column half (w - 6) / 4
+        const int q = warp & 3;
+        const int half = (warp - 2 - QF_CONV_WARPS) >> 2;
+        const int et = threadIdx.x - 32 * (2 + QF_CONV_WARPS);
+        constexpr int HC = C::HALF;
+        int buf = 0;
+        uint32_t bph = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+            const int n0 = (t / num_m) * QT_BM, m0 = (t % num_m) * BN;
+            const int n = n0 + q * 32 + lane;
+            for (int j = et; j < BN; j += 32 * QT_EPI_WARPS)
+                s_tile[j] = (m0 + j < M) ? __ldg(s + m0 + j) : 0.f;
+            const float* gsr = gs + (int64_t)(n < N ? n : 0) * ngroups;
+            float acc[HC];
+#pragma unroll
+            for (int j = 0; j < HC; ++j) acc[j] = 0.0f;
+            bool live = true;
+            // group scales in chunks of 16 groups, one chunk ahead (a group's MMAs are far
+            // shorter than an L2 round trip)
+            constexpr int GC = 16;
+            float gcur[GC], gnxt[GC];
+            auto load_chunk = [&](float (&dst)[GC], int g0) {
+#pragma unroll
+                for (int i = 0; i < GC; i += 4) {
+                    if ((ngroups & 3) == 0 && g0 + i + 3 < ngroups) {
+                        const float4 v = __ldg(reinterpret_cast<const float4*>(gsr + g0 + i));
+                        dst[i] = v.x; dst[i + 1] = v.y; dst[i + 2] = v.z; dst[i + 3] = v.w;
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            dst[i + u] = (g0 + i + u < ngroups) ? __ldg(gsr + g0 + i + u) : 0.f;
+                    }
+                }
+            };
+            load_chunk(gnxt, 0);
+            for (int gi = 0; gi < ngroups; ++gi) {
+                if (gi % GC == 0) {
+#pragma unroll
+                    for (int i = 0; i < GC; ++i) gcur[i] = gnxt[i];
+                    if (gi + GC < ngroups) load_chunk(gnxt, gi + GC);
+                }
+                float gcur_v = gcur[0];
+#pragma unroll
+                for (int i = 1; i < GC; ++i) gcur_v = (gi % GC == i) ? gcur[i] : gcur_v;
+                const bool okw = mbar_wait(&tfull[buf], bph, status, abort_flag);
+                live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                if (live) {
+                    const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
+                                           (uint32_t)(buf * BN + half * HC);
+                    constexpr int NCH = HC / 32;
+                    uint32_t u[NCH][32];
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c) qt_ld32_nowait(taddr + c * 32, u[c]);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2)
+                            ffma2(acc[c * 32 + j], acc[c * 32 + j + 1], gcur_v,
+                                  __uint_as_float(u[c][j]), __uint_as_float(u[c][j + 1]));
+                }
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+                if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
+            }
+            named_bar_sync(2, 32 * QT_EPI_WARPS);
+            if (live && n < N) {
+#pragma unroll
+                for (int j = 0; j < HC; ++j) {
+                    const int m = m0 + half * HC + j;
+                    if (m < M) st_stream_f32(y + (int64_t)m * N + n, s_tile[half * HC + j] * acc[j]);
+                }
+            }
+            named_bar_sync(2, 32 * QT_EPI_WARPS);
+        }
+    }
+
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
 // ----------------------------------------------------------------------- host side
 static bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
                               int box_cols, int box_rows) {
@@ -434,6 +754,46 @@ static cudaError_t launch_qt(const uint16_t* wb, const uint16_t* xz, const float
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k_q4_gemm_tc<BN, KB>, ma, mb, gs, s, y, G, M, N, K, status);
+}
+
+template <int BN, int KB>
+static cudaError_t launch_qf(const uint8_t* q4, const uint16_t* xz, const float* gs,
+                             const float* s, float* y, int G, int M, int N, int K,
+                             cudaStream_t st, int num_sms, int* status) {
+    using C = QfCfg<BN, KB>;
+    CUtensorMap mq, mb;
+    if (!make_tmap_u8_2d(&mq, q4, N, K / 2, C::Q_ROW, QT_BM, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&mb, xz, M, K, QT_BOXK, BN)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(k_q4_gemm_fused<BN, KB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(C::SMEM + 1024));
+    if (e != cudaSuccess) return e;
+    const int tiles = ((N + QT_BM - 1) / QT_BM) * ((M + BN - 1) / BN);
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(QF_THREADS);
+    cfg.dynamicSmemBytes = C::SMEM + 1024;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_q4_gemm_fused<BN, KB>, mq, mb, gs, s, y, G, M, N, K,
+                              status);
+}
+
+// Up to 64 activation rows the weight is expanded inside the GEMM (no bf16 copy in HBM).
+bool q4_tc_fused(int64_t M) { return M <= 64; }
+
+cudaError_t launch_q4_gemm_fused(const uint8_t* q4, const uint16_t* xz, const float* gs,
+                                 const float* s, float* y, int G, int64_t M, int64_t N, int K,
+                                 cudaStream_t st, int num_sms, int* status) {
+    return G == 32
+               ? launch_qf<64, 1>(q4, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status)
+               : launch_qf<64, 2>(q4, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
 }
 
 cudaError_t launch_q4_expand_bf16(const uint8_t* q4, int64_t N, int K, uint16_t* wb,

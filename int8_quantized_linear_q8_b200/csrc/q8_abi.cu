@@ -139,7 +139,9 @@ static Q4Plan plan_q4(int64_t M, int64_t N, int64_t K) {
     p.s = align_up(codes, 256);
     p.z = p.s + align_up((size_t)M * 4, 256);
     p.wb = p.z + align_up((size_t)M * 4, 256);
-    p.bytes = p.wb + (p.tc ? align_up((size_t)N * (size_t)K * 2, 256) : 0);
+    // the bf16 copy of the weight only where the GEMM does not expand the codes itself
+    const bool wb = p.tc && !q4_tc_fused(M);
+    p.bytes = p.wb + (wb ? align_up((size_t)N * (size_t)K * 2, 256) : 0);
     return p;
 }
 static inline bool valid_group(int G) { return G == 32 || G == 64 || G == 128 || G == 256; }
@@ -375,6 +377,10 @@ q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* g
     int32_t* z = (int32_t*)(ws + plan.z);
     if (plan.tc) {
         uint16_t* xz = (uint16_t*)(ws + plan.xq);
+        if (q4_tc_fused(M)) {
+            Q8_TRY(launched(launch_choose_qparams_shifted((const uint16_t*)x, M, (int)K, s, z, xz, st)));
+            return launched(launch_q4_gemm_fused(q4, xz, gs, s, y, G, M, N, (int)K, st, sms, status));
+        }
         uint16_t* wb = (uint16_t*)(ws + plan.wb);
         Q8_TRY(launched(launch_q4_expand_bf16(q4, N, (int)K, wb, st, sms)));
         Q8_TRY(launched(launch_choose_qparams_shifted((const uint16_t*)x, M, (int)K, s, z, xz, st)));

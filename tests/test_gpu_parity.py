@@ -396,7 +396,10 @@ def test_dq8ca_q4gsw_config(M, G):
                                      # rows longer than the stream keeps in registers
                                      (1, 300, 12288, 64), (3, 500, 10240, 128),
                                      # 256-row activation tiles: ragged last tile, odd N
-                                     (2100, 300, 512, 64), (2048, 129, 256, 256)])
+                                     (2100, 300, 512, 64), (2048, 129, 256, 256),
+                                     # 17..64 rows: the GEMM expands the int4 codes itself
+                                     (33, 1000, 2176, 64), (64, 300, 4096, 256),
+                                     (20, 129, 128, 32), (50, 257, 1024, 128)])
 def test_dq8ca_q4gsw_ragged(M, N, K, G):
     x, q4, gs, y = _q4_case(M, N, K, G, 900 + M, 901 + N)
     s, z, xq = oracle.choose_qparams(wl.bf16_bits(x))
@@ -430,12 +433,13 @@ def test_dq8ca_decode_workspace_codes(M, K, G):
     assert np.array_equal(w[off_z:off_z + 4 * M].view(np.int32), np.asarray(rz, np.int32))
 
 
-@pytest.mark.parametrize("M,K", [(300, 256), (5, 256), (16, 4096), (1, 12288), (3, 2304)])
+@pytest.mark.parametrize("M,K", [(300, 256), (5, 256), (16, 4096), (1, 12288), (3, 2304),
+                                 (40, 512)])
 def test_dq8ca_group_partials_exact(M, K):
     """Unit group scales: y / s must be the exact integer sum_k (xq - z) q4 (one fp32
-    rounding of s * T).  Above 16 rows this is the bf16 tensor-core path; up to 16 rows the
-    decode stream, whose in-kernel activation codes and zero points must then be the
-    oracle's bit for bit."""
+    rounding of s * T).  Above 16 rows this is the bf16 tensor-core path (17..64 rows with the
+    int4 -> bf16 expansion inside the GEMM); up to 16 rows the decode stream, whose in-kernel
+    activation codes and zero points must then be the oracle's bit for bit."""
     N, G = 200, 256
     g = torch.Generator().manual_seed(4242)
     x = wl.normal_bf16((M, K), 1.0, seed=4243 + M)
