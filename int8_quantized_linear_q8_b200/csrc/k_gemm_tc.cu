@@ -27,7 +27,9 @@
 
 namespace q8 {
 
-enum { EPI_S32 = 0, EPI_W8A8 = 1, EPI_TWO = 2 };
+// EPI_W8A8_N128: the one-pass epilogue on 128-row weight tiles (for grids that 256-row
+// tiles would leave unbalanced)
+enum { EPI_S32 = 0, EPI_W8A8 = 1, EPI_TWO = 2, EPI_W8A8_N128 = 3 };
 
 constexpr int TC_BM = 128;          // accumulator rows (= tensor-memory lanes)
 constexpr int TC_BK = 128;          // bytes of K per stage (one 128-byte swizzle row)
@@ -39,7 +41,7 @@ constexpr int TC_TMEM_COLS = 512;
 template <int EPI>
 struct TcCfg {
     static constexpr bool TWO = EPI == EPI_TWO;
-    static constexpr int BN = TWO ? 128 : 256;                 // weight rows per tile
+    static constexpr int BN = TWO || EPI == EPI_W8A8_N128 ? 128 : 256;   // weight rows per tile
     static constexpr int A_TILES = TWO ? 2 : 1;
     static constexpr int A_BYTES = TC_BM * TC_BK;              // 16 KB
     static constexpr int B_BYTES = BN * TC_BK;
@@ -396,6 +398,12 @@ cudaError_t launch_w8a8_tc(const int8_t* xq1, const int8_t* xq2, float s1, int z
     ep.y = y;
     if (has2)
         return launch_tc<EPI_TWO>(xq1, xq2, q, (int)M, (int)N, K, ep, st, num_sms, status);
+    // 256-row weight tiles unless they would give fewer than two tiles per SM: then the
+    // last round of tiles leaves most SMs idle, and 128-row tiles halve that round
+    const int64_t tiles256 = ((M + TC_BM - 1) / TC_BM) * ((N + 255) / 256);
+    if (tiles256 < 2 * (int64_t)num_sms)
+        return launch_tc<EPI_W8A8_N128>(xq1, nullptr, q, (int)M, (int)N, K, ep, st, num_sms,
+                                        status);
     return launch_tc<EPI_W8A8>(xq1, nullptr, q, (int)M, (int)N, K, ep, st, num_sms, status);
 }
 
