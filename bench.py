@@ -335,21 +335,34 @@ def per_case_times(sweep: W8A16Sweep, reps: int = 20, launch=None):
 
 
 def e2e_w8a16(sweep: W8A16Sweep, steps: int, warmup: int, dist: Dist):
-    """Same metric through the public API with host buffers: every step copies each case's
-    activations host->device (pinned) and reads each output back device->host."""
+    """Same metric through the public API with host buffers: every step copies all the
+    cases' activations host->device (one pinned buffer), runs the 12 calls on views of it,
+    and reads all the outputs back device->host (one pinned buffer)."""
     q8 = sweep.q8
-    hx = {k: v.cpu().pin_memory() for k, v in sweep.xs.items()}
-    hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in sweep.ys.items()}
-    dx = {k: torch.empty_like(v) for k, v in sweep.xs.items()}
-    h2d = sum(v.numel() * v.element_size() for v in hx.values())
-    d2h = sum(v.numel() * v.element_size() for v in hy.values())
+    dev = next(iter(sweep.xs.values())).device
+    # one pinned host buffer for all the step's activations and one for all its outputs;
+    # per-case tensors are views into the matching device buffers
+    keys = list(sweep.cases)
+    nx = [sweep.xs[k].numel() for k in keys]
+    ny = [sweep.ys[k].numel() for k in keys]
+    hx = torch.cat([sweep.xs[k].reshape(-1).cpu() for k in keys]).pin_memory()
+    hy = torch.empty(sum(ny), dtype=torch.bfloat16).pin_memory()
+    dxa = torch.empty(sum(nx), dtype=torch.bfloat16, device=dev)
+    dya = torch.empty(sum(ny), dtype=torch.bfloat16, device=dev)
+    dx, dy, ox, oy = {}, {}, 0, 0
+    for k, a, b in zip(keys, nx, ny):
+        dx[k] = dxa[ox:ox + a].view(sweep.xs[k].shape)
+        dy[k] = dya[oy:oy + b].view(sweep.ys[k].shape)
+        ox, oy = ox + a, oy + b
+    h2d = hx.numel() * hx.element_size()
+    d2h = hy.numel() * hy.element_size()
 
     def step(c):
-        for i, M in sweep.cases:
+        dxa.copy_(hx, non_blocking=True)
+        for i, M in keys:
             sh, copies, s = sweep.shapes[i]
-            dx[(i, M)].copy_(hx[(i, M)], non_blocking=True)
-            q8.q8_linear_w8a16(dx[(i, M)], copies[c], s, y=sweep.ys[(i, M)])
-            hy[(i, M)].copy_(sweep.ys[(i, M)], non_blocking=True)
+            q8.q8_linear_w8a16(dx[(i, M)], copies[c], s, y=dy[(i, M)])
+        hy.copy_(dya, non_blocking=True)
 
     for i in range(warmup):
         step(i % sweep.COPIES)

@@ -357,9 +357,7 @@ static cudaError_t launch_tc(const int8_t* a1, const int8_t* a2, const int8_t* b
         return cudaErrorInvalidValue;
     if (!make_tmap_u8_2d(&mb, b, N, K, TC_BK, C::BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(C::SMEM + 1024));
+    cudaError_t e = ensure_dyn_smem<k_gemm_tc<EPI>>((int)(C::SMEM + 1024));
     if (e != cudaSuccess) return e;
     const int tiles = ((M + TC_BM - 1) / TC_BM) * ((N + C::BN - 1) / C::BN);
     const int grid = tiles < num_sms ? tiles : num_sms;

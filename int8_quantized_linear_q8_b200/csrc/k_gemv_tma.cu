@@ -556,9 +556,7 @@ static cudaError_t launch_wt(const CUtensorMap& map, const uint16_t* x, const fl
     while (stages > 4 && wt_layout<SL>(M, K, MT, stages, XT).total > (size_t)WT_MAX_SMEM)
         --stages;
     const WtSmem L = wt_layout<SL>(M, K, MT, stages, XT);
-    cudaError_t e = cudaFuncSetAttribute(k_w8a16_tma<MT, XT, SL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)L.total);
+    cudaError_t e = ensure_dyn_smem<k_w8a16_tma<MT, XT, SL>>((int)L.total);
     if (e != cudaSuccess) return e;
     const int RG = (N + 15) / 16;
     int grid = RG < num_sms ? RG : num_sms;

@@ -737,9 +737,7 @@ static cudaError_t launch_qt(const uint16_t* wb, const uint16_t* xz, const float
     CUtensorMap ma, mb;
     if (!make_tmap_bf16_2d(&ma, wb, N, K, QT_BOXK, QT_BM)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16_2d(&mb, xz, M, K, QT_BOXK, BN)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(k_q4_gemm_tc<BN, KB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(C::SMEM + 1024));
+    cudaError_t e = ensure_dyn_smem<k_q4_gemm_tc<BN, KB>>((int)(C::SMEM + 1024));
     if (e != cudaSuccess) return e;
     const int tiles = ((N + QT_BM - 1) / QT_BM) * ((M + BN - 1) / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
@@ -765,9 +763,7 @@ static cudaError_t launch_qf(const uint8_t* q4, const uint16_t* xz, const float*
     if (!make_tmap_u8_2d(&mq, q4, N, K / 2, C::Q_ROW, QT_BM, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     if (!make_tmap_bf16_2d(&mb, xz, M, K, QT_BOXK, BN)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(k_q4_gemm_fused<BN, KB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(C::SMEM + 1024));
+    cudaError_t e = ensure_dyn_smem<k_q4_gemm_fused<BN, KB>>((int)(C::SMEM + 1024));
     if (e != cudaSuccess) return e;
     const int tiles = ((N + QT_BM - 1) / QT_BM) * ((M + BN - 1) / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;

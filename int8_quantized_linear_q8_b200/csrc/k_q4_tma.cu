@@ -533,8 +533,7 @@ static cudaError_t launch_qs(const CUtensorMap& qm, const CUtensorMap& gm, const
         --stages;
     const QsSmem L = qs_layout(M, K, G, MT, stages, NC);
     const size_t smem = L.total + 1024;                  // + alignment slack
-    cudaError_t e = cudaFuncSetAttribute(k_q4_tma<MT, SEG, QP, NC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = ensure_dyn_smem<k_q4_tma<MT, SEG, QP, NC>>((int)smem);
     if (e != cudaSuccess) return e;
     const int RG = (N + 15) / 16;
     int grid = RG < num_sms ? RG : num_sms;

@@ -761,8 +761,7 @@ cudaError_t launch_w8a16_tc(const uint16_t* x, const int8_t* q, const float* s_w
     a.epoch = ++g_wc_epoch;
     a.status = status;
     const size_t smem = wc_smem_bytes((int)M);
-    cudaError_t e = cudaFuncSetAttribute(k_w8a16_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = ensure_dyn_smem<k_w8a16_tc>((int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);

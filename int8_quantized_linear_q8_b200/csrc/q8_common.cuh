@@ -6,6 +6,8 @@
 #include <float.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/q8.h"
 
 #ifndef __CUDACC__
@@ -347,6 +349,30 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(addr));
     return v;
+}
+
+// ---------------------------------------------------------------- host helpers
+
+// Raises kernel K's dynamic shared-memory limit on the current device to at least `bytes`.
+// The attribute persists, so it is set once per size increase instead of before every
+// launch (a per-call runtime call costs host time on decode-sized launches).
+template <auto K>
+inline cudaError_t ensure_dyn_smem(int bytes) {
+    static std::atomic<int> set_bytes[128];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+        cudaGetLastError();
+        return cudaErrorInvalidDevice;
+    }
+    if (set_bytes[dev].load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               bytes);
+    if (e == cudaSuccess) {
+        int cur = set_bytes[dev].load(std::memory_order_relaxed);
+        while (cur < bytes && !set_bytes[dev].compare_exchange_weak(cur, bytes)) {
+        }
+    }
+    return e;
 }
 
 }  // namespace q8
