@@ -19,8 +19,11 @@
 //              step, hands the accumulator to the epilogue.  Accumulators are double-
 //              buffered so the epilogue of one tile overlaps the main loop of the next.
 //   warps 2-5: epilogue -- tcgen05.ld of 32 columns at a time (each warp reads its
-//              32-lane quarter of tensor memory), zero-point term and scales in fp32,
-//              128-byte row-contiguous stores.
+//              32-lane quarter of tensor memory), zero-point term and scales in fp32;
+//              each warp's 32 x 32 output chunk goes through a padded shared-memory tile
+//              so that every store instruction covers 4 rows x 128 bytes.
+// Weight tiles are 256 rows (BN), or 128 where 256-row tiles would give fewer than two
+// tiles per SM, and 128 for the two-pass form (two accumulators per tile).
 // Every wait is bounded (abort flag + status word), and tensor memory is released only
 // after the issuing thread has seen all of its MMAs complete.
 #include "q8_kernels.cuh"

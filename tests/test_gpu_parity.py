@@ -360,6 +360,32 @@ def test_w8a8_llama_prefill_sampled(K, N, two):
     check_f32(y.cpu().numpy()[rows], y64, absum, f"W8A8 llama K={K} N={N} two={two}")
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 32000, 4096), (16, 11008, 4096), (4, 2560, 960)])
+def test_w8a16_repeat_bit_identical(M, N, K):
+    """The warps' partial sums are added in a fixed order (no float atomics), so repeated
+    calls give the same bits (wide and narrow stages, 1 and 2 activation tiles)."""
+    W = wl.weight(N, K, seed=880 + M)
+    x = wl.normal_bf16((M, K), 1.0, seed=881 + M).to(DEV)
+    q, s, _ = q8.q8_quantize_weight(W.to(DEV), want_wsum=False)
+    ref = q8.q8_linear_w8a16(x, q, s, out_dtype=torch.float32).cpu()
+    for _ in range(5):
+        y = q8.q8_linear_w8a16(x, q, s, out_dtype=torch.float32).cpu()
+        assert torch.equal(y.view(torch.int32), ref.view(torch.int32))
+
+
+@pytest.mark.parametrize("M,G", [(1, 128), (8, 32), (16, 64)])
+def test_dq8ca_decode_repeat_bit_identical(M, G):
+    """The 8da4w decode stream is deterministic too (fixed-order partial sums)."""
+    N, K = 11008, 4096
+    W = wl.weight(N, K, seed=890 + M)
+    x = wl.normal_bf16((M, K), 1.0, seed=891 + M).to(DEV)
+    q4, gs = q8.q8_quantize_weight_q4gs(W.to(DEV), G)
+    ref = q8.q8_linear_dq8ca_q4gsw(x, q4, gs, G).cpu()
+    for _ in range(5):
+        y = q8.q8_linear_dq8ca_q4gsw(x, q4, gs, G).cpu()
+        assert torch.equal(y.view(torch.int32), ref.view(torch.int32))
+
+
 # ----------------------------------------------------------------------- 8da4w (a7)
 
 
