@@ -412,6 +412,10 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
 // subtraction of 136 leaves the code.  The converters fence the async proxy and arrive on
 // the stage's "A ready" barrier; the MMA issuer waits only on that barrier (the converters
 // waited for the stage's TMA bytes, activations included).  No global bf16 weight copy.
+// With few tiles (64 activation rows give N / 128 of them) K is split into S parts per
+// tile, S chosen on the host to need the fewest rounds of (tile, part) units over the SMs;
+// the parts write their partial sums to the workspace and k_q4_split_reduce, launched
+// next, adds them in part order (the same sum on every run) and applies s[m].
 constexpr int QF_CONV_WARPS = 4;
 constexpr int QF_THREADS = (2 + QF_CONV_WARPS + QT_EPI_WARPS) * 32;
 
@@ -458,7 +462,10 @@ template <int BN, int KB>
 __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap bmap,
     const float* __restrict__ gs, const float* __restrict__ s, float* __restrict__ y, int G,
-    int M, int N, int K, int* status) {
+    int M, int N, int K, int S, float* __restrict__ part, int* status) {
+    // Work units: (tile, K-part); S parts per tile (K-split for grids with few tiles).  The
+    // part boundaries fall on stage and group boundaries.  With S > 1 each unit leaves its
+    // partial sums in `part` and k_q4_split_reduce, launched next, adds them in part order.
     using C = QfCfg<BN, KB>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -479,6 +486,16 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
     const int num_m = (M + BN - 1) / BN;
     const int tiles = num_n * num_m;
     const int nk = K / C::BK;                                  // K % 128 == 0
+    const int gstep = G > C::BK ? G / C::BK : 1;               // stages per split step
+    const int nsplit = nk / gstep;
+    const int units = tiles * S;
+    // stages [kb0, kb1) of unit u
+    auto unit_range = [&](int u, int& tile, int& kb0, int& kb1) {
+        tile = u / S;
+        const int pp = u - tile * S;
+        kb0 = (pp * nsplit / S) * gstep;
+        kb1 = ((pp + 1) * nsplit / S) * gstep;
+    };
     const int steps_per_group = G / QT_UK;
     const int ngroups = K / G;
 
@@ -520,9 +537,11 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
             int st = 0, it = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                int t, kb0, kb1;
+                unit_range(u, t, kb0, kb1);
                 const int n0 = (t / num_m) * QT_BM, m0 = (t % num_m) * BN;
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&empty[st], ph ^ 1u, status, abort_flag)) {
                         ok = false;
                         break;
@@ -549,9 +568,11 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
             int st = 0, buf = 0;
             uint32_t ph = 0, bph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                int t, kb0, kb1;
+                unit_range(u, t, kb0, kb1);
                 int in_group = 0;                  // MMA step within the current group
-                for (int kb = 0; kb < nk && ok; ++kb) {
+                for (int kb = kb0; kb < kb1 && ok; ++kb) {
                     if (!mbar_wait(&aready[st], ph, status, abort_flag)) {
                         ok = false;
                         break;
@@ -594,8 +615,10 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
         int st = 0;
         uint32_t ph = 0;
         bool live = true;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-            for (int kb = 0; kb < nk; ++kb) {
+        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            int t, kb0, kb1;
+            unit_range(u, t, kb0, kb1);
+            for (int kb = kb0; kb < kb1; ++kb) {
                 const bool okw = mbar_wait(&full[st], ph, status, abort_flag);
                 live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
                 uint8_t* base = smem + (size_t)st * C::STAGE;
@@ -639,7 +662,10 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
         constexpr int HC = C::HALF;
         int buf = 0;
         uint32_t bph = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            int t, kb0, kb1;
+            unit_range(u, t, kb0, kb1);
+            const int g0 = kb0 * C::BK / G, g1 = kb1 * C::BK / G;
             const int n0 = (t / num_m) * QT_BM, m0 = (t % num_m) * BN;
             const int n = n0 + q * 32 + lane;
             for (int j = et; j < BN; j += 32 * QT_EPI_WARPS)
@@ -656,7 +682,8 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
             auto load_chunk = [&](float (&dst)[GC], int g0) {
 #pragma unroll
                 for (int i = 0; i < GC; i += 4) {
-                    if ((ngroups & 3) == 0 && g0 + i + 3 < ngroups) {
+                    // 16-byte loads only where aligned (a K-part may start at any group)
+                    if ((ngroups & 3) == 0 && ((g0 + i) & 3) == 0 && g0 + i + 3 < ngroups) {
                         const float4 v = __ldg(reinterpret_cast<const float4*>(gsr + g0 + i));
                         dst[i] = v.x; dst[i + 1] = v.y; dst[i + 2] = v.z; dst[i + 3] = v.w;
                     } else {
@@ -666,16 +693,17 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
                     }
                 }
             };
-            load_chunk(gnxt, 0);
-            for (int gi = 0; gi < ngroups; ++gi) {
-                if (gi % GC == 0) {
+            load_chunk(gnxt, g0);
+            for (int gi = g0; gi < g1; ++gi) {
+                const int li = gi - g0;
+                if (li % GC == 0) {
 #pragma unroll
                     for (int i = 0; i < GC; ++i) gcur[i] = gnxt[i];
-                    if (gi + GC < ngroups) load_chunk(gnxt, gi + GC);
+                    if (gi + GC < g1) load_chunk(gnxt, gi + GC);
                 }
                 float gcur_v = gcur[0];
 #pragma unroll
-                for (int i = 1; i < GC; ++i) gcur_v = (gi % GC == i) ? gcur[i] : gcur_v;
+                for (int i = 1; i < GC; ++i) gcur_v = (li % GC == i) ? gcur[i] : gcur_v;
                 const bool okw = mbar_wait(&tfull[buf], bph, status, abort_flag);
                 live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -700,7 +728,14 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
                 if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
             }
             named_bar_sync(2, 32 * QT_EPI_WARPS);
-            if (live && n < N) {
+            const int row = q * 32 + lane;                   // weight row within the tile
+            if (S > 1) {
+                // this part's sums, [tile][part][column][row] (coalesced by row)
+                float* mine = part + ((int64_t)t * S + (u - t * S)) * BN * QT_BM;
+#pragma unroll
+                for (int j = 0; j < HC; ++j) mine[(half * HC + j) * QT_BM + row] = acc[j];
+            }
+            if (S == 1 && live && n < N) {
 #pragma unroll
                 for (int j = 0; j < HC; ++j) {
                     const int m = m0 + half * HC + j;
@@ -754,10 +789,52 @@ static cudaError_t launch_qt(const uint16_t* wb, const uint16_t* xz, const float
     return cudaLaunchKernelEx(&cfg, k_q4_gemm_tc<BN, KB>, ma, mb, gs, s, y, G, M, N, K, status);
 }
 
+// y[m, n] = s[m] * sum over the S parts, in part order, of the fused GEMM's partial sums
+// (layout [tile][part][column][row] with 128-row weight tiles and 64-row activation tiles).
+__global__ __launch_bounds__(256) void k_q4_split_reduce(const float* __restrict__ part,
+                                                          const float* __restrict__ s,
+                                                          float* __restrict__ y, int M, int N,
+                                                          int S) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int num_m = (M + 63) / 64;
+    const int64_t total = (int64_t)M * N;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int m = (int)(i / N), n = (int)(i - (int64_t)m * N);
+        const int t = (n / QT_BM) * num_m + m / 64;
+        const float* p = part + ((int64_t)t * S * 64 + (m % 64)) * QT_BM + (n % QT_BM);
+        float v = 0.0f;
+        for (int pp = 0; pp < S; ++pp) v += __ldcg(p + (int64_t)pp * 64 * QT_BM);
+        y[i] = __ldg(s + m) * v;
+    }
+}
+
+// K-parts per tile of the fused GEMM: the count (at most 8) that needs the fewest rounds of
+// (tile, part) units over the SMs, measured in whole tiles; ties go to fewer parts.
+static int qf_split(int64_t M, int64_t N, int K, int G, int num_sms) {
+    const int64_t tiles = ((N + QT_BM - 1) / QT_BM) * ((M + 63) / 64);
+    const int bk = QT_BOXK * (G == 32 ? 1 : 2);
+    const int nsplit = (K / bk) / (G > bk ? G / bk : 1);
+    int best = 1;
+    double best_cost = (double)((tiles + num_sms - 1) / num_sms);
+    for (int sp = 2; sp <= 8 && sp <= nsplit; ++sp) {
+        const double cost = (double)((tiles * sp + num_sms - 1) / num_sms) / sp + 0.02 * sp;
+        if (cost < best_cost - 1e-9) { best = sp; best_cost = cost; }
+    }
+    return best;
+}
+
+size_t q4_fused_workspace_bytes(int64_t M, int64_t N, int K, int G, int num_sms) {
+    const int sp = qf_split(M, N, K, G, num_sms);
+    if (sp == 1) return 0;
+    const int64_t tiles = ((N + QT_BM - 1) / QT_BM) * ((M + 63) / 64);
+    return (size_t)(tiles * sp * 64 * QT_BM) * sizeof(float);
+}
+
 template <int BN, int KB>
 static cudaError_t launch_qf(const uint8_t* q4, const uint16_t* xz, const float* gs,
-                             const float* s, float* y, int G, int M, int N, int K,
-                             cudaStream_t st, int num_sms, int* status) {
+                             const float* s, float* y, int G, int M, int N, int K, int sp,
+                             float* part, cudaStream_t st, int num_sms, int* status) {
     using C = QfCfg<BN, KB>;
     CUtensorMap mq, mb;
     if (!make_tmap_u8_2d(&mq, q4, N, K / 2, C::Q_ROW, QT_BM, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -765,8 +842,8 @@ static cudaError_t launch_qf(const uint8_t* q4, const uint16_t* xz, const float*
     if (!make_tmap_bf16_2d(&mb, xz, M, K, QT_BOXK, BN)) return cudaErrorInvalidValue;
     cudaError_t e = ensure_dyn_smem<k_q4_gemm_fused<BN, KB>>((int)(C::SMEM + 1024));
     if (e != cudaSuccess) return e;
-    const int tiles = ((N + QT_BM - 1) / QT_BM) * ((M + BN - 1) / BN);
-    const int grid = tiles < num_sms ? tiles : num_sms;
+    const int units = ((N + QT_BM - 1) / QT_BM) * ((M + BN - 1) / BN) * sp;
+    const int grid = units < num_sms ? units : num_sms;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(QF_THREADS);
@@ -777,19 +854,39 @@ static cudaError_t launch_qf(const uint8_t* q4, const uint16_t* xz, const float*
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_q4_gemm_fused<BN, KB>, mq, mb, gs, s, y, G, M, N, K,
-                              status);
+    return cudaLaunchKernelEx(&cfg, k_q4_gemm_fused<BN, KB>, mq, mb, gs, s, y, G, M, N, K, sp,
+                              part, status);
 }
 
 // Up to 64 activation rows the weight is expanded inside the GEMM (no bf16 copy in HBM).
 bool q4_tc_fused(int64_t M) { return M <= 64; }
 
+// ws: q4_fused_workspace_bytes() bytes (the K-parts' partial sums).
 cudaError_t launch_q4_gemm_fused(const uint8_t* q4, const uint16_t* xz, const float* gs,
                                  const float* s, float* y, int G, int64_t M, int64_t N, int K,
-                                 cudaStream_t st, int num_sms, int* status) {
-    return G == 32
-               ? launch_qf<64, 1>(q4, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status)
-               : launch_qf<64, 2>(q4, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
+                                 void* ws, cudaStream_t st, int num_sms, int* status) {
+    const int sp = qf_split(M, N, K, G, num_sms);
+    float* part = (float*)ws;
+    cudaError_t e =
+        G == 32 ? launch_qf<64, 1>(q4, xz, gs, s, y, G, (int)M, (int)N, K, sp, part, st, num_sms,
+                                   status)
+                : launch_qf<64, 2>(q4, xz, gs, s, y, G, (int)M, (int)N, K, sp, part, st, num_sms,
+                                   status);
+    if (e != cudaSuccess || sp == 1) return e;
+    cudaLaunchConfig_t cfg = {};
+    const int64_t total = M * N;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_q4_split_reduce, (const float*)part, s, y, (int)M, (int)N,
+                              sp);
 }
 
 cudaError_t launch_q4_expand_bf16(const uint8_t* q4, int64_t N, int K, uint16_t* wb,

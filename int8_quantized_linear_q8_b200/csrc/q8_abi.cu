@@ -129,7 +129,8 @@ struct Q4Plan {
     bool tc = false;
     size_t xq = 0, s = 0, z = 0, wb = 0, bytes = 0;
 };
-static Q4Plan plan_q4(int64_t M, int64_t N, int64_t K) {
+// sms: the device's SM count (sizes the K-split workspace of the fused GEMM, 17..64 rows)
+static Q4Plan plan_q4(int64_t M, int64_t N, int64_t K, int G, int sms) {
     Q4Plan p;
     if (M <= 0) return p;
     p.tc = M > kQ4GemvMaxM;
@@ -139,9 +140,14 @@ static Q4Plan plan_q4(int64_t M, int64_t N, int64_t K) {
     p.s = align_up(codes, 256);
     p.z = p.s + align_up((size_t)M * 4, 256);
     p.wb = p.z + align_up((size_t)M * 4, 256);
-    // the bf16 copy of the weight only where the GEMM does not expand the codes itself
-    const bool wb = p.tc && !q4_tc_fused(M);
-    p.bytes = p.wb + (wb ? align_up((size_t)N * (size_t)K * 2, 256) : 0);
+    // the bf16 copy of the weight where the GEMM does not expand the codes itself; else
+    // (at wb) the fused GEMM's K-split partial sums and tile counters, if it splits
+    size_t rest = 0;
+    if (p.tc && !q4_tc_fused(M))
+        rest = align_up((size_t)N * (size_t)K * 2, 256);
+    else if (p.tc)
+        rest = align_up(q4_fused_workspace_bytes(M, N, (int)K, G, sms), 256);
+    p.bytes = p.wb + rest;
     return p;
 }
 static inline bool valid_group(int G) { return G == 32 || G == 64 || G == 128 || G == 256; }
@@ -316,9 +322,12 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) 
             return w8a16_tc_workspace_bytes(M, K, sms);
         }
         case Q8_OP_LINEAR_W8A8: return plan_w8a8(M, K, extra != 0).bytes;
-        case Q8_OP_LINEAR_DQ8CA_Q4GSW:
+        case Q8_OP_LINEAR_DQ8CA_Q4GSW: {
             if (!valid_group(extra) || K % 128 != 0 || K % extra != 0) return 0;
-            return plan_q4(M, N, K).bytes;
+            int sms = 0;
+            if (M > kQ4GemvMaxM && q4_tc_fused(M) && current_device(sms) != Q8_OK) return 0;
+            return plan_q4(M, N, K, extra, sms).bytes;
+        }
     }
     return 0;
 }
@@ -365,12 +374,12 @@ q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* g
     if (M == 0) return Q8_OK;
     if (!x || !q4 || !gs || !y) return Q8_ERR_NULL;
     if (!aligned16(x) || !aligned16(q4) || !aligned16(gs) || !aligned16(y)) return Q8_ERR_ALIGN;
-    const Q4Plan plan = plan_q4(M, N, K);
-    if (!workspace || ws_bytes < plan.bytes) return Q8_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return Q8_ERR_ALIGN;
     int sms = 0;
     int* status = nullptr;
     Q8_TRY(current_device(sms, &status));
+    const Q4Plan plan = plan_q4(M, N, K, G, sms);
+    if (!workspace || ws_bytes < plan.bytes) return Q8_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return Q8_ERR_ALIGN;
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* ws = (uint8_t*)workspace;
     float* s = (float*)(ws + plan.s);
@@ -378,8 +387,10 @@ q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* g
     if (plan.tc) {
         uint16_t* xz = (uint16_t*)(ws + plan.xq);
         if (q4_tc_fused(M)) {
+            void* fws = ws + plan.wb;
             Q8_TRY(launched(launch_choose_qparams_shifted((const uint16_t*)x, M, (int)K, s, z, xz, st)));
-            return launched(launch_q4_gemm_fused(q4, xz, gs, s, y, G, M, N, (int)K, st, sms, status));
+            return launched(launch_q4_gemm_fused(q4, xz, gs, s, y, G, M, N, (int)K, fws, st, sms,
+                                                 status));
         }
         uint16_t* wb = (uint16_t*)(ws + plan.wb);
         Q8_TRY(launched(launch_q4_expand_bf16(q4, N, (int)K, wb, st, sms)));

@@ -92,9 +92,11 @@ cudaError_t launch_q4_expand_bf16(const uint8_t* q4, int64_t N, int K, uint16_t*
                                   cudaStream_t st, int num_sms);
 // M <= 64: the GEMM expands the packed int4 weight itself (q4 [N, K/2], no bf16 copy)
 bool q4_tc_fused(int64_t M);
+// Workspace of the fused GEMM's K-split (the parts' partial sums; 0 without a split).
+size_t q4_fused_workspace_bytes(int64_t M, int64_t N, int K, int G, int num_sms);
 cudaError_t launch_q4_gemm_fused(const uint8_t* q4, const uint16_t* xz, const float* gs,
                                  const float* s, float* y, int G, int64_t M, int64_t N, int K,
-                                 cudaStream_t st, int num_sms, int* status);
+                                 void* ws, cudaStream_t st, int num_sms, int* status);
 cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const float* gs,
                               const float* s, float* y, int G, int64_t M, int64_t N, int K,
                               cudaStream_t st, int num_sms, int* status);

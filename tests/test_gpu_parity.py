@@ -373,9 +373,10 @@ def test_w8a16_repeat_bit_identical(M, N, K):
         assert torch.equal(y.view(torch.int32), ref.view(torch.int32))
 
 
-@pytest.mark.parametrize("M,G", [(1, 128), (8, 32), (16, 64)])
+@pytest.mark.parametrize("M,G", [(1, 128), (8, 32), (16, 64), (40, 64)])
 def test_dq8ca_decode_repeat_bit_identical(M, G):
-    """The 8da4w decode stream is deterministic too (fixed-order partial sums)."""
+    """The 8da4w decode stream is deterministic too (fixed-order partial sums), and so is
+    the K-split of the small-M GEMM (the last part adds all parts in part order)."""
     N, K = 11008, 4096
     W = wl.weight(N, K, seed=890 + M)
     x = wl.normal_bf16((M, K), 1.0, seed=891 + M).to(DEV)
