@@ -75,9 +75,12 @@ constexpr int QT_NBUF_MAX = 4;        // group accumulator buffers in tensor mem
 // that beats 4 stages of one box (measured, 256-row tiles, G = 128: 576 -> 472 us); with
 // G = 32 a group hand-off comes every 2 MMAs anyway and the deeper 6-stage ring of single
 // boxes is faster.
-template <int BN, int KB>
+// GPB groups per accumulator buffer: side by side (each its own accumulator), handed to
+// the epilogue together -- one hand-off per GPB groups (G = 32 with 128-row tiles).
+template <int BN, int KB, int GPB = 1>
 struct QtCfg {
     static constexpr int KBOX = KB;
+    static constexpr int BUFW = BN * GPB;                  // tensor-memory columns per buffer
     static constexpr int BK = QT_BOXK * KB;                // K elements per stage
     static constexpr int STAGE_SZ = (QT_BM + BN) * QT_BOXK * 2 * KB;
     // QT_RING / KB stages, as many as fit next to the control region (192 KB of ring)
@@ -88,9 +91,9 @@ struct QtCfg {
     static constexpr int A_BYTES = A_BOX * KB;
     static constexpr int B_BYTES = B_BOX * KB;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int NBUF = 512 / BN < QT_NBUF_MAX ? 512 / BN : QT_NBUF_MAX;
-    static constexpr int TMEM_COLS = NBUF * BN < 32 ? 32 : NBUF * BN;
-    static_assert(NBUF >= 2 && NBUF * BN <= 512, "tensor memory");
+    static constexpr int NBUF = 512 / BUFW < QT_NBUF_MAX ? 512 / BUFW : QT_NBUF_MAX;
+    static constexpr int TMEM_COLS = NBUF * BUFW < 32 ? 32 : NBUF * BUFW;
+    static_assert(NBUF >= 2 && NBUF * BUFW <= 512, "tensor memory");
     static constexpr int HALF = BN / 2;                    // columns per epilogue warp
     static constexpr size_t SMEM = (size_t)STAGES * STAGE + 4096;
 };
@@ -163,12 +166,12 @@ __device__ __forceinline__ void qt_ld32(uint32_t taddr, float (&r)[32]) {
     for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
 
-template <int BN, int KB>
+template <int BN, int KB, int GPB>
 __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
     const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
     const float* __restrict__ gs, const float* __restrict__ s, float* __restrict__ y, int G,
     int M, int N, int K, int* status) {
-    using C = QtCfg<BN, KB>;
+    using C = QtCfg<BN, KB, GPB>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* ctrl = smem + (size_t)C::STAGES * C::STAGE;
@@ -265,6 +268,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                 // every MMA of the CTA, so its loop must stay short -- a modulo per step
                 // made the issue loop, not the tensor core, the limit)
                 int in_group = 0;
+                int gin = 0;                        // group within the current buffer
                 for (int kb = 0; kb < nk && ok; ++kb) {
                     if (!mbar_wait(&full[st], ph, status, abort_flag)) {
                         ok = false;
@@ -279,19 +283,23 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                         const uint64_t a = qt_desc_sw128(base + (k / KPB) * C::A_BOX) + 2 * (k % KPB);
                         const uint64_t b =
                             qt_desc_sw128(base + C::A_BYTES + (k / KPB) * C::B_BOX) + 2 * (k % KPB);
-                        if (in_group == 0) {
-                            // a new group: wait until the epilogue has drained this buffer
+                        if (in_group == 0 && gin == 0) {
+                            // a new buffer: wait until the epilogue has drained it
                             if (!mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag)) {
                                 ok = false;
                                 break;
                             }
                             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                         }
-                        qt_mma_f16(tmem_base + (uint32_t)(buf * BN), a, b, idesc, in_group != 0);
+                        qt_mma_f16(tmem_base + (uint32_t)(buf * C::BUFW + gin * BN), a, b, idesc,
+                                   in_group != 0);
                         if (++in_group == steps_per_group) {
                             in_group = 0;
-                            qt_commit(&tfull[buf]);             // group partial ready
-                            if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
+                            if (++gin == GPB) {
+                                gin = 0;
+                                qt_commit(&tfull[buf]);         // GPB group partials ready
+                                if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
+                            }
                         }
                     }
                     qt_commit(&empty[st]);                      // stage free after these MMAs
@@ -340,7 +348,13 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                 }
             };
             load_chunk(gnxt, 0);
-            for (int gi = 0; gi < ngroups; ++gi) {
+            for (int gb = 0; gb < ngroups; gb += GPB) {      // one hand-off per GPB groups
+                const bool okw = mbar_wait(&tfull[buf], bph, status, abort_flag);
+                live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+              for (int sub = 0; sub < GPB; ++sub) {
+                const int gi = gb + sub;
                 if (gi % GC == 0) {
 #pragma unroll
                     for (int i = 0; i < GC; ++i) gcur[i] = gnxt[i];
@@ -350,12 +364,9 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
 #pragma unroll
                 for (int i = 1; i < GC; ++i) gsel = (gi % GC == i) ? gcur[i] : gsel;
                 const float gcur_v = gsel;
-                const bool okw = mbar_wait(&tfull[buf], bph, status, abort_flag);
-                live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
-                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 if (live) {
                     const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
-                                           (uint32_t)(buf * BN + half * HC);
+                                           (uint32_t)(buf * C::BUFW + sub * BN + half * HC);
                     // 32-column chunks, up to two per tensor-memory wait (with 128 columns
                     // per warp one at a time: 128 fp32 sums already take the registers)
                     constexpr int NCH = HC / 32;
@@ -374,6 +385,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                                       __uint_as_float(u[c][j]), __uint_as_float(u[c][j + 1]));
                     }
                 }
+              }
                 asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -764,15 +776,15 @@ static bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, int64_t rows, 
                            CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <int BN, int KB>
+template <int BN, int KB, int GPB = 1>
 static cudaError_t launch_qt(const uint16_t* wb, const uint16_t* xz, const float* gs,
                              const float* s, float* y, int G, int M, int N, int K,
                              cudaStream_t st, int num_sms, int* status) {
-    using C = QtCfg<BN, KB>;
+    using C = QtCfg<BN, KB, GPB>;
     CUtensorMap ma, mb;
     if (!make_tmap_bf16_2d(&ma, wb, N, K, QT_BOXK, QT_BM)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16_2d(&mb, xz, M, K, QT_BOXK, BN)) return cudaErrorInvalidValue;
-    cudaError_t e = ensure_dyn_smem<k_q4_gemm_tc<BN, KB>>((int)(C::SMEM + 1024));
+    cudaError_t e = ensure_dyn_smem<k_q4_gemm_tc<BN, KB, GPB>>((int)(C::SMEM + 1024));
     if (e != cudaSuccess) return e;
     const int tiles = ((N + QT_BM - 1) / QT_BM) * ((M + BN - 1) / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
@@ -786,7 +798,7 @@ static cudaError_t launch_qt(const uint16_t* wb, const uint16_t* xz, const float
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_q4_gemm_tc<BN, KB>, ma, mb, gs, s, y, G, M, N, K, status);
+    return cudaLaunchKernelEx(&cfg, k_q4_gemm_tc<BN, KB, GPB>, ma, mb, gs, s, y, G, M, N, K, status);
 }
 
 // y[m, n] = s[m] * sum over the S parts, in part order, of the fused GEMM's partial sums
@@ -912,8 +924,10 @@ cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const floa
     // a time, registers short) then falls behind the MMAs (G = 32: 1062 -> 1395 us).
     if (M >= Q4TC_WIDE_M && G >= Q4TC_WIDE_G)
         return launch_qt<256, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
-    return G == 32 ? launch_qt<128, 1>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status)
-                   : launch_qt<128, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
+    // G = 32: two groups per accumulator buffer (K / 32 groups, a multiple of 4)
+    return G == 32
+               ? launch_qt<128, 1, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status)
+               : launch_qt<128, 2>(wb, xz, gs, s, y, G, (int)M, (int)N, K, st, num_sms, status);
 }
 
 }  // namespace q8
