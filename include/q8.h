@@ -176,8 +176,9 @@ q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w,
  * the tighter rounding.
  *   workspace: at least q8_workspace_bytes(Q8_OP_LINEAR_W8A16_PLANES, M, N, K, 0) bytes,
  *   16-byte aligned, ZERO-FILLED before its first use and then left to this function (it
- *   keeps per-call flags there); one workspace must not serve two calls that may run at
- *   the same time.  The kernel keeps one CTA per SM resident and its CTAs wait on each
+ *   keeps a call counter and per-call flags there, so calls captured in a CUDA graph may be
+ *   replayed); one workspace must not serve two calls that may run at the same time, nor
+ *   any other operation.  After a call that returned an error status, zero-fill it again.  The kernel keeps one CTA per SM resident and its CTAs wait on each
  *   other (bounded): it must not share the GPU with a limit on SMs.
  *   Q8_ERR_WORKSPACE if the workspace is NULL or too small.  M > 16 (workspace size 0)
  *   runs q8_linear_w8a16. */

@@ -32,7 +32,9 @@
 // its first unit (for that CTA it is the last tile of its range); the others write their
 // int32 partial accumulators to a workspace slot and raise a flag, which the owner waits
 // for before its epilogue.  Flags carry a per-call 64-bit epoch, so they never need
-// resetting (the workspace must be zero-filled once before its first use).
+// resetting (the workspace must be zero-filled once before its first use).  The epoch is
+// kept on the device, in the workspace (one more than the calls completed on it), so a
+// CUDA graph that replays a captured call gets a new epoch on every replay.
 //
 // CTA structure (6 warps, one CTA per SM):
 //   warp 0   : TMA producer.  Weight tiles (128 rows x 128 bytes) start streaming at once;
@@ -92,8 +94,8 @@ struct WcRes {
     float v;      // its value
 };
 
-// Grid-wide state of one call, at the start of the workspace.  Every field is zero
-// between calls: the flags are compared with the call's epoch, and the counters and
+// Grid-wide state of one call, at the start of the workspace.  Every field but `calls` is
+// zero between calls: the flags are compared with the call's epoch, and the counters and
 // statistics are returned to zero by the CTA that consumes them.
 struct WcHdr {
     unsigned long long stats_flag;     // = epoch once every row's planes count is known
@@ -102,8 +104,11 @@ struct WcHdr {
     int fmax1[WC_MAX_M];               // 1 + largest exponent of the row (0: none yet)
     int fmin1[WC_MAX_M];               // 1000 - smallest exponent (0: none yet)
     int nres[WC_MAX_M];                // residual elements of the row
-    int pad[2];
+    int done;                          // CTAs of the current call that have finished
+    int pad;
+    unsigned long long calls;          // calls completed on this workspace; epoch = calls + 1
 };
+static_assert(sizeof(WcHdr) <= 256, "the CTA flags start at byte 256");
 
 // Workspace layout (byte offsets), for M activation rows, K columns and G CTAs.  The header
 // and the flags come first, at offsets that depend on nothing but G (the device's SM
@@ -139,7 +144,6 @@ struct WcArgs {
     WcHdr* hdr;
     unsigned long long* cta_flag;
     int32_t* slots;
-    unsigned long long epoch;
     int* status;
 };
 
@@ -281,7 +285,7 @@ __device__ __forceinline__ void wc_split(uint32_t bits, int& S, int& fp, bool& f
 //      or non-finite); the last CTA to arrive publishes the residual counts, zeroes the
 //      counters and raises planes_flag, which the producers and the epilogues wait for.
 // sm: shared scratch of 4 * WC_MAX_M + 1 ints.  Returns false if a wait expired.
-__device__ bool wc_build_planes(const WcArgs& a, int jcap, int et, int* sm,
+__device__ bool wc_build_planes(const WcArgs& a, unsigned long long epoch, int jcap, int et, int* sm,
                                 volatile int* abort_flag) {
     const int G = (int)gridDim.x, b = (int)blockIdx.x, K = a.K, M = a.M;
     const int n8 = K >> 3;
@@ -350,9 +354,9 @@ __device__ bool wc_build_planes(const WcArgs& a, int jcap, int et, int* sm,
             }
             a.hdr->arrive1 = 0;
             __threadfence();
-            st_release_u64(&a.hdr->stats_flag, a.epoch);
+            st_release_u64(&a.hdr->stats_flag, epoch);
         } else {
-            ok = wait_flag(&a.hdr->stats_flag, a.epoch, a.status, abort_flag);
+            ok = wait_flag(&a.hdr->stats_flag, epoch, a.status, abort_flag);
         }
         *last = ok ? 1 : 0;
     }
@@ -413,7 +417,7 @@ __device__ bool wc_build_planes(const WcArgs& a, int jcap, int et, int* sm,
             for (int m = 0; m < M; ++m) a.meta[m].nres = atomicExch(&a.hdr->nres[m], 0);
             a.hdr->arrive2 = 0;
             __threadfence();
-            st_release_u64(&a.hdr->planes_flag, a.epoch);
+            st_release_u64(&a.hdr->planes_flag, epoch);
         }
     }
     return ok;
@@ -479,6 +483,10 @@ __global__ __launch_bounds__(WC_THREADS, 1) void k_w8a16_tc(
     // access below waits for the previous kernel (its outputs may be our inputs).
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // This call's epoch.  The previous call on the workspace has completed (the wait
+    // above), and `calls` only advances once every CTA of this call has read it (the last
+    // CTA to finish advances it, below).
+    const unsigned long long epoch = ld_acquire_u64(&a.hdr->calls) + 1ull;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -495,7 +503,7 @@ __global__ __launch_bounds__(WC_THREADS, 1) void k_w8a16_tc(
                             (int)(u / KB) * WC_BM, &full[i]);
             }
             int jmax = 0;
-            bool ok = wait_flag(&a.hdr->planes_flag, a.epoch, a.status, abort_flag);
+            bool ok = wait_flag(&a.hdr->planes_flag, epoch, a.status, abort_flag);
             fence_proxy_async_global();
             if (ok)
                 for (int m = 0; m < a.M; ++m)
@@ -578,9 +586,9 @@ __global__ __launch_bounds__(WC_THREADS, 1) void k_w8a16_tc(
         const int et = threadIdx.x - 64;                     // 0..127
         const int qd = warp & 3;                             // TMEM lane quarter
         const int row = qd * 32 + lane;                      // tile row of this thread
-        bool built = wc_build_planes(a, shp.jcap, et, bsm, abort_flag);
+        bool built = wc_build_planes(a, epoch, shp.jcap, et, bsm, abort_flag);
         if (et == 0) {
-            const bool ok = built && wait_flag(&a.hdr->planes_flag, a.epoch, a.status, abort_flag);
+            const bool ok = built && wait_flag(&a.hdr->planes_flag, epoch, a.status, abort_flag);
             for (int m = 0; m < WC_MAX_M; ++m) {
                 const bool v = ok && m < a.M;
                 mJ[m] = v ? min(max(__ldcg(&a.meta[m].J), 0), shp.jcap) : 0;
@@ -623,11 +631,11 @@ __global__ __launch_bounds__(WC_THREADS, 1) void k_w8a16_tc(
                 }
                 __threadfence();
                 named_bar_sync(3, 128);
-                if (et == 0 && live) st_release_u64(&a.cta_flag[b], a.epoch);
+                if (et == 0 && live) st_release_u64(&a.cta_flag[b], epoch);
             } else {
                 if (et == 0)
                     for (int c = b + 1; c <= last_cta; ++c)
-                        if (!wait_flag(&a.cta_flag[c], a.epoch, a.status, abort_flag)) break;
+                        if (!wait_flag(&a.cta_flag[c], epoch, a.status, abort_flag)) break;
                 named_bar_sync(3, 128);
                 if (live && last_cta > b) {
                     // add the other CTAs' partials into this tile's accumulator, in groups of
@@ -716,11 +724,18 @@ __global__ __launch_bounds__(WC_THREADS, 1) void k_w8a16_tc(
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                      "r"(WC_TMEM_COLS)
                      : "memory");
+    if (threadIdx.x == 0) {
+        // every thread of this CTA read the epoch before the barrier above
+        __threadfence();
+        if (atomicAdd(&a.hdr->done, 1) == G - 1) {
+            atomicExch(&a.hdr->done, 0);
+            __threadfence();
+            atomicAdd(&a.hdr->calls, 1ull);
+        }
+    }
 }
 
 // ----------------------------------------------------------------------- host side
-static std::atomic<unsigned long long> g_wc_epoch{0};
-
 size_t w8a16_tc_workspace_bytes(int64_t M, int64_t K, int num_sms) {
     if (M < 1 || M > WC_MAX_M || K < 16 || K % 16) return 0;
     return wc_plan((int)M, (int)K, num_sms).bytes;
@@ -758,7 +773,6 @@ cudaError_t launch_w8a16_tc(const uint16_t* x, const int8_t* q, const float* s_w
     a.hdr = reinterpret_cast<WcHdr*>(w + p.hdr);
     a.cta_flag = reinterpret_cast<unsigned long long*>(w + p.cta_flag);
     a.slots = reinterpret_cast<int32_t*>(w + p.slots);
-    a.epoch = ++g_wc_epoch;
     a.status = status;
     const size_t smem = wc_smem_bytes((int)M);
     cudaError_t e = ensure_dyn_smem<k_w8a16_tc>((int)smem);

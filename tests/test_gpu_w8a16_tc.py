@@ -179,3 +179,34 @@ def test_w8a16_tc_workspace_checks():
     rq, rs, _ = oracle.quantize_weight(W.numpy())
     y64, absum = oracle.linear_w8a16(wl.bf16_bits(x17), rq, rs)
     check_f32(y.cpu().numpy(), y64, absum, "M=17 fallback")
+
+
+def test_w8a16_tc_graph_replay():
+    """One call captured in a CUDA graph and replayed with new activations each time: the
+    cross-CTA flags must belong to each replay, not to the capture, so every replay matches
+    the oracle on its own inputs (tiles here span several CTAs: 64 tiles x 16 K-blocks)."""
+    M, N, K = 4, 8192, 2048
+    W = wl.weight(N, K, seed=70)
+    q, s, _ = q8.q8_quantize_weight(W.to(DEV), want_wsum=False)
+    rq, rs, _ = oracle.quantize_weight(W.numpy())
+    ws = q8.q8_w8a16_planes_workspace(M, N, K, device=DEV)
+    xs = torch.empty(M, K, dtype=torch.bfloat16, device=DEV)
+    y = torch.empty(M, N, dtype=torch.float32, device=DEV)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        xs.copy_(wl.normal_bf16((M, K), 1.0, seed=71).to(DEV))
+        q8.q8_linear_w8a16_planes(xs, q, s, ws, y=y, out_dtype=torch.float32)   # warm
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        q8.q8_linear_w8a16_planes(xs, q, s, ws, y=y, out_dtype=torch.float32)
+    for r in range(4):
+        x = wl.normal_bf16((M, K), 1.0 + r, seed=72 + r)
+        xs.copy_(x.to(DEV))
+        y.fill_(float("nan"))
+        gr.replay()
+        torch.cuda.synchronize()
+        y64, absum = oracle.linear_w8a16(wl.bf16_bits(x), rq, rs)
+        _tight(y.cpu().numpy(), y64, absum, f"graph replay {r}")
