@@ -9,8 +9,9 @@ bf16 activations + bf16 outputs) per second.  Two copies of every weight rotate 
 steps (390 MB, over 3x the 126 MB L2), and within a step cases run M-major, so a weight
 is never re-read from L2.
 
-Extra sub-benchmarks (same JSON line, key "paths"): W8A8 static int8 linear (K = 960) and
-the quantizers.
+Extra sub-benchmarks (same JSON line, key "paths"): the sweep through the digit-plane
+form and with a bias, W8A8 static int8 linear (K = 960) and prefill (M = 4096, also with a
+bias), 8da4w, the quantizers (both weight grids) and a Llama-shaped stack.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -445,7 +446,8 @@ def int8_peak_tops(peaks) -> float:
 
 def bench_w8a8_prefill(dev, peaks, reps=5):
     """W8A8 (static per-tensor activations) at M = 4096 on the Llama-shaped linears
-    (tcgen05 int8 GEMM incl. its activation-code pre-kernel), one and two passes."""
+    (tcgen05 int8 GEMM incl. its activation-code pre-kernel), one and two passes, and the
+    4096 x 11008 case once more with a bias."""
     import int8_quantized_linear_q8_b200 as q8
 
     out = []
@@ -473,6 +475,15 @@ def bench_w8a8_prefill(dev, peaks, reps=5):
             out.append({"M": M, "K": K, "N": N, "two_pass": two, "us": round(us, 1),
                         "TOPS": round(tops, 1),
                         "frac_int8_peak": round(tops / int8_peak_tops(peaks), 4)})
+            if N == 11008:
+                b = torch.randn(N, generator=g, device=dev)
+                fn = lambda: q8.q8_linear_w8a8(x, first, q, ws, s, second=sec, y=y,
+                                               workspace=work, bias=b)
+                us = _graph_time(fn, reps)
+                tops = ops / us / 1e6
+                out.append({"M": M, "K": K, "N": N, "two_pass": two, "bias": True,
+                            "us": round(us, 1), "TOPS": round(tops, 1),
+                            "frac_int8_peak": round(tops / int8_peak_tops(peaks), 4)})
         del x, q, s, ws, y, work
     return out
 
@@ -493,6 +504,26 @@ def planes_case_times(sweep: W8A16Sweep):
 
     out = per_case_times(sweep, launch=launch)
     total_b = sum(w8a16_bytes(c["M"], c["N"], c["K"]) for c in out)
+    total_us = sum(c["us"] for c in out)
+    return {"cases": out, "GBps_sum_of_cases": round(total_b / total_us / 1e3, 1)}
+
+
+def bias_case_times(sweep: W8A16Sweep):
+    """The sweep's cases through q8_linear_w8a16 with an fp32 bias [N] (4 N more bytes),
+    timed like the headline's per-case times."""
+    q8 = sweep.q8
+    g = torch.Generator(device=sweep.shapes[0][1][0].device)
+    g.manual_seed(91)
+    bias = [torch.randn(sh.N, generator=g, device=g.device) for sh, _, _ in sweep.shapes]
+
+    def launch(i, M, copy):
+        sh, copies, s = sweep.shapes[i]
+        q8.q8_linear_w8a16(sweep.xs[(i, M)], copies[copy], s, y=sweep.ys[(i, M)], bias=bias[i])
+
+    out = per_case_times(sweep, launch=launch)
+    for c in out:
+        c["GBps"] = round((w8a16_bytes(c["M"], c["N"], c["K"]) + 4 * c["N"]) / c["us"] / 1e3, 1)
+    total_b = sum(w8a16_bytes(c["M"], c["N"], c["K"]) + 4 * c["N"] for c in out)
     total_us = sum(c["us"] for c in out)
     return {"cases": out, "GBps_sum_of_cases": round(total_b / total_us / 1e3, 1)}
 
@@ -542,6 +573,10 @@ def bench_quantizers(dev, peaks, reps=5):
     us = _graph_time(lambda: q8.q8_quantize_weight(W, q=q, s_w=sw, wsum=ws), reps)
     b = 32000 * 4096 * 5 + 32000 * 8
     out.append({"op": "quantize_weight", "shape": [32000, 4096], "us": round(us, 1),
+                "GBps": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / peaks["hbm_gbs"], 4)})
+    us = _graph_time(lambda: q8.q8_quantize_weight(W, q=q, s_w=sw, wsum=ws, grid="full128"),
+                     reps)
+    out.append({"op": "quantize_weight_full128", "shape": [32000, 4096], "us": round(us, 1),
                 "GBps": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / peaks["hbm_gbs"], 4)})
     del W, q
     xb = torch.randn(4096, 4096, generator=g, device=dev).to(torch.bfloat16)
@@ -709,6 +744,7 @@ def run_ours(args):
     if dist.rank == 0 and not args.no_paths:
         result["paths"] = {
             "w8a16_planes": planes_case_times(sweep),
+            "w8a16_bias": bias_case_times(sweep),
             "w8a8_static_k960": bench_w8a8_paths(dev),
             "w8a8_prefill_m4096": bench_w8a8_prefill(dev, peaks),
             "dq8ca_q4gsw": bench_q4(dev, peaks),

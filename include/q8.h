@@ -98,6 +98,25 @@ int q8_version(void);
 q8_status q8_quantize_weight(const float* W, int64_t N, int64_t K,
                              int8_t* q, float* s_w, int32_t* wsum, void* stream);
 
+/* Weight grids of q8_quantize_weight_grid. */
+typedef enum {
+    /* [ROCm-INT8] quantize_weight: s = absmax / 127, codes in [-127, 127] (the grid of
+     * q8_quantize_weight). */
+    Q8_GRID_SYM127 = 0,
+    /* [SmolVLM-Q8] weight_int8 (per-channel symmetric min/max observer on [-128, 127]):
+     *     s_w[n] = max(absmax(W[n,:]) / 127.5, FLT_EPSILON)    (fp32 IEEE division)
+     *     q[n,k] = clamp(round(W[n,k] / s_w[n]), -128, 127)   (division, ties to even)
+     * An all-zero row gets s_w[n] = FLT_EPSILON and all codes 0; the largest positive
+     * element of a row lands on 127 and the largest negative one on -128 or -127. */
+    Q8_GRID_FULL128 = 1
+} q8_grid;
+
+/* q8_quantize_weight on a chosen grid; same arguments and outputs otherwise (wsum is the
+ * code sum on that grid).  Q8_ERR_ARG for an unknown grid.  Every linear below accepts
+ * weights of either grid: codes of -128 are exact in the bf16 and int8 operand paths. */
+q8_status q8_quantize_weight_grid(const float* W, int64_t N, int64_t K, q8_grid grid,
+                                  int8_t* q, float* s_w, int32_t* wsum, void* stream);
+
 /* Per-row asymmetric int8 activation parameters.  [ET-21229] choose_qparams_affine
  * (formula of the per-tensor observer in [SmolVLM-Q8] act_observer), per row m:
  *     mn = min(0, min_k x), mx = max(0, max_k x)
@@ -161,6 +180,16 @@ q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w,
                           void* y, q8_dtype yt, int64_t M, int64_t N, int64_t K,
                           void* stream);
 
+/* q8_linear_w8a16 with a bias ([ROCm-INT8] Int8Linear keeps an optional bias and adds it
+ * after the scaled matmul):
+ *     y[m,n] = s_w[n] * sum_k x[m,k] * q[n,k] + bias[n]
+ * the product and the bias fused in one fp32 multiply-add, then one rounding to yt.
+ *   bias device fp32 [N] (4-byte aligned; Q8_ERR_ALIGN otherwise); NULL is q8_linear_w8a16.
+ * Same kernels and cost as q8_linear_w8a16 (the bias is read once per output column). */
+q8_status q8_linear_w8a16_bias(const void* x, const int8_t* q, const float* s_w,
+                               const float* bias, void* y, q8_dtype yt, int64_t M, int64_t N,
+                               int64_t K, void* stream);
+
 /* W8A16, same definition and arguments as q8_linear_w8a16, computed on the int8 tensor
  * cores for decode-sized M (1..16): the bf16 activations are rewritten once per call as
  * exact int8 digit planes (per row: base-128 digits of the values on a common power of
@@ -205,6 +234,17 @@ q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* sec
                          const int8_t* q, const int32_t* wsum, const float* s_w,
                          float* y, int64_t M, int64_t N, int64_t K,
                          void* workspace, size_t ws_bytes, void* stream);
+
+/* q8_linear_w8a8 with a bias.  [SmolVLM-Q8] Q8Linear.forward adds the bias to the first
+ * pass only (the residual pass is a bias-free linear), so the bias enters once:
+ *     y[m,n] = s_w[n] * (s1 * (acc1 - z1 * wsum[n]) [+ s2 * (acc2 - z2 * wsum[n])]) + bias[n]
+ * the last multiply and the bias fused in one fp32 multiply-add.
+ *   bias device fp32 [N] (4-byte aligned; Q8_ERR_ALIGN otherwise); NULL is q8_linear_w8a8.
+ * Other arguments, workspace and errors as q8_linear_w8a8. */
+q8_status q8_linear_w8a8_bias(const float* x, q8_qparams first, const q8_qparams* second,
+                              const int8_t* q, const int32_t* wsum, const float* s_w,
+                              const float* bias, float* y, int64_t M, int64_t N, int64_t K,
+                              void* workspace, size_t ws_bytes, void* stream);
 
 /* 8da4w: dynamic per-row int8 activations folded into the 4-bit group-symmetric
  * weight GEMM ([ET-21229] linear_dq8ca_q4gsw):

@@ -25,6 +25,8 @@ Q8_ERR_NULL, Q8_ERR_SHAPE, Q8_ERR_ALIGN, Q8_ERR_ARG = 1, 2, 3, 4
 Q8_ERR_UNSUPPORTED_ARCH, Q8_ERR_LAUNCH, Q8_ERR_WORKSPACE, Q8_ERR_DEVICE = 5, 6, 7, 8
 Q8_F32, Q8_BF16 = 0, 1
 Q8_OP_LINEAR_W8A8, Q8_OP_LINEAR_DQ8CA_Q4GSW, Q8_OP_LINEAR_W8A16_PLANES = 0, 1, 2
+Q8_GRID_SYM127, Q8_GRID_FULL128 = 0, 1
+_GRIDS = {"sym127": Q8_GRID_SYM127, "full128": Q8_GRID_FULL128}
 
 # Every entry point of include/q8.h, for export checks.
 SYMBOLS = (
@@ -33,6 +35,7 @@ SYMBOLS = (
     "q8_quantize_weight_q4gs", "q8_linear_w8a16", "q8_linear_w8a8", "q8_linear_dq8ca_q4gsw",
     "q8_workspace_bytes", "q8_gemm_s8s8_s32", "q8_last_device_status",
     "q8_linear_w8a8_noalloc", "q8_selftest_bounded_wait", "q8_linear_w8a16_planes",
+    "q8_quantize_weight_grid", "q8_linear_w8a16_bias", "q8_linear_w8a8_bias",
 )
 # Built-in scratch of q8_linear_w8a8_noalloc (bytes).
 Q8_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -67,6 +70,8 @@ def _lib() -> ctypes.CDLL:
     L.q8_version.restype = ctypes.c_int
     L.q8_quantize_weight.restype = st
     L.q8_quantize_weight.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp]
+    L.q8_quantize_weight_grid.restype = st
+    L.q8_quantize_weight_grid.argtypes = [_vp, _i64, _i64, st, _vp, _vp, _vp, _vp]
     L.q8_choose_qparams.restype = st
     L.q8_choose_qparams.argtypes = [_vp, st, _i64, _i64, _vp, _vp, _vp, _vp]
     L.q8_quantize_static.restype = st
@@ -81,12 +86,17 @@ def _lib() -> ctypes.CDLL:
     L.q8_quantize_weight_q4gs.argtypes = [_vp, _i64, _i64, st, _vp, _vp, _vp]
     L.q8_linear_w8a16.restype = st
     L.q8_linear_w8a16.argtypes = [_vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp]
+    L.q8_linear_w8a16_bias.restype = st
+    L.q8_linear_w8a16_bias.argtypes = [_vp, _vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp]
     L.q8_linear_w8a16_planes.restype = st
     L.q8_linear_w8a16_planes.argtypes = [_vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp, _sz,
                                          _vp]
     L.q8_linear_w8a8.restype = st
     L.q8_linear_w8a8.argtypes = [_vp, q8_qparams, ctypes.POINTER(q8_qparams), _vp, _vp, _vp,
                                  _vp, _i64, _i64, _i64, _vp, _sz, _vp]
+    L.q8_linear_w8a8_bias.restype = st
+    L.q8_linear_w8a8_bias.argtypes = [_vp, q8_qparams, ctypes.POINTER(q8_qparams), _vp, _vp,
+                                      _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp]
     L.q8_linear_dq8ca_q4gsw.restype = st
     L.q8_linear_dq8ca_q4gsw.argtypes = [_vp, _vp, _vp, st, _vp, _i64, _i64, _i64, _vp, _sz, _vp]
     L.q8_workspace_bytes.restype = _sz
@@ -160,8 +170,11 @@ def _qp(p) -> q8_qparams:
 
 
 def q8_quantize_weight(W: torch.Tensor, q=None, s_w=None, wsum=None, want_wsum=True,
-                       stream=None):
-    """Per-row symmetric int8 codes of an fp32 [N, K] weight -> (q, s_w, wsum|None)."""
+                       stream=None, grid: str = "sym127"):
+    """Per-row symmetric int8 codes of an fp32 [N, K] weight -> (q, s_w, wsum|None).
+    grid "sym127": amax/127 on [-127, 127]; "full128": max(amax/127.5, eps) on [-128, 127]."""
+    if grid not in _GRIDS:
+        raise ValueError(f"grid must be one of {sorted(_GRIDS)}")
     if W.dim() != 2:
         raise ValueError("W must be 2-D [N, K]")
     N, K = W.shape
@@ -170,8 +183,8 @@ def q8_quantize_weight(W: torch.Tensor, q=None, s_w=None, wsum=None, want_wsum=T
     s_w = _out(s_w, "s_w", torch.float32, (N,), W.device)
     if want_wsum or wsum is not None:
         wsum = _out(wsum, "wsum", torch.int32, (N,), W.device)
-    _check(_lib().q8_quantize_weight(_ptr(W), N, K, _ptr(q), _ptr(s_w), _ptr(wsum),
-                                     _stream(stream)), "q8_quantize_weight")
+    _check(_lib().q8_quantize_weight_grid(_ptr(W), N, K, _GRIDS[grid], _ptr(q), _ptr(s_w),
+                                          _ptr(wsum), _stream(stream)), "q8_quantize_weight")
     return q, s_w, wsum
 
 
@@ -252,19 +265,27 @@ def _workspace(ws, nbytes, device):
 
 
 def q8_linear_w8a16(x: torch.Tensor, q: torch.Tensor, s_w: torch.Tensor, y=None,
-                    out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
-    """y[m,n] = s_w[n] * sum_k x[m,k] q[n,k]; x bf16 [M,K], q int8 [N,K], y bf16|fp32 [M,N]."""
+                    out_dtype: torch.dtype = torch.bfloat16, stream=None,
+                    bias: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y[m,n] = s_w[n] * sum_k x[m,k] q[n,k] (+ bias[n]); x bf16 [M,K], q int8 [N,K],
+    bias fp32 [N], y bf16|fp32 [M,N]."""
     M, K = x.shape
     N = q.shape[0]
     _need(x, "x", torch.bfloat16, (M, K))
     _need(q, "q", torch.int8, (N, K))
     _need(s_w, "s_w", torch.float32, (N,))
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (N,))
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out_dtype must be bfloat16 or float32")
     y = _out(y, "y", out_dtype, (M, N), x.device)
     yt = Q8_BF16 if y.dtype == torch.bfloat16 else Q8_F32
-    _check(_lib().q8_linear_w8a16(_ptr(x), _ptr(q), _ptr(s_w), _ptr(y), yt, M, N, K,
-                                  _stream(stream)), "q8_linear_w8a16")
+    if bias is None:
+        _check(_lib().q8_linear_w8a16(_ptr(x), _ptr(q), _ptr(s_w), _ptr(y), yt, M, N, K,
+                                      _stream(stream)), "q8_linear_w8a16")
+    else:
+        _check(_lib().q8_linear_w8a16_bias(_ptr(x), _ptr(q), _ptr(s_w), _ptr(bias), _ptr(y), yt,
+                                           M, N, K, _stream(stream)), "q8_linear_w8a16_bias")
     return y
 
 
@@ -300,21 +321,30 @@ def q8_linear_w8a16_planes(x: torch.Tensor, q: torch.Tensor, s_w: torch.Tensor, 
 
 def q8_linear_w8a8(x: torch.Tensor, first, q: torch.Tensor, wsum: torch.Tensor,
                    s_w: torch.Tensor, second=None, y=None, workspace=None,
-                   stream=None) -> torch.Tensor:
-    """Static int8 activations x int8 weights (one or two passes); fp32 in, fp32 out."""
+                   stream=None, bias: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Static int8 activations x int8 weights (one or two passes); fp32 in, fp32 out; an
+    fp32 [N] bias is added once (the first pass's)."""
     M, K = x.shape
     N = q.shape[0]
     _need(x, "x", torch.float32, (M, K))
     _need(q, "q", torch.int8, (N, K))
     _need(wsum, "wsum", torch.int32, (N,))
     _need(s_w, "s_w", torch.float32, (N,))
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (N,))
     y = _out(y, "y", torch.float32, (M, N), x.device)
     nbytes = q8_workspace_bytes(Q8_OP_LINEAR_W8A8, M, N, K, int(second is not None))
     workspace, wsb = _workspace(workspace, nbytes, x.device)
     sec = None if second is None else ctypes.byref(_qp(second))
-    _check(_lib().q8_linear_w8a8(_ptr(x), _qp(first), sec, _ptr(q), _ptr(wsum), _ptr(s_w),
-                                 _ptr(y), M, N, K, _ptr(workspace), wsb, _stream(stream)),
-           "q8_linear_w8a8")
+    if bias is None:
+        _check(_lib().q8_linear_w8a8(_ptr(x), _qp(first), sec, _ptr(q), _ptr(wsum), _ptr(s_w),
+                                     _ptr(y), M, N, K, _ptr(workspace), wsb, _stream(stream)),
+               "q8_linear_w8a8")
+    else:
+        _check(_lib().q8_linear_w8a8_bias(_ptr(x), _qp(first), sec, _ptr(q), _ptr(wsum),
+                                          _ptr(s_w), _ptr(bias), _ptr(y), M, N, K,
+                                          _ptr(workspace), wsb, _stream(stream)),
+               "q8_linear_w8a8_bias")
     return y
 
 

@@ -6,6 +6,7 @@
 //   EPI_S32 : acc itself (the exported int32 GEMM);
 //   EPI_W8A8: y = s_w[n] * s1 * (acc1 - z1 * wsum[n])                 (one pass);
 //   EPI_TWO : y = s_w[n] * (s1 * (acc1 - z1 wsum[n]) + s2 * (acc2 - z2 wsum[n]))
+//   (the two W8A8 forms add bias[n] once, when a bias is given)
 //             where acc1 and acc2 come from the two activation-code tensors of the
 //             two-pass residual and share every weight tile.
 //
@@ -60,6 +61,7 @@ struct TcEpi {
     int z1, z2;
     const int32_t* wsum;
     const float* s_w;
+    const float* bias;     // nullable
     float* y;
     int32_t* acc;
 };
@@ -115,7 +117,8 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 // -------------------------------------------------------------------- the kernel
-template <int EPI>
+// BIAS: the W8A8 epilogues add ep.bias[n] (staged per tile like s_w and wsum).
+template <int EPI, bool BIAS>
 __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
     const __grid_constant__ CUtensorMap amap1, const __grid_constant__ CUtensorMap amap2,
     const __grid_constant__ CUtensorMap bmap, int M, int N, int K, TcEpi ep, int* status) {
@@ -133,6 +136,7 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* epi_sw = reinterpret_cast<float*>(ctrl + 1024);      // [2][256]
     int* epi_ws = reinterpret_cast<int*>(ctrl + 1024 + 2048);   // [2][256] (ends at 5 KB)
+    float* epi_b = reinterpret_cast<float*>(ctrl + 5120);        // [2][256] (ends at 7 KB)
     float* epi_tile = reinterpret_cast<float*>(ctrl + 8192);     // [4 warps][32][36]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -254,6 +258,7 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
                     const int n = n0 + i;
                     epi_sw[acc * 256 + i] = n < N ? __ldg(ep.s_w + n) : 0.0f;
                     epi_ws[acc * 256 + i] = n < N ? __ldg(ep.wsum + n) : 0;
+                    if (BIAS) epi_b[acc * 256 + i] = n < N ? __ldg(ep.bias + n) : 0.0f;
                 }
                 named_bar_sync(2, 128);
             }
@@ -299,8 +304,14 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
                         for (int j = 0; j < 32; ++j)
                             v[j] += ep.s2 * (float)((int)r2[j] - ep.z2 * ws[j]);
                     }
+                    if (BIAS) {
+                        const float* bb = epi_b + acc * 256 + c * 32;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] *= sw[j];
+                        for (int j = 0; j < 32; ++j) v[j] = fmaf(v[j], sw[j], bb[j]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] *= sw[j];
+                    }
                     // Each thread holds one output row; written directly, every store
                     // instruction would touch 32 rows.  Transpose the warp's 32 x 32 chunk
                     // through shared memory (rows padded to 36 floats: conflict-free
@@ -349,7 +360,7 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
 }
 
 // ----------------------------------------------------------------------- host side
-template <int EPI>
+template <int EPI, bool BIAS = false>
 static cudaError_t launch_tc(const int8_t* a1, const int8_t* a2, const int8_t* b, int M, int N,
                              int K, const TcEpi& ep, cudaStream_t st, int num_sms, int* status) {
     using C = TcCfg<EPI>;
@@ -360,7 +371,7 @@ static cudaError_t launch_tc(const int8_t* a1, const int8_t* a2, const int8_t* b
         return cudaErrorInvalidValue;
     if (!make_tmap_u8_2d(&mb, b, N, K, TC_BK, C::BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_dyn_smem<k_gemm_tc<EPI>>((int)(C::SMEM + 1024));
+    cudaError_t e = ensure_dyn_smem<k_gemm_tc<EPI, BIAS>>((int)(C::SMEM + 1024));
     if (e != cudaSuccess) return e;
     const int tiles = ((M + TC_BM - 1) / TC_BM) * ((N + C::BN - 1) / C::BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
@@ -374,7 +385,7 @@ static cudaError_t launch_tc(const int8_t* a1, const int8_t* a2, const int8_t* b
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_gemm_tc<EPI>, ma1, ma2, mb, M, N, K, ep, status);
+    return cudaLaunchKernelEx(&cfg, k_gemm_tc<EPI, BIAS>, ma1, ma2, mb, M, N, K, ep, status);
 }
 
 cudaError_t launch_gemm_s8s8_s32_tc(const int8_t* a, const int8_t* b, int32_t* acc, int64_t M,
@@ -387,9 +398,10 @@ cudaError_t launch_gemm_s8s8_s32_tc(const int8_t* a, const int8_t* b, int32_t* a
 
 cudaError_t launch_w8a8_tc(const int8_t* xq1, const int8_t* xq2, float s1, int z1, int has2,
                            float s2, int z2, const int8_t* q, const int32_t* wsum,
-                           const float* s_w, float* y, int64_t M, int64_t N, int K,
-                           cudaStream_t st, int num_sms, int* status) {
+                           const float* s_w, const float* bias, float* y, int64_t M, int64_t N,
+                           int K, cudaStream_t st, int num_sms, int* status) {
     TcEpi ep = {};
+    ep.bias = bias;
     ep.s1 = s1;
     ep.z1 = z1;
     ep.s2 = s2;
@@ -397,15 +409,16 @@ cudaError_t launch_w8a8_tc(const int8_t* xq1, const int8_t* xq2, float s1, int z
     ep.wsum = wsum;
     ep.s_w = s_w;
     ep.y = y;
-    if (has2)
-        return launch_tc<EPI_TWO>(xq1, xq2, q, (int)M, (int)N, K, ep, st, num_sms, status);
+#define TC_W8A8(EPI_, A2_)                                                                  \
+    (bias ? launch_tc<EPI_, true>(xq1, A2_, q, (int)M, (int)N, K, ep, st, num_sms, status)  \
+          : launch_tc<EPI_, false>(xq1, A2_, q, (int)M, (int)N, K, ep, st, num_sms, status))
+    if (has2) return TC_W8A8(EPI_TWO, xq2);
     // 256-row weight tiles unless they would give fewer than two tiles per SM: then the
     // last round of tiles leaves most SMs idle, and 128-row tiles halve that round
     const int64_t tiles256 = ((M + TC_BM - 1) / TC_BM) * ((N + 255) / 256);
-    if (tiles256 < 2 * (int64_t)num_sms)
-        return launch_tc<EPI_W8A8_N128>(xq1, nullptr, q, (int)M, (int)N, K, ep, st, num_sms,
-                                        status);
-    return launch_tc<EPI_W8A8>(xq1, nullptr, q, (int)M, (int)N, K, ep, st, num_sms, status);
+    if (tiles256 < 2 * (int64_t)num_sms) return TC_W8A8(EPI_W8A8_N128, nullptr);
+    return TC_W8A8(EPI_W8A8, nullptr);
+#undef TC_W8A8
 }
 
 }  // namespace q8

@@ -24,11 +24,12 @@ constexpr int GEMV_THREADS = 128;
 constexpr int GEMV_WARPS = GEMV_THREADS / 32;
 
 // ------------------------------------------------------------------------- W8A16
-// y[m, n] = s_w[n] * sum_k x[m, k] * q[n, k]; MT n8-tiles cover 8*MT activation rows.
+// y[m, n] = s_w[n] * sum_k x[m, k] * q[n, k] (+ bias[n]); MT n8-tiles cover 8*MT
+// activation rows.
 template <int MT, int UNROLL>
 __global__ __launch_bounds__(GEMV_THREADS) void k_w8a16_gemv(
     const uint16_t* __restrict__ x, const int8_t* __restrict__ q, const float* __restrict__ s_w,
-    void* __restrict__ y, int y_bf16, int M, int N, int K) {
+    const float* __restrict__ bias, void* __restrict__ y, int y_bf16, int M, int N, int K) {
     __shared__ float red[GEMV_WARPS][MT][32][4];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -104,7 +105,8 @@ __global__ __launch_bounds__(GEMV_THREADS) void k_w8a16_gemv(
         const int m = m0 + mt * 8 + 2 * (l & 3) + (ci & 1);
         const int n = n0 + (l >> 2) + 8 * (ci >> 1);
         if (m < M && n < N) {
-            const float r = v * __ldg(s_w + n);
+            const float sv = __ldg(s_w + n);
+            const float r = bias ? fmaf(v, sv, __ldg(bias + n)) : v * sv;
             if (y_bf16)
                 reinterpret_cast<__nv_bfloat16*>(y)[(int64_t)m * N + n] = __float2bfloat16_rn(r);
             else
@@ -115,12 +117,13 @@ __global__ __launch_bounds__(GEMV_THREADS) void k_w8a16_gemv(
 
 // -------------------------------------------------------------------------- W8A8
 // acc = sum_k xq * q (int32, exact) from activation codes xq1 (and xq2) [M, K];
-// y[m, n] = s_w[n] * (s1 * (acc1 - z1 * wsum[n]) + s2 * (acc2 - z2 * wsum[n])).
+// y[m, n] = s_w[n] * (s1 * (acc1 - z1 * wsum[n]) + s2 * (acc2 - z2 * wsum[n])) (+ bias[n]).
 template <int MT, int UNROLL, bool TWO>
 __global__ __launch_bounds__(GEMV_THREADS) void k_w8a8_gemv(
     const int8_t* __restrict__ xq1, const int8_t* __restrict__ xq2, float s1, int z1, float s2,
     int z2, const int8_t* __restrict__ q, const int32_t* __restrict__ wsum,
-    const float* __restrict__ s_w, float* __restrict__ y, int M, int N, int K) {
+    const float* __restrict__ s_w, const float* __restrict__ bias, float* __restrict__ y, int M,
+    int N, int K) {
     __shared__ int red[GEMV_WARPS][TWO ? 2 : 1][MT][32][4];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -210,23 +213,26 @@ __global__ __launch_bounds__(GEMV_THREADS) void k_w8a8_gemv(
             const int ws = __ldg(wsum + n);
             float v = s1 * (float)(a1 - z1 * ws);
             if (TWO) v += s2 * (float)(a2 - z2 * ws);
-            y[(int64_t)m * N + n] = __ldg(s_w + n) * v;
+            y[(int64_t)m * N + n] =
+                bias ? fmaf(__ldg(s_w + n), v, __ldg(bias + n)) : __ldg(s_w + n) * v;
         }
     }
 }
 
 // ---------------------------------------------------------------------- launchers
-cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
-                              int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,
-                              int num_sms) {
+cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w,
+                              const float* bias, void* y, int y_bf16, int64_t M, int64_t N, int K,
+                              cudaStream_t st, int num_sms) {
     (void)num_sms;
     const unsigned gx = (unsigned)((N + 15) / 16);
     if (M <= 8) {
         dim3 grid(gx, 1);
-        k_w8a16_gemv<1, 4><<<grid, GEMV_THREADS, 0, st>>>(x, q, s_w, y, y_bf16, (int)M, (int)N, K);
+        k_w8a16_gemv<1, 4><<<grid, GEMV_THREADS, 0, st>>>(x, q, s_w, bias, y, y_bf16, (int)M,
+                                                          (int)N, K);
     } else {
         dim3 grid(gx, (unsigned)((M + 15) / 16));
-        k_w8a16_gemv<2, 2><<<grid, GEMV_THREADS, 0, st>>>(x, q, s_w, y, y_bf16, (int)M, (int)N, K);
+        k_w8a16_gemv<2, 2><<<grid, GEMV_THREADS, 0, st>>>(x, q, s_w, bias, y, y_bf16, (int)M,
+                                                          (int)N, K);
     }
     return cudaGetLastError();
 }
@@ -234,8 +240,8 @@ cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s
 template <int MT, int U, bool TWO>
 static cudaError_t launch_w8a8_gemv_t(dim3 grid, const int8_t* xq1, const int8_t* xq2, float s1,
                                       int z1, float s2, int z2, const int8_t* q,
-                                      const int32_t* wsum, const float* s_w, float* y, int M,
-                                      int N, int K, cudaStream_t st) {
+                                      const int32_t* wsum, const float* s_w, const float* bias,
+                                      float* y, int M, int N, int K, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(GEMV_THREADS);
@@ -247,26 +253,26 @@ static cudaError_t launch_w8a8_gemv_t(dim3 grid, const int8_t* xq1, const int8_t
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k_w8a8_gemv<MT, U, TWO>, xq1, xq2, s1, z1, s2, z2, q, wsum,
-                              s_w, y, M, N, K);
+                              s_w, bias, y, M, N, K);
 }
 
 cudaError_t launch_w8a8_gemv_codes(const int8_t* xq1, const int8_t* xq2, float s1, int z1,
                                    int has2, float s2, int z2, const int8_t* q,
-                                   const int32_t* wsum, const float* s_w, float* y, int64_t M,
-                                   int64_t N, int K, cudaStream_t st) {
+                                   const int32_t* wsum, const float* s_w, const float* bias,
+                                   float* y, int64_t M, int64_t N, int K, cudaStream_t st) {
     const unsigned gx = (unsigned)((N + 15) / 16);
     if (M <= 8) {
         dim3 grid(gx, 1);
         return has2 ? launch_w8a8_gemv_t<1, 4, true>(grid, xq1, xq2, s1, z1, s2, z2, q, wsum, s_w,
-                                                     y, (int)M, (int)N, K, st)
+                                                     bias, y, (int)M, (int)N, K, st)
                     : launch_w8a8_gemv_t<1, 4, false>(grid, xq1, xq2, s1, z1, s2, z2, q, wsum,
-                                                      s_w, y, (int)M, (int)N, K, st);
+                                                      s_w, bias, y, (int)M, (int)N, K, st);
     }
     dim3 grid(gx, (unsigned)((M + 15) / 16));
-    return has2 ? launch_w8a8_gemv_t<2, 2, true>(grid, xq1, xq2, s1, z1, s2, z2, q, wsum, s_w, y,
-                                                 (int)M, (int)N, K, st)
+    return has2 ? launch_w8a8_gemv_t<2, 2, true>(grid, xq1, xq2, s1, z1, s2, z2, q, wsum, s_w,
+                                                 bias, y, (int)M, (int)N, K, st)
                 : launch_w8a8_gemv_t<2, 2, false>(grid, xq1, xq2, s1, z1, s2, z2, q, wsum, s_w,
-                                                  y, (int)M, (int)N, K, st);
+                                                  bias, y, (int)M, (int)N, K, st);
 }
 
 }  // namespace q8

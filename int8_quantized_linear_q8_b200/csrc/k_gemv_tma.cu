@@ -56,14 +56,15 @@ constexpr int WT_SLOTS = 16;                            // most partial-sum slot
 struct WtSmem {
     int stages;
     int nslots;                        // partial-sum slots (row groups in flight)
-    size_t ring, xs, red, sws, bars, total;
+    size_t ring, xs, red, sws, sbias, bars, total;
 };
 
 // Rows of q a CTA may own (its s_w slice is staged in shared memory).
 constexpr int WT_MAX_ROWS = 1024;
 
 template <int SL>
-static __host__ __device__ inline WtSmem wt_layout(int M, int K, int MT, int stages, bool xt) {
+static __host__ __device__ inline WtSmem wt_layout(int M, int K, int MT, int stages, bool xt,
+                                                   bool bias = false) {
     WT_GEOMETRY(SL);
     WtSmem L;
     L.stages = stages;
@@ -80,7 +81,8 @@ static __host__ __device__ inline WtSmem wt_layout(int M, int K, int MT, int sta
     if (L.nslots > WT_SLOTS) L.nslots = WT_SLOTS;
     const size_t redbytes = (size_t)L.nslots * WT_CONSUMERS * MT * 32 * 4 * sizeof(float);
     L.sws = L.red + redbytes;
-    L.bars = L.sws + (size_t)WT_MAX_ROWS * sizeof(float);
+    L.sbias = L.sws + (size_t)WT_MAX_ROWS * sizeof(float);       // bias slice, when given
+    L.bars = L.sbias + (bias ? (size_t)WT_MAX_ROWS * sizeof(float) : 0);
     // barriers, slot counters, abort flag, TMEM address
     L.total = L.bars + (size_t)2 * stages * sizeof(uint64_t) + (WT_SLOTS + 4) * sizeof(int);
     return L;
@@ -120,17 +122,18 @@ __device__ __forceinline__ void tmem_wait_ld_x8(uint32_t (&v)[8]) {
                    "+r"(v[6]), "+r"(v[7])::"memory");
 }
 
-template <int MT, bool XT, int SL>
+template <int MT, bool XT, int SL, bool BIAS>
 __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
     const __grid_constant__ CUtensorMap wmap, const uint16_t* __restrict__ x,
-    const float* __restrict__ s_w, void* __restrict__ y, int y_bf16, int M, int N, int K,
-    int stages, int* status) {
+    const float* __restrict__ s_w, const float* __restrict__ bias, void* __restrict__ y,
+    int y_bf16, int M, int N, int K, int stages, int* status) {
     WT_GEOMETRY(SL);
     extern __shared__ __align__(1024) uint8_t smem[];
-    const WtSmem L = wt_layout<SL>(M, K, MT, stages, XT);
+    const WtSmem L = wt_layout<SL>(M, K, MT, stages, XT, BIAS);
     uint8_t* ring = smem + L.ring;
     float* slots = reinterpret_cast<float*>(smem + L.red);  // [nslots][WT_CONSUMERS][MT][32][4]
     float* sws = reinterpret_cast<float*>(smem + L.sws);          // s_w of this CTA's rows
+    float* sbias = reinterpret_cast<float*>(smem + L.sbias);      // and their bias (BIAS)
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint64_t* empty = full + stages;
     int* cnt = reinterpret_cast<int*>(empty + stages);               // [WT_SLOTS]
@@ -217,7 +220,10 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
         // The epilogue must not wait on global loads (a stalled warp holds back the ring):
         // stage this CTA's per-channel scales once.
         const int row0 = rg0 * 16, rows = min(rg1 * 16, N) - row0;
-        for (int i = threadIdx.x; i < rows; i += WT_CONSUMERS * 32) sws[i] = __ldg(s_w + row0 + i);
+        for (int i = threadIdx.x; i < rows; i += WT_CONSUMERS * 32) {
+            sws[i] = __ldg(s_w + row0 + i);
+            if (BIAS) sbias[i] = __ldg(bias + row0 + i);
+        }
     }
     const int g = lane >> 2, t = lane & 3;
     const int Kpad = nst * WT_SLABS * 64;
@@ -441,7 +447,9 @@ __global__ __launch_bounds__(WT_THREADS, 1) void k_w8a16_tma(
                     const int m = mt * 8 + 2 * t + (i & 1);
                     const int n = n0 + g + 8 * (i >> 1);
                     if (m < M && n < N) {
-                        const float r = vv[mt][i] * sws[n - rg0 * 16];
+                        const float sv = sws[n - rg0 * 16];
+                        const float r = BIAS ? fmaf(vv[mt][i], sv, sbias[n - rg0 * 16])
+                                             : vv[mt][i] * sv;
                         if (y_bf16)
                             reinterpret_cast<__nv_bfloat16*>(y)[(int64_t)m * N + n] =
                                 __float2bfloat16_rn(r);
@@ -537,7 +545,7 @@ static bool wt_use_wide(int M, int K, int64_t N, int num_sms) {
 // Whether the TMA path takes this problem: K % 64 == 0, M <= 16 and the activations fit
 // in tensor memory, or in shared memory next to at least 4 ring stages (16-slab stages;
 // 32-slab stages are only chosen where they fit too).
-bool w8a16_tma_fits(int64_t M, int64_t K) {
+bool w8a16_tma_fits(int64_t M, int64_t K, bool bias) {
     WT_GEOMETRY(16);
     if (M < 1 || M > 16 || (K % 64) != 0 || K > (int64_t)1 << 30) return false;
     const int MT = M <= 8 ? 1 : 2;
@@ -545,18 +553,20 @@ bool w8a16_tma_fits(int64_t M, int64_t K) {
     if (wt_tmem_cols<16>(nst, MT) <= WT_TMEM_MAX_COLS) return true;
     // (with 9..16 rows, activations too long for tensor memory do not fit shared memory
     // next to 4 stages either)
-    return MT == 1 && wt_layout<16>((int)M, (int)K, 1, 4, false).total <= (size_t)WT_MAX_SMEM;
+    return MT == 1 &&
+           wt_layout<16>((int)M, (int)K, 1, 4, false, bias).total <= (size_t)WT_MAX_SMEM;
 }
 
-template <int MT, bool XT, int SL>
-static cudaError_t launch_wt(const CUtensorMap& map, const uint16_t* x, const float* s_w, void* y,
-                             int y_bf16, int M, int N, int K, cudaStream_t st, int num_sms,
-                             int* status) {
+template <int MT, bool XT, int SL, bool BIAS>
+static cudaError_t launch_wt(const CUtensorMap& map, const uint16_t* x, const float* s_w,
+                             const float* bias, void* y, int y_bf16, int M, int N, int K,
+                             cudaStream_t st, int num_sms, int* status) {
     int stages = 8;    // must stay <= WT_SLOTS - 2
-    while (stages > 4 && wt_layout<SL>(M, K, MT, stages, XT).total > (size_t)WT_MAX_SMEM)
+    while (stages > 4 && wt_layout<SL>(M, K, MT, stages, XT, BIAS).total > (size_t)WT_MAX_SMEM)
         --stages;
-    const WtSmem L = wt_layout<SL>(M, K, MT, stages, XT);
-    cudaError_t e = ensure_dyn_smem<k_w8a16_tma<MT, XT, SL>>((int)L.total);
+    const WtSmem L = wt_layout<SL>(M, K, MT, stages, XT, BIAS);
+    if (L.total > (size_t)WT_MAX_SMEM) return cudaErrorInvalidValue;
+    cudaError_t e = ensure_dyn_smem<k_w8a16_tma<MT, XT, SL, BIAS>>((int)L.total);
     if (e != cudaSuccess) return e;
     const int RG = (N + 15) / 16;
     int grid = RG < num_sms ? RG : num_sms;
@@ -572,26 +582,29 @@ static cudaError_t launch_wt(const CUtensorMap& map, const uint16_t* x, const fl
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_w8a16_tma<MT, XT, SL>, map, x, s_w, y, y_bf16, M, N, K,
-                              stages, status);
+    return cudaLaunchKernelEx(&cfg, k_w8a16_tma<MT, XT, SL, BIAS>, map, x, s_w, bias, y, y_bf16, M,
+                              N, K, stages, status);
 }
 
-cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
-                             int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,
-                             int num_sms, int* status) {
+cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_w,
+                             const float* bias, void* y, int y_bf16, int64_t M, int64_t N, int K,
+                             cudaStream_t st, int num_sms, int* status) {
     CUtensorMap map;
     if (!make_tmap_u8_2d(&map, q, N, K, WT_BOX, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     const int m = (int)M, n = (int)N;
+#define WT_LAUNCH(MT_, XT_, SL_)                                                            \
+    (bias ? launch_wt<MT_, XT_, SL_, true>(map, x, s_w, bias, y, y_bf16, m, n, K, st, num_sms, \
+                                           status)                                         \
+          : launch_wt<MT_, XT_, SL_, false>(map, x, s_w, bias, y, y_bf16, m, n, K, st,        \
+                                            num_sms, status))
     if (wt_use_wide(m, K, N, num_sms))
-        return M <= 8 ? launch_wt<1, true, 32>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status)
-                      : launch_wt<2, true, 32>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status);
+        return M <= 8 ? WT_LAUNCH(1, true, 32) : WT_LAUNCH(2, true, 32);
     const bool xt = wt_use_tmem(m, K, N, num_sms);
-    if (M <= 8)
-        return xt ? launch_wt<1, true, 16>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status)
-                  : launch_wt<1, false, 16>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status);
+    if (M <= 8) return xt ? WT_LAUNCH(1, true, 16) : WT_LAUNCH(1, false, 16);
     if (!xt) return cudaErrorInvalidValue;             // excluded by w8a16_tma_fits
-    return launch_wt<2, true, 16>(map, x, s_w, y, y_bf16, m, n, K, st, num_sms, status);
+    return WT_LAUNCH(2, true, 16);
+#undef WT_LAUNCH
 }
 
 }  // namespace q8

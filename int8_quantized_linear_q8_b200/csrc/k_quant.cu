@@ -46,10 +46,15 @@ __device__ __forceinline__ int block_sum_i(int v, int* red) {
 // ------------------------------------------------------------ int8 weight codes (a1)
 // One CTA per row n.  Pass 1: absmax.  Pass 2 (row re-read from L1/L2): codes with a
 // true division by the scale, the code sum, and 4-byte code stores.
+//   full == 0 (ROCm-INT8 quantize_weight): s = amax / 127, codes clamp(rne(w / s), -127, 127);
+//             an all-zero row gets s = 1 and zero codes.
+//   full == 1 (SmolVLM-Q8 weight_int8, the per-channel symmetric min/max observer):
+//             s = max(amax / 127.5, FLT_EPSILON), codes clamp(rne(w / s), -128, 127).
 constexpr int QW_THREADS = 256;
 
 __global__ __launch_bounds__(QW_THREADS) void k_quantize_weight(const float* __restrict__ W,
-                                                                int K, int8_t* __restrict__ q,
+                                                                int K, int full,
+                                                                int8_t* __restrict__ q,
                                                                 float* __restrict__ s_w,
                                                                 int32_t* __restrict__ wsum) {
     __shared__ float redf[QW_THREADS / 32];
@@ -63,19 +68,21 @@ __global__ __launch_bounds__(QW_THREADS) void k_quantize_weight(const float* __r
         amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
     }
     amax = block_max<QW_THREADS>(amax, redf);
-    float scale = __fdiv_rn(amax, 127.0f);
-    const bool zero = (scale == 0.0f);
+    float scale = __fdiv_rn(amax, full ? 127.5f : 127.0f);
+    const bool zero = !full && scale == 0.0f;
     if (zero) scale = 1.0f;
+    if (full && scale < FLT_EPSILON) scale = FLT_EPSILON;
+    const float lo = full ? -128.0f : -127.0f;
     int sum = 0;
     uint32_t* qrow = reinterpret_cast<uint32_t*>(q + n * (int64_t)K);
     for (int i = threadIdx.x; i < K4; i += QW_THREADS) {
         int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
         if (!zero) {
             float4 v = ldg_f4(row + 4 * i);
-            c0 = weight_code(v.x, scale, 127.0f);
-            c1 = weight_code(v.y, scale, 127.0f);
-            c2 = weight_code(v.z, scale, 127.0f);
-            c3 = weight_code(v.w, scale, 127.0f);
+            c0 = weight_code(v.x, scale, lo, 127.0f);
+            c1 = weight_code(v.y, scale, lo, 127.0f);
+            c2 = weight_code(v.z, scale, lo, 127.0f);
+            c3 = weight_code(v.w, scale, lo, 127.0f);
         }
         sum += c0 + c1 + c2 + c3;
         qrow[i] = pack4_s8(c0, c1, c2, c3);
@@ -324,7 +331,7 @@ __global__ __launch_bounds__(256) void k_quantize_weight_q4gs(const float* __res
     if (zero) scale = 1.0f;
     int c[E];
 #pragma unroll
-    for (int j = 0; j < E; ++j) c[j] = zero ? 0 : weight_code(v[j], scale, 7.0f);
+    for (int j = 0; j < E; ++j) c[j] = zero ? 0 : weight_code(v[j], scale, -7.0f, 7.0f);
     uint8_t* out = q4 + n * (int64_t)(K / 2) + ((int64_t)gi * G + lane * E) / 2;
     if constexpr (E == 1) {
         int other = __shfl_down_sync(0xffffffffu, c[0], 1);
@@ -341,9 +348,9 @@ __global__ __launch_bounds__(256) void k_quantize_weight_q4gs(const float* __res
 }
 
 // ---------------------------------------------------------------------- launchers
-cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int8_t* q, float* s_w,
-                                   int32_t* wsum, cudaStream_t st) {
-    k_quantize_weight<<<(unsigned)N, QW_THREADS, 0, st>>>(W, K, q, s_w, wsum);
+cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int full, int8_t* q,
+                                   float* s_w, int32_t* wsum, cudaStream_t st) {
+    k_quantize_weight<<<(unsigned)N, QW_THREADS, 0, st>>>(W, K, full, q, s_w, wsum);
     return cudaGetLastError();
 }
 

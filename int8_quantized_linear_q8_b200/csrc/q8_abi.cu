@@ -73,6 +73,7 @@ static q8_status current_device(int& num_sms, int** status = nullptr) {
 }
 
 static inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+static inline bool aligned4(const void* p) { return ((uintptr_t)p & 3u) == 0; }
 
 static inline q8_status check_k(int64_t K) {
     if (K < 16 || K > 65535 || (K % 16) != 0) return Q8_ERR_SHAPE;
@@ -194,13 +195,20 @@ int q8_version(void) { return 100; }
 
 q8_status q8_quantize_weight(const float* W, int64_t N, int64_t K, int8_t* q, float* s_w,
                              int32_t* wsum, void* stream) {
+    return q8_quantize_weight_grid(W, N, K, Q8_GRID_SYM127, q, s_w, wsum, stream);
+}
+
+q8_status q8_quantize_weight_grid(const float* W, int64_t N, int64_t K, q8_grid grid, int8_t* q,
+                                  float* s_w, int32_t* wsum, void* stream) {
+    if (grid != Q8_GRID_SYM127 && grid != Q8_GRID_FULL128) return Q8_ERR_ARG;
     if (!W || !q || !s_w) return Q8_ERR_NULL;
     if (N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
     Q8_TRY(check_k(K));
     if (!aligned16(W) || !aligned16(q)) return Q8_ERR_ALIGN;
     int sms = 0;
     Q8_TRY(current_device(sms));
-    return launched(launch_quantize_weight(W, N, (int)K, q, s_w, wsum, (cudaStream_t)stream));
+    return launched(launch_quantize_weight(W, N, (int)K, grid == Q8_GRID_FULL128 ? 1 : 0, q, s_w,
+                                           wsum, (cudaStream_t)stream));
 }
 
 q8_status q8_choose_qparams(const void* x, q8_dtype xt, int64_t M, int64_t K, float* s,
@@ -277,20 +285,26 @@ q8_status q8_quantize_weight_q4gs(const float* W, int64_t N, int64_t K, int G, u
 
 q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w, void* y,
                           q8_dtype yt, int64_t M, int64_t N, int64_t K, void* stream) {
+    return q8_linear_w8a16_bias(x, q, s_w, nullptr, y, yt, M, N, K, stream);
+}
+
+q8_status q8_linear_w8a16_bias(const void* x, const int8_t* q, const float* s_w,
+                               const float* bias, void* y, q8_dtype yt, int64_t M, int64_t N,
+                               int64_t K, void* stream) {
     if (yt != Q8_F32 && yt != Q8_BF16) return Q8_ERR_ARG;
     if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
     Q8_TRY(check_k(K));
     if (M == 0) return Q8_OK;
     if (!x || !q || !s_w || !y) return Q8_ERR_NULL;
-    if (!aligned16(x) || !aligned16(q)) return Q8_ERR_ALIGN;
+    if (!aligned16(x) || !aligned16(q) || !aligned4(bias)) return Q8_ERR_ALIGN;
     int sms = 0;
     int* status = nullptr;
     Q8_TRY(current_device(sms, &status));
-    if (w8a16_tma_fits(M, K))
-        return launched(launch_w8a16_tma((const uint16_t*)x, q, s_w, y, yt == Q8_BF16, M, N,
-                                         (int)K, (cudaStream_t)stream, sms, status));
-    return launched(launch_w8a16_gemv((const uint16_t*)x, q, s_w, y, yt == Q8_BF16, M, N, (int)K,
-                                      (cudaStream_t)stream, sms));
+    if (w8a16_tma_fits(M, K, bias != nullptr))
+        return launched(launch_w8a16_tma((const uint16_t*)x, q, s_w, bias, y, yt == Q8_BF16, M,
+                                         N, (int)K, (cudaStream_t)stream, sms, status));
+    return launched(launch_w8a16_gemv((const uint16_t*)x, q, s_w, bias, y, yt == Q8_BF16, M, N,
+                                      (int)K, (cudaStream_t)stream, sms));
 }
 
 q8_status q8_linear_w8a16_planes(const void* x, const int8_t* q, const float* s_w, void* y,
@@ -336,13 +350,21 @@ q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* sec
                          const int8_t* q, const int32_t* wsum, const float* s_w, float* y,
                          int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes,
                          void* stream) {
+    return q8_linear_w8a8_bias(x, first, second, q, wsum, s_w, nullptr, y, M, N, K, workspace,
+                               ws_bytes, stream);
+}
+
+q8_status q8_linear_w8a8_bias(const float* x, q8_qparams first, const q8_qparams* second,
+                              const int8_t* q, const int32_t* wsum, const float* s_w,
+                              const float* bias, float* y, int64_t M, int64_t N, int64_t K,
+                              void* workspace, size_t ws_bytes, void* stream) {
     if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
     Q8_TRY(check_k(K));
     Q8_TRY(check_qparams(first));
     if (second) Q8_TRY(check_qparams(*second));
     if (M == 0) return Q8_OK;
     if (!x || !q || !wsum || !s_w || !y) return Q8_ERR_NULL;
-    if (!aligned16(x) || !aligned16(q) || !aligned16(y)) return Q8_ERR_ALIGN;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(y) || !aligned4(bias)) return Q8_ERR_ALIGN;
     const int two = second != nullptr;
     const W8A8Plan plan = plan_w8a8(M, K, two);
     if (plan.bytes > 0 && (!workspace || ws_bytes < plan.bytes)) return Q8_ERR_WORKSPACE;
@@ -359,9 +381,9 @@ q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* sec
                                            z2, xq1, xq2, st, sms)));
     if (M > kW8A8GemvMaxM && K >= kTcMinK)
         return launched(launch_w8a8_tc(xq1, xq2, first.scale, first.zero_point, two, s2, z2, q,
-                                       wsum, s_w, y, M, N, (int)K, st, sms, status));
+                                       wsum, s_w, bias, y, M, N, (int)K, st, sms, status));
     return launched(launch_w8a8_gemv_codes(xq1, xq2, first.scale, first.zero_point, two, s2, z2,
-                                           q, wsum, s_w, y, M, N, (int)K, st));
+                                           q, wsum, s_w, bias, y, M, N, (int)K, st));
 }
 
 q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* gs, int G,

@@ -42,10 +42,10 @@ __device__ __forceinline__ void qparams_from_range(float mn, float mx, float& s,
     zf = fminf(fmaxf(zf, -128.0f), 127.0f);
 }
 
-// Weight code: clamp(round(w / s), -lim, lim) with a true IEEE division.
-__device__ __forceinline__ int weight_code(float w, float s, float lim) {
+// Weight code: clamp(round(w / s), lo, hi) with a true IEEE division.
+__device__ __forceinline__ int weight_code(float w, float s, float lo, float hi) {
     float r = rintf(__fdiv_rn(w, s));
-    r = fminf(fmaxf(r, -lim), lim);
+    r = fminf(fmaxf(r, lo), hi);
     return __float2int_rn(r);
 }
 

@@ -37,8 +37,9 @@ __device__ __forceinline__ void static_codes16(const float (&v)[16], float s1, f
 }
 
 // k_quant.cu
-cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int8_t* q, float* s_w,
-                                   int32_t* wsum, cudaStream_t st);
+// full: 0 = amax/127 on +-127, 1 = max(amax/127.5, FLT_EPSILON) on [-128, 127]
+cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int full, int8_t* q,
+                                   float* s_w, int32_t* wsum, cudaStream_t st);
 cudaError_t launch_choose_qparams(const uint16_t* x, int64_t M, int K, float* s, int32_t* z,
                                   int8_t* xq, cudaStream_t st);
 cudaError_t launch_choose_qparams_shifted(const uint16_t* x, int64_t M, int K, float* s,
@@ -54,10 +55,11 @@ cudaError_t launch_quantize_weight_q4gs(const float* W, int64_t N, int K, int G,
 // k_gemv_tma.cu
 bool make_tmap_u8_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
                      int box_cols, int box_rows, CUtensorMapSwizzle swz);
-bool w8a16_tma_fits(int64_t M, int64_t K);
-cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
-                             int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,
-                             int num_sms, int* status);
+bool w8a16_tma_fits(int64_t M, int64_t K, bool bias = false);
+// bias (nullable, fp32 [N]) is added after the scale in every linear launcher below
+cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_w,
+                             const float* bias, void* y, int y_bf16, int64_t M, int64_t N, int K,
+                             cudaStream_t st, int num_sms, int* status);
 
 // k_w8a16_tc.cu
 size_t w8a16_tc_workspace_bytes(int64_t M, int64_t K, int num_sms);
@@ -70,8 +72,8 @@ cudaError_t launch_gemm_s8s8_s32_tc(const int8_t* a, const int8_t* b, int32_t* a
                                     int64_t N, int K, cudaStream_t st, int num_sms, int* status);
 cudaError_t launch_w8a8_tc(const int8_t* xq1, const int8_t* xq2, float s1, int z1, int has2,
                            float s2, int z2, const int8_t* q, const int32_t* wsum,
-                           const float* s_w, float* y, int64_t M, int64_t N, int K,
-                           cudaStream_t st, int num_sms, int* status);
+                           const float* s_w, const float* bias, float* y, int64_t M, int64_t N,
+                           int K, cudaStream_t st, int num_sms, int* status);
 
 // k_q4.cu
 cudaError_t launch_q4_gemv(const int8_t* xq, const float* s, const int32_t* z, const uint8_t* q4,
@@ -102,12 +104,12 @@ cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const floa
                               cudaStream_t st, int num_sms, int* status);
 
 // k_gemv.cu
-cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
-                              int y_bf16, int64_t M, int64_t N, int K, cudaStream_t st,
-                              int num_sms);
+cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w,
+                              const float* bias, void* y, int y_bf16, int64_t M, int64_t N, int K,
+                              cudaStream_t st, int num_sms);
 cudaError_t launch_w8a8_gemv_codes(const int8_t* xq1, const int8_t* xq2, float s1, int z1,
                                    int has2, float s2, int z2, const int8_t* q,
-                                   const int32_t* wsum, const float* s_w, float* y, int64_t M,
-                                   int64_t N, int K, cudaStream_t st);
+                                   const int32_t* wsum, const float* s_w, const float* bias,
+                                   float* y, int64_t M, int64_t N, int K, cudaStream_t st);
 
 }  // namespace q8

@@ -35,6 +35,8 @@ def lib() -> ctypes.CDLL:
         L.q8o_set_num_threads.argtypes = [ctypes.c_int]
         L.q8o_quantize_weight.restype = ctypes.c_int
         L.q8o_quantize_weight.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
+        L.q8o_quantize_weight_full128.restype = ctypes.c_int
+        L.q8o_quantize_weight_full128.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
         L.q8o_qparams_from_minmax.argtypes = [_f32, _f32, _vp, _vp]
         L.q8o_minmax.argtypes = [_vp, _i64, _vp, _vp]
         L.q8o_choose_qparams.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
@@ -103,14 +105,19 @@ def set_num_threads(n: int) -> None:
     lib().q8o_set_num_threads(int(n))
 
 
-def quantize_weight(W: np.ndarray):
-    """Per-row symmetric int8 codes -> (q int8 [N,K], s fp32 [N], wsum int32 [N])."""
+def quantize_weight(W: np.ndarray, grid: str = "sym127"):
+    """Per-row symmetric int8 codes -> (q int8 [N,K], s fp32 [N], wsum int32 [N]).
+    grid "sym127": [ROCm-INT8] quantize_weight (amax/127, codes +-127);
+    grid "full128": [SmolVLM-Q8] weight_int8 (observer scale amax/127.5, codes -128..127)."""
+    if grid not in ("sym127", "full128"):
+        raise ValueError("grid must be 'sym127' or 'full128'")
     W = _c(W, np.float32)
     N, K = W.shape
     q = np.empty((N, K), np.int8)
     s = np.empty(N, np.float32)
     ws = np.empty(N, np.int32)
-    if lib().q8o_quantize_weight(_p(W), N, K, _p(q), _p(s), _p(ws)) != 0:
+    fn = lib().q8o_quantize_weight if grid == "sym127" else lib().q8o_quantize_weight_full128
+    if fn(_p(W), N, K, _p(q), _p(s), _p(ws)) != 0:
         raise OverflowError("a row's code sum does not fit int32")
     return q, s, ws
 
@@ -156,8 +163,20 @@ def static_quant(x: np.ndarray, first, second=None):
     return xq1, xq2
 
 
-def linear_w8a16(x_bf16, q, s_w, rows=None):
-    """fp64 y [R,N] and magnitude sums [R,N] for the listed rows (all if None)."""
+def _add_bias(y, a, bias):
+    """[ROCm-INT8] Int8Linear / [SmolVLM-Q8] Q8Linear: F.linear adds bias[n] to every row
+    (once: the residual pass of the two-pass form is a bias-free linear)."""
+    if bias is None:
+        return y, a
+    b = _c(bias, np.float32).astype(np.float64)
+    if b.shape != (y.shape[1],):
+        raise ValueError("bias must be [N]")
+    return y + b[None, :], a + np.abs(b)[None, :]
+
+
+def linear_w8a16(x_bf16, q, s_w, rows=None, bias=None):
+    """fp64 y [R,N] and magnitude sums [R,N] for the listed rows (all if None); with a
+    bias [N], y + bias."""
     x = _c(x_bf16, np.uint16)
     q = _c(q, np.int8)
     s_w = _c(s_w, np.float32)
@@ -167,11 +186,12 @@ def linear_w8a16(x_bf16, q, s_w, rows=None):
     y = np.empty((R, N), np.float64)
     a = np.empty((R, N), np.float64)
     lib().q8o_linear_w8a16(_p(x), _p(q), _p(s_w), M, N, K, _p(r), R, _p(y), _p(a))
-    return y, a
+    return _add_bias(y, a, bias)
 
 
-def linear_w8a8(x, first, q, s_w, second=None, rows=None):
-    """fp64 y, magnitude sums, and raw int32 dot products (acc1, acc2|None)."""
+def linear_w8a8(x, first, q, s_w, second=None, rows=None, bias=None):
+    """fp64 y, magnitude sums, and raw int32 dot products (acc1, acc2|None); with a bias
+    [N], the first pass's output carries it (y + bias)."""
     x = _c(x, np.float32)
     q = _c(q, np.int8)
     s_w = _c(s_w, np.float32)
@@ -186,6 +206,7 @@ def linear_w8a8(x, first, q, s_w, second=None, rows=None):
     lib().q8o_linear_w8a8(_p(x), float(first[0]), int(first[1]), int(second is not None),
                           float(s2), int(z2), _p(q), _p(s_w), M, N, K, _p(r), R,
                           _p(y), _p(a), _p(acc1), _p(acc2))
+    y, a = _add_bias(y, a, bias)
     return y, a, acc1, acc2
 
 

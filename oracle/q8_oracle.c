@@ -113,6 +113,51 @@ int q8o_quantize_weight(const float* W, int64_t N, int64_t K,
     return bad;
 }
 
+/* ------------------------------------- weight quantization, observer grid (f1)
+ * [SmolVLM-Q8] weight_int8: the codes span the full int8 range [-128, 127] and the
+ * per-channel scale comes from torchao's per-channel symmetric min/max observer, whose
+ * rule the page states as amax / 127.5.  Written out per row n (the observer's steps,
+ * the pages' order; fp32 throughout):
+ *   lo = min(min_k w, 0), hi = max(max_k w, 0)         (range widened to contain 0)
+ *   amax = max(-lo, hi)
+ *   scale = amax / ((127 - (-128)) / 2) = amax / 127.5  (fp32 IEEE division)
+ *   scale = max(scale, FLT_EPSILON)                     (the observer's eps floor)
+ *   q = clamp(round(w / scale), -128, 127)              (true division, ties to even)
+ * An all-zero row therefore gets scale FLT_EPSILON and all codes 0.
+ * Returns 0, or 1 if a code sum does not fit int32.
+ */
+int q8o_quantize_weight_full128(const float* W, int64_t N, int64_t K,
+                                int8_t* q, float* s, int32_t* wsum) {
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(|:bad)
+    for (int64_t n = 0; n < N; ++n) {
+        const float* w = W + n * K;
+        float lo = 0.0f, hi = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            if (w[k] < lo) lo = w[k];
+            if (w[k] > hi) hi = w[k];
+        }
+        const float amax = (-lo > hi) ? -lo : hi;
+        const float half_range = (127.0f - (-128.0f)) / 2.0f;    /* 127.5, exact */
+        float scale = amax / half_range;
+        if (scale < FLT_EPSILON) scale = FLT_EPSILON;
+        int64_t sum = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            float r = nearbyintf(w[k] / scale);
+            r = clampf(r, -128.0f, 127.0f);
+            const int code = (int)r;
+            q[n * K + k] = (int8_t)code;
+            sum += code;
+        }
+        s[n] = scale;
+        if (wsum) {
+            if (sum > INT32_MAX || sum < INT32_MIN) bad = 1;
+            wsum[n] = (int32_t)sum;
+        }
+    }
+    return bad;
+}
+
 /* ------------------------------------------ affine activation qparams (a2, R5)
  * The pages use torchao's per-tensor MinMaxObserver ([SmolVLM-Q8] act_observer,
  * qparams) and per-row choose_qparams_affine ([ET-21229]) without printing the

@@ -17,6 +17,8 @@ void q8o_set_num_threads(int n);
 
 int  q8o_quantize_weight(const float* W, int64_t N, int64_t K,
                          int8_t* q, float* s, int32_t* wsum);
+int  q8o_quantize_weight_full128(const float* W, int64_t N, int64_t K,
+                                 int8_t* q, float* s, int32_t* wsum);
 void q8o_qparams_from_minmax(float mn, float mx, float* s, int32_t* z);
 void q8o_minmax(const float* x, int64_t n, float* mn, float* mx);
 void q8o_choose_qparams(const uint16_t* x, int64_t M, int64_t K,

@@ -95,6 +95,23 @@ def test_argument_validation_before_device(L):
                             None) == q8.Q8_ERR_WORKSPACE
     assert L.q8_quantize_weight_q4gs(good, 4, 64, 48, good, good, None) == q8.Q8_ERR_ARG
     assert L.q8_quantize_weight_q4gs(good, 4, 96, 64, good, good, None) == q8.Q8_ERR_SHAPE
+    # weight grid option and bias entry points
+    assert L.q8_quantize_weight_grid(good, 4, 64, 2, good, good, None, None) == q8.Q8_ERR_ARG
+    assert L.q8_quantize_weight_grid(good, 4, 60, q8.Q8_GRID_FULL128, good, good, None,
+                                     None) == q8.Q8_ERR_SHAPE
+    assert L.q8_quantize_weight_grid(odd, 4, 64, q8.Q8_GRID_FULL128, good, good, None,
+                                     None) == q8.Q8_ERR_ALIGN
+    odd4 = _p(0x10002)                                   # 2-byte aligned: not a float pointer
+    assert L.q8_linear_w8a16_bias(good, good, good, odd4, good, q8.Q8_F32, 1, 16, 64,
+                                  None) == q8.Q8_ERR_ALIGN
+    assert L.q8_linear_w8a16_bias(good, good, good, good, good, 7, 1, 16, 64,
+                                  None) == q8.Q8_ERR_ARG
+    assert L.q8_linear_w8a16_bias(good, good, good, good, good, q8.Q8_F32, 0, 16, 64,
+                                  None) == q8.Q8_OK
+    assert L.q8_linear_w8a8_bias(good, qp, None, good, good, good, odd4, good, 1, 16, 64, good,
+                                 1024, None) == q8.Q8_ERR_ALIGN
+    assert L.q8_linear_w8a8_bias(good, bad_qp, None, good, good, good, good, good, 1, 16, 64,
+                                 good, 1024, None) == q8.Q8_ERR_ARG
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU failure mode")

@@ -47,6 +47,18 @@ MUTANTS = [
      "int64_t p = ((int64_t)xr[k]) * q4_code(wr, k);", ["test_dq8ca_q4gsw_reductions"]),
     ("bf16 rounding truncates", "double r = nearbyint(ldexp(m, 8));",
      "double r = trunc(ldexp(m, 8));", ["test_round_bf16"]),
+    ("full grid clamps at -127",
+     "r = clampf(r, -128.0f, 127.0f);\n            const int code = (int)r;",
+     "r = clampf(r, -127.0f, 127.0f);\n            const int code = (int)r;",
+     ["test_golden_weight_rows_full128"]),
+    ("full grid scale amax/127", "float scale = amax / half_range;",
+     "float scale = amax / 127.0f;", ["test_golden_weight_rows_full128"]),
+    ("full grid eps floor only for a zero scale",
+     "float scale = amax / half_range;\n        if (scale < FLT_EPSILON) scale = FLT_EPSILON;",
+     "float scale = amax / half_range;\n        if (scale == 0.0f) scale = FLT_EPSILON;",
+     ["test_golden_weight_rows_full128"]),
+    ("full grid ignores negative extremes", "const float amax = (-lo > hi) ? -lo : hi;",
+     "const float amax = hi;", ["test_golden_weight_rows_full128"]),
 ]
 
 

@@ -404,3 +404,97 @@ def test_round_bf16():
     exp = [rn_bf16(Fraction(c)) for c in cases]
     assert [bf16_bits_to_fraction(g) for g in got] == exp
     assert got[3] == 0x3F81                          # just above the tie: rounds up
+
+
+# ------------------------------------------------- full int8 weight grid (f1)
+
+
+def _weight_codes_full128_exact(row):
+    """weight_int8 (SmolVLM q8 page) in exact rational arithmetic with fp32 rounding at
+    each step: observer scale max(amax / 127.5, 2^-23), codes clamp(rne(w / s), -128, 127)."""
+    vals = [f32(v) for v in row]
+    amax = max([Fraction(0)] + [abs(v) for v in vals])
+    s = rn32(amax / Fraction(255, 2)) if amax else Fraction(0)
+    eps = Fraction(2) ** -23
+    if s < eps:
+        s = eps
+    codes = [max(-128, min(127, rne_int(rn32(v / s)))) for v in vals]
+    return s, codes
+
+
+def test_golden_weight_rows_full128():
+    """weight_int8's observer grid (SmolVLM q8 page) on hand-worked rows."""
+    rows = _parse("weight_int8_full128_rows.txt")
+    W = np.array([[float(v) for v in r[0]] for r in rows], np.float32)
+    q, s, ws = oracle.quantize_weight(W, grid="full128")
+    for i, r in enumerate(rows):
+        assert q[i].tolist() == [int(v) for v in r[2]], f"row {i} codes"
+        assert ws[i] == int(r[3][0]), f"row {i} code sum"
+        assert s[i] == np.float32(float(r[1][0])), f"row {i} scale"
+
+
+def test_quantize_weight_full128_exact_rational():
+    W = wl.weight(12, 37, seed=31).numpy()
+    W[2] = 0.0
+    W[4] *= 1e-8                                     # below the eps floor
+    W[6, 3] = -np.abs(W[6]).max() * 1.5              # a dominant negative element
+    for n in range(W.shape[0]):
+        Wn = W[n:n + 1]
+        q, s, ws = oracle.quantize_weight(Wn, grid="full128")
+        s_ex, codes = _weight_codes_full128_exact(Wn[0])
+        assert Fraction(float(s[0])) == s_ex, f"row {n} scale"
+        assert q[0].tolist() == codes, f"row {n} codes"
+        assert int(ws[0]) == sum(codes)
+
+
+def test_full128_nearest_grid_and_asymmetric_clamp():
+    """|q*s - w| <= s/2 on [-128, 127], up to the rounding of the fp32 quotient w/s (at most
+    2^-17 for |w/s| <= 128); the positive extreme never passes 127, and over many rows the
+    negative extreme reaches -128 (when amax/127.5 rounds down in fp32) as well as -127
+    (when it rounds up)."""
+    W = wl.weight(512, 64, seed=32).numpy()
+    W[:, 0] = -np.abs(W).max(axis=1) * 1.01          # each row's extreme is negative
+    q, s, _ = oracle.quantize_weight(W, grid="full128")
+    err = np.abs(q.astype(np.float64) * s[:, None].astype(np.float64) - W.astype(np.float64))
+    assert np.all(err <= s[:, None] * (0.5 + 2.0 ** -17))
+    assert q.max() <= 127 and q.min() >= -128
+    assert (q[:, 0] == -128).any() and (q[:, 0] == -127).any()
+    qp, _, _ = oracle.quantize_weight(-W, grid="full128")
+    assert np.all(qp[:, 0] == 127)                   # positive extremes clamp at 127
+
+
+# ------------------------------------------------------------------ bias (f1)
+
+
+def test_w8a16_bias_closed_form():
+    """Int8Linear.forward with a bias (ROCm page: F.linear(x, w, bias)): with q = I and
+    s_w = 1 the linear is the identity, so y = x + bias exactly."""
+    K = 32
+    q = np.eye(K, dtype=np.int8)
+    sw = np.ones(K, np.float32)
+    xt = wl.normal_bf16((5, K), 1.0, seed=33)
+    b = wl.normal((K,), 3.0, seed=34).numpy()
+    y, a = oracle.linear_w8a16(wl.bf16_bits(xt), q, sw, bias=b)
+    x64 = xt.float().numpy().astype(np.float64)
+    assert np.array_equal(y, x64 + b.astype(np.float64)[None, :])
+    y0, a0 = oracle.linear_w8a16(wl.bf16_bits(xt), q, sw)
+    assert np.array_equal(a - a0, np.broadcast_to(np.abs(b).astype(np.float64), a.shape))
+
+
+def test_w8a8_bias_first_pass_only():
+    """Q8Linear.forward (SmolVLM q8 page) with a bias: linear(dq(q(x)), dq(W), bias) +
+    linear(dq(q(r)), dq(W)) -- the bias enters once, also in the two-pass form."""
+    x, calib = wl.w8a8_inputs(6, K=64)
+    x = x.numpy()
+    s1, z1 = oracle.qparams_from_minmax(*oracle.minmax(calib.numpy()))
+    s2 = float(np.float32(s1) / np.float32(255.0))
+    q, sw, _ = oracle.quantize_weight(wl.weight(24, 64, seed=35).numpy())
+    b = wl.normal((24,), 2.0, seed=36).numpy()
+    dqw = q.astype(np.float64) * sw.astype(np.float64)[:, None]
+    for second in (None, (s2, 0)):
+        y, a, _, _ = oracle.linear_w8a8(x, (s1, z1), q, sw, second=second, bias=b)
+        xq1, xq2 = oracle.static_quant(x, (s1, z1), second)
+        ref = ((xq1.astype(np.float64) - z1) * s1) @ dqw.T + b.astype(np.float64)[None, :]
+        if second is not None:
+            ref += (xq2.astype(np.float64) * s2) @ dqw.T
+        assert np.all(np.abs(y - ref) <= 1e-12 * a)
