@@ -558,9 +558,9 @@ def bench_q4(dev, peaks, reps=5):
 
 
 def bench_quantizers(dev, peaks, reps=5):
-    """The quantizers as HBM streams: weight codes (fp32 32000x4096 in), per-row activation
-    qparams + codes (bf16 4096x4096), static activation codes with the residual pass
-    (fp32 4096x4096)."""
+    """The quantizers as HBM streams: weight codes on both grids (fp32 32000x4096 in),
+    per-row activation qparams + codes (bf16 4096x4096), static activation codes with the
+    residual pass, and the residual calibration observer (fp32 4096x4096)."""
     import int8_quantized_linear_q8_b200 as q8
 
     g = torch.Generator(device=dev)
@@ -593,6 +593,11 @@ def bench_quantizers(dev, peaks, reps=5):
                      reps)
     b = 4096 * 4096 * 6
     out.append({"op": "quantize_static_two_pass", "shape": [4096, 4096], "us": round(us, 1),
+                "GBps": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / peaks["hbm_gbs"], 4)})
+    mm = torch.empty(2, device=dev)
+    us = _graph_time(lambda: q8.q8_observe_residual_minmax(xf, (0.05, 3), mm, reset=True), reps)
+    b = 4096 * 4096 * 4
+    out.append({"op": "observe_residual_minmax", "shape": [4096, 4096], "us": round(us, 1),
                 "GBps": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / peaks["hbm_gbs"], 4)})
     return out
 

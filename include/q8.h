@@ -149,6 +149,16 @@ q8_status q8_quantize_static(const float* x, int64_t M, int64_t K, q8_qparams fi
 q8_status q8_observe_minmax(const float* x, int64_t n, float* minmax, int reset,
                             void* stream);
 
+/* Residual observer of the two-pass calibration ([SmolVLM-Q8] calibrate: the second
+ * calibration run observes each linear's first-pass rounding error, x - fake_quant(x, first)).
+ * Same as q8_observe_minmax on the values
+ *     r = x - (xq1 - z1) * s1,   xq1 = clamp(round(x * (1/s1)) + z1, -128, 127)
+ * computed with exactly the fp32 steps of q8_quantize_static (so the statistics describe
+ * the residual the second pass will quantize).  q8_qparams_from_minmax on the result gives
+ * the second pass's (s2, z2).  `first` must satisfy the q8_qparams rules (Q8_ERR_ARG). */
+q8_status q8_observe_residual_minmax(const float* x, int64_t n, q8_qparams first, float* minmax,
+                                     int reset, void* stream);
+
 /* Host.  Per-tensor affine qparams from an observed range (same formula as
  * q8_choose_qparams): out->scale = max((max(mx,0) - min(mn,0)) / 255, FLT_EPSILON),
  * out->zero_point = clamp(-128 - round(min(mn,0) / scale), -128, 127).

@@ -36,6 +36,7 @@ SYMBOLS = (
     "q8_workspace_bytes", "q8_gemm_s8s8_s32", "q8_last_device_status",
     "q8_linear_w8a8_noalloc", "q8_selftest_bounded_wait", "q8_linear_w8a16_planes",
     "q8_quantize_weight_grid", "q8_linear_w8a16_bias", "q8_linear_w8a8_bias",
+    "q8_observe_residual_minmax",
 )
 # Built-in scratch of q8_linear_w8a8_noalloc (bytes).
 Q8_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -79,6 +80,8 @@ def _lib() -> ctypes.CDLL:
                                      _vp, _vp, _vp]
     L.q8_observe_minmax.restype = st
     L.q8_observe_minmax.argtypes = [_vp, _i64, _vp, st, _vp]
+    L.q8_observe_residual_minmax.restype = st
+    L.q8_observe_residual_minmax.argtypes = [_vp, _i64, q8_qparams, _vp, st, _vp]
     L.q8_qparams_from_minmax.restype = st
     L.q8_qparams_from_minmax.argtypes = [ctypes.c_float, ctypes.c_float,
                                          ctypes.POINTER(q8_qparams)]
@@ -225,6 +228,17 @@ def q8_observe_minmax(x: torch.Tensor, minmax: torch.Tensor, reset: bool = False
     _need(minmax, "minmax", torch.float32, (2,))
     _check(_lib().q8_observe_minmax(_ptr(x), x.numel(), _ptr(minmax), int(bool(reset)),
                                     _stream(stream)), "q8_observe_minmax")
+    return minmax
+
+
+def q8_observe_residual_minmax(x: torch.Tensor, first, minmax: torch.Tensor,
+                               reset: bool = False, stream=None) -> torch.Tensor:
+    """Lower/raise {min, max} by the first-pass rounding errors x - fake_quant(x, first)."""
+    _need(x, "x", torch.float32, tuple(x.shape))
+    _need(minmax, "minmax", torch.float32, (2,))
+    _check(_lib().q8_observe_residual_minmax(_ptr(x), x.numel(), _qp(first), _ptr(minmax),
+                                             int(bool(reset)), _stream(stream)),
+           "q8_observe_residual_minmax")
     return minmax
 
 

@@ -270,21 +270,40 @@ __global__ void k_minmax_reset(float* mm) {
     mm[1] = __int_as_float(0xff800000);   // -inf
 }
 
+// RES = false: min / max of the values themselves (act_observer).
+// RES = true:  min / max of the first-pass rounding error r = x - fake_quant(x, s1, z1),
+//              the transform the second calibration run observes ([SmolVLM-Q8] calibrate):
+//              r = x - (code - z1) * s1 with code = clamp(round(x * (1/s1)) + z1, -128, 127),
+//              every step rounded to fp32 exactly as the two-pass quantizer computes it.
+template <bool RES>
+__device__ __forceinline__ float observed(float v, float s1, float inv1, float z1f) {
+    if (!RES) return v;
+    const float d1 = __fmul_rn(__fsub_rn((float)act_code(v, inv1, z1f), z1f), s1);
+    return __fsub_rn(v, d1);
+}
+
+template <bool RES>
 __global__ __launch_bounds__(256) void k_observe_minmax(const float* __restrict__ x, int64_t n,
-                                                        float* mm) {
+                                                        float s1, float z1f, float* mm) {
     __shared__ float red[8];
+    const float inv1 = RES ? __fdiv_rn(1.0f, s1) : 0.0f;
     float lo = FLT_MAX, hi = -FLT_MAX;
     const int64_t n4 = n >> 2;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
          i += (int64_t)gridDim.x * blockDim.x) {
         float4 v = ldg_f4(x + 4 * i);
+        v.x = observed<RES>(v.x, s1, inv1, z1f);
+        v.y = observed<RES>(v.y, s1, inv1, z1f);
+        v.z = observed<RES>(v.z, s1, inv1, z1f);
+        v.w = observed<RES>(v.w, s1, inv1, z1f);
         lo = fminf(lo, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
         hi = fmaxf(hi, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
     }
     for (int64_t i = 4 * n4 + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
-        lo = fminf(lo, x[i]);
-        hi = fmaxf(hi, x[i]);
+        const float v = observed<RES>(x[i], s1, inv1, z1f);
+        lo = fminf(lo, v);
+        hi = fmaxf(hi, v);
     }
     lo = block_min<256>(lo, red);
     hi = block_max<256>(hi, red);
@@ -379,15 +398,18 @@ cudaError_t launch_quantize_static(const float* x, int64_t M, int K, float s1, i
     return cudaGetLastError();
 }
 
-cudaError_t launch_observe_minmax(const float* x, int64_t n, float* mm, int reset,
-                                  cudaStream_t st, int num_sms) {
+cudaError_t launch_observe_minmax(const float* x, int64_t n, float* mm, int reset, int residual,
+                                  float s1, int z1, cudaStream_t st, int num_sms) {
     if (reset) k_minmax_reset<<<1, 1, 0, st>>>(mm);
     if (n > 0) {
         int64_t blocks = (n / 4 + 255) / 256;
         const int64_t cap = (int64_t)num_sms * 4;
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
-        k_observe_minmax<<<(unsigned)blocks, 256, 0, st>>>(x, n, mm);
+        if (residual)
+            k_observe_minmax<true><<<(unsigned)blocks, 256, 0, st>>>(x, n, s1, (float)z1, mm);
+        else
+            k_observe_minmax<false><<<(unsigned)blocks, 256, 0, st>>>(x, n, 1.0f, 0.0f, mm);
     }
     return cudaGetLastError();
 }

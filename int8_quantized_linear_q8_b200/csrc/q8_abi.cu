@@ -249,7 +249,21 @@ q8_status q8_observe_minmax(const float* x, int64_t n, float* minmax, int reset,
     if (x && !aligned16(x)) return Q8_ERR_ALIGN;
     int sms = 0;
     Q8_TRY(current_device(sms));
-    return launched(launch_observe_minmax(x, n, minmax, reset, (cudaStream_t)stream, sms));
+    return launched(
+        launch_observe_minmax(x, n, minmax, reset, 0, 1.0f, 0, (cudaStream_t)stream, sms));
+}
+
+q8_status q8_observe_residual_minmax(const float* x, int64_t n, q8_qparams first, float* minmax,
+                                     int reset, void* stream) {
+    if (n < 0) return Q8_ERR_SHAPE;
+    Q8_TRY(check_qparams(first));
+    if (!minmax || (n > 0 && !x)) return Q8_ERR_NULL;
+    if (n == 0 && !reset) return Q8_OK;
+    if (x && !aligned16(x)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_observe_minmax(x, n, minmax, reset, 1, first.scale, first.zero_point,
+                                          (cudaStream_t)stream, sms));
 }
 
 q8_status q8_qparams_from_minmax(float mn, float mx, q8_qparams* out) {

@@ -47,8 +47,9 @@ cudaError_t launch_choose_qparams_shifted(const uint16_t* x, int64_t M, int K, f
 cudaError_t launch_quantize_static(const float* x, int64_t M, int K, float s1, int z1, int has2,
                                    float s2, int z2, int8_t* xq1, int8_t* xq2, cudaStream_t st,
                                    int num_sms);
-cudaError_t launch_observe_minmax(const float* x, int64_t n, float* mm, int reset,
-                                  cudaStream_t st, int num_sms);
+// residual != 0: observe x - fake_quant(x, s1, z1) instead of x
+cudaError_t launch_observe_minmax(const float* x, int64_t n, float* mm, int reset, int residual,
+                                  float s1, int z1, cudaStream_t st, int num_sms);
 cudaError_t launch_quantize_weight_q4gs(const float* W, int64_t N, int K, int G, uint8_t* q4,
                                         float* gs, cudaStream_t st);
 

@@ -39,6 +39,7 @@ def lib() -> ctypes.CDLL:
         L.q8o_quantize_weight_full128.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
         L.q8o_qparams_from_minmax.argtypes = [_f32, _f32, _vp, _vp]
         L.q8o_minmax.argtypes = [_vp, _i64, _vp, _vp]
+        L.q8o_residual_minmax.argtypes = [_vp, _i64, _f32, _i32, _vp, _vp]
         L.q8o_choose_qparams.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
         L.q8o_static_quant.argtypes = [_vp, _i64, _i64, _f32, _i32, _vp, ctypes.c_int,
                                        _f32, _i32, _vp]
@@ -137,6 +138,18 @@ def minmax(x: np.ndarray):
     lo = np.empty(1, np.float32)
     hi = np.empty(1, np.float32)
     lib().q8o_minmax(_p(x), x.size, _p(lo), _p(hi))
+    return float(lo[0]), float(hi[0])
+
+
+def residual_minmax(x: np.ndarray, first):
+    """Min and max of the first-pass rounding errors x - fake_quant(x, s1, z1) (the second
+    calibration run's observer input)."""
+    x = _c(x, np.float32).reshape(-1)
+    if x.size == 0:
+        raise ValueError("empty tensor")
+    lo = np.empty(1, np.float32)
+    hi = np.empty(1, np.float32)
+    lib().q8o_residual_minmax(_p(x), x.size, float(first[0]), int(first[1]), _p(lo), _p(hi))
     return float(lo[0]), float(hi[0])
 
 

@@ -253,6 +253,28 @@ void q8o_static_quant(const float* x, int64_t M, int64_t K, float s1, int32_t z1
                          has2 ? xq2 + m * K : NULL);
 }
 
+/* ------------------------------------------- residual calibration observer (f2)
+ * [SmolVLM-Q8] calibrate: with two passes, a second calibration run feeds each linear's
+ * observer with x - fake_quant(x, *first), and the observer keeps the min and max of
+ * everything it saw.  fake_quant as the page defines it, in fp32 one step at a time:
+ *     fake_quant(x, s, z) = (clamp(round(x * (1/s)) + z, -128, 127) - z) * s
+ * with 1/s the fp32 reciprocal (the reading the activation codes above use).
+ * Writes the min and max of the n residuals (n >= 1). */
+void q8o_residual_minmax(const float* x, int64_t n, float s1, int32_t z1,
+                         float* mn, float* mx) {
+    const float inv = 1.0f / s1;
+    float lo = 0.0f, hi = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float q = clampf(nearbyintf(x[i] * inv) + (float)z1, -128.0f, 127.0f);
+        float fq = (q - (float)z1) * s1;
+        float r = x[i] - fq;
+        if (i == 0 || r < lo) lo = r;
+        if (i == 0 || r > hi) hi = r;
+    }
+    *mn = lo;
+    *mx = hi;
+}
+
 /* ------------------------------------------------------------ W8A16 (a4)
  * [tiny-llm] module docstring (the factorisation identity) and Int8Linear.forward:
  *     y[m,n] = s_w[n] * sum_k x[m,k] * q[n,k]

@@ -21,6 +21,8 @@ int  q8o_quantize_weight_full128(const float* W, int64_t N, int64_t K,
                                  int8_t* q, float* s, int32_t* wsum);
 void q8o_qparams_from_minmax(float mn, float mx, float* s, int32_t* z);
 void q8o_minmax(const float* x, int64_t n, float* mn, float* mx);
+void q8o_residual_minmax(const float* x, int64_t n, float s1, int32_t z1,
+                         float* mn, float* mx);
 void q8o_choose_qparams(const uint16_t* x, int64_t M, int64_t K,
                         float* s, int32_t* z, int8_t* xq);
 void q8o_static_quant(const float* x, int64_t M, int64_t K, float s1, int32_t z1,

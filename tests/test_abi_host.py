@@ -112,6 +112,12 @@ def test_argument_validation_before_device(L):
                                  1024, None) == q8.Q8_ERR_ALIGN
     assert L.q8_linear_w8a8_bias(good, bad_qp, None, good, good, good, good, good, 1, 16, 64,
                                  good, 1024, None) == q8.Q8_ERR_ARG
+    mmp = _p(0x10000)
+    assert L.q8_observe_residual_minmax(good, 64, bad_qp, mmp, 1, None) == q8.Q8_ERR_ARG
+    assert L.q8_observe_residual_minmax(good, -1, qp, mmp, 1, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_observe_residual_minmax(odd, 64, qp, mmp, 1, None) == q8.Q8_ERR_ALIGN
+    assert L.q8_observe_residual_minmax(None, 64, qp, mmp, 1, None) == q8.Q8_ERR_NULL
+    assert L.q8_observe_residual_minmax(good, 0, qp, mmp, 0, None) == q8.Q8_OK
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU failure mode")

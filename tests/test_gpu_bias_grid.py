@@ -157,3 +157,46 @@ def test_bias_none_is_bit_identical_to_plain_call():
     yz = q8.q8_linear_w8a16(x, q, s, out_dtype=torch.float32,
                             bias=torch.zeros(N, device=DEV))
     assert torch.equal(y0, yz)
+
+
+# ------------------------------------------- residual calibration observer (f2)
+
+
+@pytest.mark.parametrize("chunks", [[1], [4096 * 960], [1000, 3, 4097, 250000], [960] * 9])
+def test_observe_residual_minmax_bit_exact(chunks):
+    """The second calibration run's observer (x - fake_quant(x, first)) over a stream of
+    chunks: reset on the first, then accumulate; min and max bit-exact against the oracle."""
+    first = (float(np.float32(0.0625)), -3)
+    xs = [wl.normal((n,), 2.0, seed=750 + i).numpy() for i, n in enumerate(chunks)]
+    xs[0][0] = 1e4                                      # clamped at 127
+    xs[-1][-1] = -1e4                                   # clamped at -128
+    mm = torch.empty(2, device=DEV)
+    for i, x in enumerate(xs):
+        q8.q8_observe_residual_minmax(torch.from_numpy(x).to(DEV), first, mm, reset=(i == 0))
+    got = tuple(mm.cpu().tolist())
+    assert got == oracle.residual_minmax(np.concatenate(xs), first)
+
+
+def test_two_pass_calibration_chain():
+    """calibrate with two passes (SmolVLM q8 page) end to end on the GPU: observe the
+    calibration draw -> (s1, z1); observe its first-pass errors -> (s2, z2); both equal the
+    oracle's; then the two-pass W8A8 linear with those qparams matches the oracle."""
+    K, N, M = wl.W8A8_K, 2560, 37
+    x, calib = wl.w8a8_inputs(M, K=K)
+    mm = torch.empty(2, device=DEV)
+    q8.q8_observe_minmax(calib.to(DEV), mm, reset=True)
+    first = q8.q8_qparams_from_minmax(*mm.cpu().tolist())
+    assert first == oracle.qparams_from_minmax(*oracle.minmax(calib.numpy()))
+    q8.q8_observe_residual_minmax(calib.to(DEV), first, mm, reset=True)
+    rmin, rmax = mm.cpu().tolist()
+    assert (rmin, rmax) == oracle.residual_minmax(calib.numpy(), first)
+    second = q8.q8_qparams_from_minmax(rmin, rmax)
+    assert second == oracle.qparams_from_minmax(rmin, rmax)
+    W = wl.weight(N, K, seed=760)
+    q, s, ws = q8.q8_quantize_weight(W.to(DEV))
+    for xm in (x, calib[:2048]):
+        y = q8.q8_linear_w8a8(xm.to(DEV), first, q, ws, s, second=second)
+        torch.cuda.synchronize()
+        rq, rs, _ = oracle.quantize_weight(W.numpy())
+        y64, absum, _, _ = oracle.linear_w8a8(xm.numpy(), first, rq, rs, second=second)
+        check_f32(y.cpu().numpy(), y64, absum, f"calibrated two-pass M={xm.shape[0]}")

@@ -57,6 +57,13 @@ MUTANTS = [
      "float scale = amax / half_range;\n        if (scale < FLT_EPSILON) scale = FLT_EPSILON;",
      "float scale = amax / half_range;\n        if (scale == 0.0f) scale = FLT_EPSILON;",
      ["test_golden_weight_rows_full128"]),
+    ("residual observer without the clamp",
+     "float q = clampf(nearbyintf(x[i] * inv) + (float)z1, -128.0f, 127.0f);",
+     "float q = nearbyintf(x[i] * inv) + (float)z1;", ["test_golden_residual_observer_rows"]),
+    ("residual observer sign", "float r = x[i] - fq;", "float r = fq - x[i];",
+     ["test_golden_residual_observer_rows"]),
+    ("residual observer drops the zero point", "float fq = (q - (float)z1) * s1;",
+     "float fq = q * s1;", ["test_golden_residual_observer_rows"]),
     ("full grid ignores negative extremes", "const float amax = (-lo > hi) ? -lo : hi;",
      "const float amax = hi;", ["test_golden_weight_rows_full128"]),
 ]

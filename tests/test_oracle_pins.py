@@ -498,3 +498,45 @@ def test_w8a8_bias_first_pass_only():
         if second is not None:
             ref += (xq2.astype(np.float64) * s2) @ dqw.T
         assert np.all(np.abs(y - ref) <= 1e-12 * a)
+
+
+# ------------------------------------------- residual calibration observer (f2)
+
+
+def test_golden_residual_observer_rows():
+    """calibrate's second run (SmolVLM q8 page) on hand-worked rows."""
+    for r in _parse("residual_observer_rows.txt"):
+        s1, z1 = float(r[0][0]), int(r[0][1])
+        x = np.array([float(v) for v in r[1]], np.float32)
+        assert oracle.residual_minmax(x, (s1, z1)) == (float(r[2][0]), float(r[2][1]))
+
+
+def _residual_exact(x_vals, s1, z1):
+    inv = rn32(1 / s1)
+    out = []
+    for v in x_vals:
+        c = max(-128, min(127, rne_int(rn32(v * inv)) + z1))
+        out.append(rn32(v - rn32((c - z1) * s1)))
+    return out
+
+
+def test_residual_observer_exact_rational():
+    x, calib = wl.w8a8_inputs(3, K=64)
+    x = x.numpy().reshape(-1)
+    x[5] = 1e4                                       # clamped above
+    x[9] = -1e4                                      # clamped below
+    for s1, z1 in [(0.05, 3), (float(np.float32(0.0371)), -17), (1.0 / 3.0, 0)]:
+        s1 = float(np.float32(s1))
+        r = _residual_exact([f32(v) for v in x], f32(s1), z1)
+        assert oracle.residual_minmax(x, (s1, z1)) == (float(min(r)), float(max(r)))
+
+
+def test_residual_observer_half_step_bound():
+    """Inside the clamp range the first-pass error is at most half a step (s1/2, up to the
+    fp32 rounding of x * (1/s1)); values on the grid leave no residual."""
+    s1, z1 = 0.02, 7
+    x = wl.normal((4096,), 0.5, seed=37).numpy()      # |x| well inside (-128-7..127-7)*s1
+    lo, hi = oracle.residual_minmax(x, (s1, z1))
+    assert -s1 * (0.5 + 2.0 ** -16) <= lo <= 0.0 <= hi <= s1 * (0.5 + 2.0 ** -16)
+    grid = (np.arange(-100, 100, dtype=np.float32) * np.float32(0.25)).astype(np.float32)
+    assert oracle.residual_minmax(grid, (0.25, 0)) == (0.0, 0.0)
