@@ -50,6 +50,12 @@ def lib() -> ctypes.CDLL:
         L.q8o_linear_dq8ca_q4gsw.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_int,
                                              _i64, _i64, _i64, _vp, _i64, _vp, _vp]
         L.q8o_gemm_s8s8_s32.argtypes = [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp]
+        L.q8o_gram_rows.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp]
+        L.q8o_gptq_hinv.restype = ctypes.c_int
+        L.q8o_gptq_hinv.argtypes = [_vp, _i64, ctypes.c_double, _vp, _vp]
+        L.q8o_gptq_int8.restype = ctypes.c_int
+        L.q8o_gptq_int8.argtypes = [_vp, _vp, _i64, _i64, ctypes.c_double, _i64, _vp, _i64,
+                                    _vp, _vp, _vp]
         L.q8o_round_bf16.restype = ctypes.c_uint16
         L.q8o_round_bf16.argtypes = [ctypes.c_double]
         L.q8o_round_bf16_array.argtypes = [_vp, _i64, _vp]
@@ -261,6 +267,53 @@ def gemm_s8s8_s32(a, b, rows=None):
     acc = np.empty((R, N), np.int32)
     lib().q8o_gemm_s8s8_s32(_p(a), _p(b), M, N, K, _p(r), R, _p(acc))
     return acc
+
+
+def gram(x: np.ndarray, rows=None):
+    """x^T x in fp64 for one calibration batch x [R, K] (fp32): rows `rows` (all if None)."""
+    x = _c(x, np.float32)
+    R, K = x.shape
+    r, NR = _rows(rows, K)
+    out = np.empty((NR, K), np.float64)
+    lib().q8o_gram_rows(_p(x), R, K, _p(r), NR, _p(out))
+    return out
+
+
+def hessian(batches, rows=None):
+    """[SmolVLM-Q8] hessians: the first batch's x^T x, then H = H + x^T x for each next batch
+    (in order; fp64)."""
+    H = None
+    for x in batches:
+        g = gram(x, rows)
+        H = g if H is None else H + g
+    return H
+
+
+def gptq_hinv(H: np.ndarray, damp: float = 0.01):
+    """Upper factor U (U^T U = damped H^-1) and the dead-column mask used by gptq_int8."""
+    H = _c(H, np.float64)
+    K = H.shape[0]
+    U = np.empty((K, K), np.float64)
+    dead = np.empty(K, np.uint8)
+    if lib().q8o_gptq_hinv(_p(H), K, float(damp), _p(U), _p(dead)) != 0:
+        raise np.linalg.LinAlgError("H is not positive definite after damping")
+    return U, dead.astype(bool)
+
+
+def gptq_int8(W: np.ndarray, H: np.ndarray, damp: float = 0.01, block: int = 128, rows=None):
+    """[SmolVLM-Q8] gptq_int8 -> (q int8 [R,K], s fp32 [R], wsum int32 [R]) for the listed
+    rows of W (all if None)."""
+    W = _c(W, np.float32)
+    H = _c(H, np.float64)
+    N, K = W.shape
+    r, R = _rows(rows, N)
+    q = np.empty((R, K), np.int8)
+    s = np.empty(R, np.float32)
+    ws = np.empty(R, np.int32)
+    if lib().q8o_gptq_int8(_p(W), _p(H), N, K, float(damp), int(block), _p(r), R, _p(q),
+                           _p(s), _p(ws)) != 0:
+        raise np.linalg.LinAlgError("H is not positive definite after damping")
+    return q, s, ws
 
 
 def round_bf16(y64: np.ndarray) -> np.ndarray:

@@ -454,6 +454,166 @@ void q8o_gemm_s8s8_s32(const int8_t* a, const int8_t* b,
     }
 }
 
+/* -------------------------------------------------- GPTQ on the int8 grid (f3)
+ * [SmolVLM-Q8] gptq_int8 (Frantar et al. 2022) and hessians, float64 throughout:
+ *   H = sum over calibration batches of x^T x (x the linear's fp32 inputs as float64);
+ *   scale s[n] from weight_int8 of the ORIGINAL row (observer grid, amax / 127.5);
+ *   dead columns (diag(H) == 0): H[k,k] = 1 and w[:,k] = 0;
+ *   H += damp * mean(diag(H)) * I;
+ *   hinv = upper Cholesky factor of H^-1, computed as the page does: the lower Cholesky
+ *          factor L of H, H^-1 = L^-T L^-1 (cholesky_inverse), then the upper factor U of
+ *          that (U^T U = H^-1);
+ *   columns in order, in blocks of `block`: q = clamp(round(w / s), -128, 127),
+ *          e = (w - q s) / U[i,i], the block's later columns w[:, j] -= e U[i, j], and after
+ *          the block every later column w[:, j] -= sum_t e_t U[t, j] (one matrix product).
+ * The page leaves the library routines' summation orders open; here every sum runs in
+ * ascending index order, one fp64 operation at a time (no fused multiply-add), which is
+ * the order the GPU implementation follows too.  Rows of W are independent once U exists.
+ */
+
+/* out[r][j] = sum_t x[t][rows[r]] * x[t][j] for t = 0..R-1 (ascending; fp32 products are
+ * exact in fp64).  rows == NULL means every row. */
+void q8o_gram_rows(const float* x, int64_t R, int64_t K, const int64_t* rows, int64_t nrows,
+                   double* out) {
+    const int64_t NR = rows ? nrows : K;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t r = 0; r < NR; ++r) {
+        const int64_t i = rows ? rows[r] : r;
+        double* o = out + r * K;
+        for (int64_t j = 0; j < K; ++j) o[j] = 0.0;
+        for (int64_t t = 0; t < R; ++t) {
+            const double xi = (double)x[t * K + i];
+            const float* xt = x + t * K;
+            for (int64_t j = 0; j < K; ++j) o[j] = o[j] + xi * (double)xt[j];
+        }
+    }
+}
+
+/* Lower Cholesky factor, left-looking, row-major L (zeros above the diagonal).
+ * Returns 1 if a pivot is not positive (H not positive definite). */
+static int chol_lower(const double* A, int64_t K, double* L) {
+    for (int64_t i = 0; i < K * K; ++i) L[i] = 0.0;
+    for (int64_t j = 0; j < K; ++j) {
+        double d = A[j * K + j];
+        for (int64_t k = 0; k < j; ++k) d = d - L[j * K + k] * L[j * K + k];
+        if (!(d > 0.0)) return 1;
+        d = sqrt(d);
+        L[j * K + j] = d;
+#pragma omp parallel for schedule(static)
+        for (int64_t i = j + 1; i < K; ++i) {
+            double t = A[i * K + j];
+            for (int64_t k = 0; k < j; ++k) t = t - L[i * K + k] * L[j * K + k];
+            L[i * K + j] = t / d;
+        }
+    }
+    return 0;
+}
+
+/* U (row-major, upper) with U^T U = (H damped)^-1; `dead` (nullable) receives the dead
+ * columns.  Returns 0, or 1 if a Cholesky pivot is not positive. */
+int q8o_gptq_hinv(const double* H0, int64_t K, double damp, double* U, unsigned char* dead) {
+    double* H = malloc(sizeof(double) * K * K);
+    double* L = malloc(sizeof(double) * K * K);
+    double* Li = malloc(sizeof(double) * K * K);
+    int bad = 0;
+    memcpy(H, H0, sizeof(double) * K * K);
+    for (int64_t k = 0; k < K; ++k) {
+        const int d = H[k * K + k] == 0.0;
+        if (dead) dead[k] = (unsigned char)d;
+        if (d) H[k * K + k] = 1.0;
+    }
+    double tr = 0.0;
+    for (int64_t k = 0; k < K; ++k) tr = tr + H[k * K + k];
+    const double add = damp * (tr / (double)K);
+    for (int64_t k = 0; k < K; ++k) H[k * K + k] = H[k * K + k] + add;
+    bad = chol_lower(H, K, L);
+    if (!bad) {
+        /* L^-1, column by column (forward substitution) */
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t j = 0; j < K; ++j) {
+            for (int64_t i = 0; i < j; ++i) Li[i * K + j] = 0.0;
+            Li[j * K + j] = 1.0 / L[j * K + j];
+            for (int64_t i = j + 1; i < K; ++i) {
+                double t = 0.0;
+                for (int64_t k = j; k < i; ++k) t = t - L[i * K + k] * Li[k * K + j];
+                Li[i * K + j] = t / L[i * K + i];
+            }
+        }
+        /* H^-1 = L^-T L^-1: entry (i, j) = sum over k >= max(i, j), ascending */
+#pragma omp parallel for schedule(dynamic, 4)
+        for (int64_t i = 0; i < K; ++i)
+            for (int64_t j = i; j < K; ++j) {
+                double t = 0.0;
+                for (int64_t k = j; k < K; ++k) t = t + Li[k * K + i] * Li[k * K + j];
+                H[i * K + j] = t;
+                H[j * K + i] = t;
+            }
+        /* upper factor of H^-1: the transpose of its lower factor */
+        bad = chol_lower(H, K, L);
+        if (!bad)
+            for (int64_t i = 0; i < K; ++i)
+                for (int64_t j = 0; j < K; ++j) U[i * K + j] = L[j * K + i];
+    }
+    free(H);
+    free(L);
+    free(Li);
+    return bad;
+}
+
+/* GPTQ codes of the listed rows of W (rows == NULL: all N), scale s[r] and code sum
+ * wsum[r] (nullable) per listed row.  Returns 0, or 1 if H is not positive definite. */
+int q8o_gptq_int8(const float* W, const double* H, int64_t N, int64_t K, double damp,
+                  int64_t block, const int64_t* rows, int64_t nrows, int8_t* q, float* s,
+                  int32_t* wsum) {
+    double* U = malloc(sizeof(double) * K * K);
+    unsigned char* dead = malloc((size_t)K);
+    const int bad = q8o_gptq_hinv(H, K, damp, U, dead);
+    const int64_t NR = rows ? nrows : N;
+    if (!bad) {
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t r = 0; r < NR; ++r) {
+            const int64_t n = rows ? rows[r] : r;
+            const float* wrow = W + n * K;
+            int8_t* qrow = q + r * K;
+            float sc;
+            int8_t* tmp = malloc((size_t)K);
+            q8o_quantize_weight_full128(wrow, 1, K, tmp, &sc, NULL);  /* scale of the original row */
+            free(tmp);
+            const double sd = (double)sc;
+            double* w = malloc(sizeof(double) * K);
+            double* err = malloc(sizeof(double) * block);
+            for (int64_t k = 0; k < K; ++k) w[k] = dead[k] ? 0.0 : (double)wrow[k];
+            int64_t sum = 0;
+            for (int64_t i1 = 0; i1 < K; i1 += block) {
+                const int64_t i2 = i1 + block < K ? i1 + block : K;
+                for (int64_t i = i1; i < i2; ++i) {
+                    const double col = w[i];
+                    double qc = nearbyint(col / sd);
+                    if (qc < -128.0) qc = -128.0;
+                    if (qc > 127.0) qc = 127.0;
+                    qrow[i] = (int8_t)(int)qc;
+                    sum += (int)qc;
+                    const double e = (col - qc * sd) / U[i * K + i];
+                    for (int64_t j = i; j < i2; ++j) w[j] = w[j] - e * U[i * K + j];
+                    err[i - i1] = e;
+                }
+                for (int64_t j = i2; j < K; ++j) {
+                    double p = 0.0;
+                    for (int64_t t = i1; t < i2; ++t) p = p + err[t - i1] * U[t * K + j];
+                    w[j] = w[j] - p;
+                }
+            }
+            s[r] = sc;
+            if (wsum) wsum[r] = (int32_t)sum;
+            free(w);
+            free(err);
+        }
+    }
+    free(U);
+    free(dead);
+    return bad;
+}
+
 /* ------------------------------------------------------- output rounding
  * Round an fp64 value once to bf16 (8 significant bits, ties to even), returned
  * as its 16-bit pattern.  Used to form "the fp64 result rounded to bf16".

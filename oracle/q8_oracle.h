@@ -47,6 +47,12 @@ void q8o_linear_dq8ca_q4gsw(const int8_t* xq, const float* s, const int32_t* z,
 void q8o_gemm_s8s8_s32(const int8_t* a, const int8_t* b,
                        int64_t M, int64_t N, int64_t K,
                        const int64_t* rows, int64_t nrows, int32_t* acc);
+void q8o_gram_rows(const float* x, int64_t R, int64_t K, const int64_t* rows, int64_t nrows,
+                   double* out);
+int  q8o_gptq_hinv(const double* H0, int64_t K, double damp, double* U, unsigned char* dead);
+int  q8o_gptq_int8(const float* W, const double* H, int64_t N, int64_t K, double damp,
+                   int64_t block, const int64_t* rows, int64_t nrows, int8_t* q, float* s,
+                   int32_t* wsum);
 uint16_t q8o_round_bf16(double v);
 void q8o_round_bf16_array(const double* v, int64_t n, uint16_t* out);
 

@@ -64,6 +64,22 @@ MUTANTS = [
      ["test_golden_residual_observer_rows"]),
     ("residual observer drops the zero point", "float fq = (q - (float)z1) * s1;",
      "float fq = q * s1;", ["test_golden_residual_observer_rows"]),
+    ("gptq error not scaled by the inverse-Hessian pivot",
+     "const double e = (col - qc * sd) / U[i * K + i];", "const double e = (col - qc * sd);",
+     ["test_gptq_codes_are_obs_optimal_roundings"]),
+    ("gptq block update sign", "w[j] = w[j] - p;", "w[j] = w[j] + p;",
+     ["test_gptq_codes_are_obs_optimal_roundings"]),
+    ("gptq damping on every entry",
+     "for (int64_t k = 0; k < K; ++k) H[k * K + k] = H[k * K + k] + add;",
+     "for (int64_t k = 0; k < K * K; ++k) H[k] = H[k] + add;",
+     ["test_gptq_hinv_is_upper_factor_of_damped_inverse"]),
+    ("gptq dead column kept", "w[k] = dead[k] ? 0.0 : (double)wrow[k];",
+     "w[k] = (double)wrow[k];", ["test_gptq_dead_columns_and_error_reduction"]),
+    ("gptq lower factor instead of upper", "U[i * K + j] = L[j * K + i];",
+     "U[i * K + j] = L[i * K + j];", ["test_gptq_hinv_is_upper_factor_of_damped_inverse"]),
+    ("gram drops the last calibration row", "for (int64_t t = 0; t < R; ++t) {\n            const double xi",
+     "for (int64_t t = 0; t < R - 1; ++t) {\n            const double xi",
+     ["test_gram_and_hessian_match_numpy"]),
     ("full grid ignores negative extremes", "const float amax = (-lo > hi) ? -lo : hi;",
      "const float amax = hi;", ["test_golden_weight_rows_full128"]),
 ]

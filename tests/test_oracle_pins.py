@@ -540,3 +540,112 @@ def test_residual_observer_half_step_bound():
     assert -s1 * (0.5 + 2.0 ** -16) <= lo <= 0.0 <= hi <= s1 * (0.5 + 2.0 ** -16)
     grid = (np.arange(-100, 100, dtype=np.float32) * np.float32(0.25)).astype(np.float32)
     assert oracle.residual_minmax(grid, (0.25, 0)) == (0.0, 0.0)
+
+
+# ------------------------------------------------------- GPTQ on the int8 grid (f3)
+
+
+def _calib_x(R, K, seed, dead=()):
+    """Correlated calibration inputs (mixed Gaussian columns), some columns never active."""
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal((R, K))
+    mix = np.eye(K) + 0.6 * rng.standard_normal((K, K)) / np.sqrt(K)
+    x = (z @ mix).astype(np.float32)
+    for k in dead:
+        x[:, k] = 0.0
+    return x
+
+
+def test_gram_and_hessian_match_numpy():
+    """hessians (SmolVLM q8 page): sum over batches of x^T x in fp64, against numpy's matmul
+    (fp32 products are exact in fp64, so only the summation order differs)."""
+    x = _calib_x(300, 40, seed=41)
+    b1, b2 = x[:170], x[170:]
+    H = oracle.hessian([b1, b2])
+    ref = b1.astype(np.float64).T @ b1.astype(np.float64) + \
+        b2.astype(np.float64).T @ b2.astype(np.float64)
+    mag = np.abs(x.astype(np.float64)).T @ np.abs(x.astype(np.float64))
+    assert np.all(np.abs(H - ref) <= mag * 300 * 2.0 ** -52)
+    assert np.array_equal(oracle.gram(b1, rows=[3, 17]), oracle.gram(b1)[[3, 17]])
+
+
+def test_gptq_hinv_is_upper_factor_of_damped_inverse():
+    K = 48
+    x = _calib_x(200, K, seed=42, dead=(5, 30))
+    H = oracle.hessian([x])
+    U, dead = oracle.gptq_hinv(H, 0.01)
+    assert dead.tolist() == [k in (5, 30) for k in range(K)]
+    Hd = H.copy()
+    Hd[dead, dead] = 1.0
+    Hd += 0.01 * np.mean(np.diag(Hd)) * np.eye(K)
+    assert np.abs(np.tril(U, -1)).max() == 0.0 and np.all(np.diag(U) > 0)
+    assert np.abs(U.T @ U @ Hd - np.eye(K)).max() < 1e-9
+
+
+def test_gptq_identity_hessian_is_round_to_nearest():
+    """With H a multiple of I no error propagates (hinv is diagonal): GPTQ reduces to round
+    to nearest on weight_int8's grid and scales -- with the page's float64 division w / s."""
+    W = wl.weight(9, 64, seed=43).numpy()
+    q, s, ws = oracle.gptq_int8(W, 3.0 * np.eye(64), block=16)
+    _, rs, _ = oracle.quantize_weight(W, grid="full128")
+    want = np.clip(np.rint(W.astype(np.float64) / rs.astype(np.float64)[:, None]), -128, 127)
+    assert np.array_equal(s, rs)
+    assert np.array_equal(q, want.astype(np.int8))
+    assert np.array_equal(ws, want.sum(axis=1).astype(np.int32))
+
+
+def _obs_values(w, q, s, Hd):
+    """Per column i, the least-squares value of w_i once columns < i are fixed at q * s:
+    argmin over u of (w - [q_<i s, u]) Hd (w - [q_<i s, u])^T, solved directly."""
+    K = w.size
+    v = np.empty(K)
+    for i in range(K):
+        a = w[:i] - q[:i] * s
+        rhs = Hd[i:, :i] @ a
+        v[i] = w[i] + np.linalg.solve(Hd[i:, i:], rhs)[0]
+    return v
+
+
+def test_gptq_codes_are_obs_optimal_roundings():
+    """Frantar et al.'s result that gptq_int8 implements: the value rounded at column i is
+    the optimum of the layer's quadratic error over the not-yet-rounded weights, given the
+    codes already chosen.  Checked per column against a direct solve (numpy), away from
+    rounding ties."""
+    K, N = 20, 4
+    x = _calib_x(80, K, seed=44, dead=(3,))
+    H = oracle.hessian([x])
+    W = wl.weight(N, K, seed=45).numpy() * 50
+    _, dead = oracle.gptq_hinv(H)
+    Hd = H.copy()
+    Hd[dead, dead] = 1.0
+    Hd += 0.01 * np.mean(np.diag(Hd)) * np.eye(K)
+    for block in (4, 7, 128):                        # ragged last block with 7
+        q, s, ws = oracle.gptq_int8(W, H, block=block)
+        checked = 0
+        for n in range(N):
+            w = np.where(dead, 0.0, W[n].astype(np.float64))
+            v = _obs_values(w, q[n].astype(np.float64), float(s[n]), Hd) / float(s[n])
+            want = np.clip(np.rint(v), -128, 127)
+            away = np.abs(np.abs(v - np.floor(v)) - 0.5) > 1e-7
+            assert np.array_equal(q[n][away], want[away]), f"row {n} block {block}"
+            checked += away.sum()
+        assert checked >= 0.95 * N * K
+        assert np.array_equal(ws, q.astype(np.int64).sum(axis=1))
+
+
+def test_gptq_dead_columns_and_error_reduction():
+    """Dead columns (never-active inputs) get code 0 even where W is large, and GPTQ's
+    quadratic error tr((W - Qs) H (W - Qs)^T) beats round-to-nearest on correlated inputs."""
+    K, N = 64, 16
+    x = _calib_x(400, K, seed=46, dead=(0, 17))
+    H = oracle.hessian([x])
+    W = wl.weight(N, K, seed=47).numpy()
+    W[:, 17] = 0.05
+    q, s, _ = oracle.gptq_int8(W, H, block=16)
+    assert not q[:, [0, 17]].any()
+    rq, rs, _ = oracle.quantize_weight(W, grid="full128")
+
+    def qerr(codes, sc):
+        d = W.astype(np.float64) - codes.astype(np.float64) * sc.astype(np.float64)[:, None]
+        return float(np.einsum("nk,kl,nl->", d, H, d))
+    assert qerr(q, s) < 0.8 * qerr(rq, rs)
