@@ -11,7 +11,8 @@ is never re-read from L2.
 
 Extra sub-benchmarks (same JSON line, key "paths"): the sweep through the digit-plane
 form and with a bias, W8A8 static int8 linear (K = 960) and prefill (M = 4096, also with a
-bias), 8da4w, the quantizers (both weight grids) and a Llama-shaped stack.
+bias), 8da4w, the quantizers (both weight grids), a Llama-shaped stack and the offline
+GPTQ path (calibration Hessian + GPTQ of one 11008 x 4096 layer).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -602,6 +603,43 @@ def bench_quantizers(dev, peaks, reps=5):
     return out
 
 
+def bench_gptq(dev):
+    """The offline GPTQ path on one Llama MLP up-projection (N = 11008, K = 4096): the
+    calibration Hessian of 4096 fp32 rows (float64 x^T x), then GPTQ on the int8 grid
+    (float64 factorisations and updates).  Event-timed, one run each after a warm-up."""
+    import int8_quantized_linear_q8_b200 as q8
+
+    N, K, R = 11008, 4096, 4096
+    g = torch.Generator(device=dev)
+    g.manual_seed(93)
+    x = torch.randn(R, K, generator=g, device=dev)
+    W = torch.randn(N, K, generator=g, device=dev) * 0.02
+    H = torch.empty(K, K, dtype=torch.float64, device=dev)
+    nb = q8.q8_workspace_bytes(q8.Q8_OP_GPTQ_INT8, 0, N, K, 128)
+    work = torch.empty(nb, dtype=torch.uint8, device=dev)
+    q = torch.empty(N, K, dtype=torch.int8, device=dev)
+    s = torch.empty(N, device=dev)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    ms_h = timed(lambda: q8.q8_hessian_accumulate(x, H, reset=True))
+    ms_g = timed(lambda: q8.q8_gptq_int8(W, H, q=q, s_w=s, want_wsum=False, workspace=work))
+    out = {"hessian": {"R": R, "K": K, "ms": round(ms_h, 2),
+                       "fp64_Gops": round(R * K * (K + 1) / 2 * 2 / ms_h / 1e6, 1)},
+           "gptq": {"N": N, "K": K, "block": 128, "ms": round(ms_g, 1),
+                    "fp64_Gops": round((K ** 3 + N * K * K) * 2 / ms_g / 1e6, 1)}}
+    del x, W, H, work, q, s
+    return out
+
+
 def bench_llama_stack(dev, peaks, prefill=True):
     """Llama-shaped stack, 32 layers x (q, k, v, o 4096x4096; gate, up 4096->11008; down
     11008->4096): decode at M = 1 through the W8A16 GEMV (6.5 GB of int8 weights per pass,
@@ -755,6 +793,7 @@ def run_ours(args):
             "dq8ca_q4gsw": bench_q4(dev, peaks),
             "quantizers": bench_quantizers(dev, peaks),
             "llama_stack": bench_llama_stack(dev, peaks),
+            "gptq_offline": bench_gptq(dev),
         }
     dist.barrier()
     if dist.rank == 0:

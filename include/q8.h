@@ -72,7 +72,8 @@ typedef struct {
 typedef enum {
     Q8_OP_LINEAR_W8A8 = 0,
     Q8_OP_LINEAR_DQ8CA_Q4GSW = 1,
-    Q8_OP_LINEAR_W8A16_PLANES = 2   /* q8_linear_w8a16_planes */
+    Q8_OP_LINEAR_W8A16_PLANES = 2,  /* q8_linear_w8a16_planes */
+    Q8_OP_GPTQ_INT8 = 3             /* q8_gptq_int8 (M unused, extra = block) */
 } q8_op;
 
 /* Host.  Human-readable name of a status code (static string). */
@@ -269,6 +270,40 @@ q8_status q8_linear_w8a8_bias(const float* x, q8_qparams first, const q8_qparams
 q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* gs, int G,
                                 float* y, int64_t M, int64_t N, int64_t K,
                                 void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------- GPTQ (offline) */
+
+/* Calibration Hessian ([SmolVLM-Q8] hessians): the sum over calibration batches of x^T x,
+ * in float64 (the fp32 products are exact; each entry sums its batch's rows in ascending
+ * order, then adds to the running total).
+ *     H  = x^T x        (reset != 0)        H += x^T x      (reset == 0)
+ *   x device fp32 [R, K] (R >= 0); H device fp64 [K, K], symmetric on entry when
+ *   reset == 0 (as this call leaves it).  K as the shape conventions; R == 0 with reset
+ *   zeroes H. */
+q8_status q8_hessian_accumulate(const float* x, int64_t R, int64_t K, double* H, int reset,
+                                void* stream);
+
+/* GPTQ on the int8 grid of q8_quantize_weight_grid(Q8_GRID_FULL128) ([SmolVLM-Q8]
+ * gptq_int8, Frantar et al. 2022), float64 throughout:
+ *   s_w[n] = the observer-grid scale of the ORIGINAL row n of W;
+ *   dead columns (H[k,k] == 0): H[k,k] = 1 and W[:,k] = 0;  H += damp * mean(diag H) * I;
+ *   U = upper Cholesky factor of H^-1;  columns in order, in blocks of `block`:
+ *       q = clamp(round(w / s), -128, 127), e = (w - q s) / U[i,i], the block's later
+ *       columns w[:, j] -= e U[i, j]; after the block every later column
+ *       w[:, j] -= sum_t e_t U[t, j].
+ *   W device fp32 [N, K]; H device fp64 [K, K] (read); q device int8 [N, K]; s_w device
+ *   fp32 [N]; wsum device int32 [N] (code sums; nullable).  damp finite, >= 0; block in
+ *   [1, 256]; K <= 16384 (the three K x K float64 work matrices); Q8_ERR_ARG / SHAPE.
+ *   workspace: q8_workspace_bytes(Q8_OP_GPTQ_INT8, 0, N, K, block) bytes (about
+ *   24 K^2 + 2.1 kB N + 8 N K); contents on entry do not matter.
+ * Every float64 sum runs in ascending index order, one correctly rounded operation at a
+ * time, so the codes are the same bits as that sequential definition.  A Hessian that is
+ * not positive definite after damping records a device failure (q8_last_device_status
+ * returns Q8_ERR_DEVICE) and leaves q undefined.  Offline: O(K^3 + N K^2) float64 work,
+ * thousands of small launches. */
+q8_status q8_gptq_int8(const float* W, const double* H, int64_t N, int64_t K, double damp,
+                       int64_t block, int8_t* q, float* s_w, int32_t* wsum, void* workspace,
+                       size_t ws_bytes, void* stream);
 
 /* Host.  Workspace bytes a linear needs for these sizes (0 if none).  `extra` is
  * "two-pass" (0/1) for Q8_OP_LINEAR_W8A8, G for Q8_OP_LINEAR_DQ8CA_Q4GSW and unused (0)

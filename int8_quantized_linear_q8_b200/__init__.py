@@ -25,6 +25,7 @@ Q8_ERR_NULL, Q8_ERR_SHAPE, Q8_ERR_ALIGN, Q8_ERR_ARG = 1, 2, 3, 4
 Q8_ERR_UNSUPPORTED_ARCH, Q8_ERR_LAUNCH, Q8_ERR_WORKSPACE, Q8_ERR_DEVICE = 5, 6, 7, 8
 Q8_F32, Q8_BF16 = 0, 1
 Q8_OP_LINEAR_W8A8, Q8_OP_LINEAR_DQ8CA_Q4GSW, Q8_OP_LINEAR_W8A16_PLANES = 0, 1, 2
+Q8_OP_GPTQ_INT8 = 3
 Q8_GRID_SYM127, Q8_GRID_FULL128 = 0, 1
 _GRIDS = {"sym127": Q8_GRID_SYM127, "full128": Q8_GRID_FULL128}
 
@@ -36,7 +37,7 @@ SYMBOLS = (
     "q8_workspace_bytes", "q8_gemm_s8s8_s32", "q8_last_device_status",
     "q8_linear_w8a8_noalloc", "q8_selftest_bounded_wait", "q8_linear_w8a16_planes",
     "q8_quantize_weight_grid", "q8_linear_w8a16_bias", "q8_linear_w8a8_bias",
-    "q8_observe_residual_minmax",
+    "q8_observe_residual_minmax", "q8_hessian_accumulate", "q8_gptq_int8",
 )
 # Built-in scratch of q8_linear_w8a8_noalloc (bytes).
 Q8_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -80,6 +81,11 @@ def _lib() -> ctypes.CDLL:
                                      _vp, _vp, _vp]
     L.q8_observe_minmax.restype = st
     L.q8_observe_minmax.argtypes = [_vp, _i64, _vp, st, _vp]
+    L.q8_hessian_accumulate.restype = st
+    L.q8_hessian_accumulate.argtypes = [_vp, _i64, _i64, _vp, st, _vp]
+    L.q8_gptq_int8.restype = st
+    L.q8_gptq_int8.argtypes = [_vp, _vp, _i64, _i64, ctypes.c_double, _i64, _vp, _vp, _vp,
+                               _vp, _sz, _vp]
     L.q8_observe_residual_minmax.restype = st
     L.q8_observe_residual_minmax.argtypes = [_vp, _i64, q8_qparams, _vp, st, _vp]
     L.q8_qparams_from_minmax.restype = st
@@ -381,6 +387,39 @@ def q8_linear_w8a8_noalloc(x: torch.Tensor, first, q: torch.Tensor, wsum: torch.
                                          _ptr(s_w), _ptr(y), M, N, K, _stream(stream)),
            "q8_linear_w8a8_noalloc")
     return y
+
+
+def q8_hessian_accumulate(x: torch.Tensor, H: Optional[torch.Tensor] = None,
+                          reset: bool = False, stream=None) -> torch.Tensor:
+    """H (= if reset or H is None, else +=) x^T x in float64; x fp32 [R, K]."""
+    R, K = x.shape
+    _need(x, "x", torch.float32, (R, K))
+    if H is None:
+        H = torch.empty(K, K, dtype=torch.float64, device=x.device)
+        reset = True
+    _need(H, "H", torch.float64, (K, K))
+    _check(_lib().q8_hessian_accumulate(_ptr(x), R, K, _ptr(H), int(bool(reset)),
+                                        _stream(stream)), "q8_hessian_accumulate")
+    return H
+
+
+def q8_gptq_int8(W: torch.Tensor, H: torch.Tensor, damp: float = 0.01, block: int = 128,
+                 q=None, s_w=None, wsum=None, want_wsum=True, workspace=None, stream=None):
+    """GPTQ int8 codes of an fp32 [N, K] weight against a float64 [K, K] calibration Hessian
+    -> (q int8 [N, K], s_w fp32 [N], wsum int32 [N] | None)."""
+    N, K = W.shape
+    _need(W, "W", torch.float32, (N, K))
+    _need(H, "H", torch.float64, (K, K))
+    q = _out(q, "q", torch.int8, (N, K), W.device)
+    s_w = _out(s_w, "s_w", torch.float32, (N,), W.device)
+    if want_wsum or wsum is not None:
+        wsum = _out(wsum, "wsum", torch.int32, (N,), W.device)
+    nbytes = q8_workspace_bytes(Q8_OP_GPTQ_INT8, 0, N, K, int(block))
+    workspace, wsb = _workspace(workspace, nbytes, W.device)
+    _check(_lib().q8_gptq_int8(_ptr(W), _ptr(H), N, K, float(damp), int(block), _ptr(q),
+                               _ptr(s_w), _ptr(wsum), _ptr(workspace), wsb, _stream(stream)),
+           "q8_gptq_int8")
+    return q, s_w, wsum
 
 
 def q8_linear_dq8ca_q4gsw(x: torch.Tensor, q4: torch.Tensor, gs: torch.Tensor, G: int, y=None,

@@ -107,6 +107,7 @@ static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; 
 // 128-byte steps and needs at least one whole step.
 constexpr int64_t kW8A8GemvMaxM = 16;
 constexpr int64_t kTcMinK = 128;
+constexpr int64_t kGptqMaxK = 16384;     // three K x K float64 work matrices (6 GB at the cap)
 
 // Workspace plans (byte offsets inside the caller's workspace).
 struct W8A8Plan {
@@ -350,6 +351,9 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) 
             return w8a16_tc_workspace_bytes(M, K, sms);
         }
         case Q8_OP_LINEAR_W8A8: return plan_w8a8(M, K, extra != 0).bytes;
+        case Q8_OP_GPTQ_INT8:
+            if (K > kGptqMaxK || !gptq_block_ok(extra)) return 0;
+            return plan_gptq(N, K).bytes;
         case Q8_OP_LINEAR_DQ8CA_Q4GSW: {
             if (!valid_group(extra) || K % 128 != 0 || K % extra != 0) return 0;
             int sms = 0;
@@ -358,6 +362,37 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) 
         }
     }
     return 0;
+}
+
+q8_status q8_hessian_accumulate(const float* x, int64_t R, int64_t K, double* H, int reset,
+                                void* stream) {
+    if (R < 0 || R > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (R == 0 && !reset) return Q8_OK;
+    if (!H || (R > 0 && !x)) return Q8_ERR_NULL;
+    if ((x && !aligned16(x)) || !aligned16(H)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_hessian_accumulate(x, R, (int)K, H, reset, (cudaStream_t)stream));
+}
+
+q8_status q8_gptq_int8(const float* W, const double* H, int64_t N, int64_t K, double damp,
+                       int64_t block, int8_t* q, float* s_w, int32_t* wsum, void* workspace,
+                       size_t ws_bytes, void* stream) {
+    if (N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (K > kGptqMaxK) return Q8_ERR_SHAPE;
+    if (!gptq_block_ok(block) || !isfinite(damp) || damp < 0.0) return Q8_ERR_ARG;
+    if (!W || !H || !q || !s_w) return Q8_ERR_NULL;
+    if (!aligned16(W) || !aligned16(H) || !aligned16(q) || !aligned4(wsum)) return Q8_ERR_ALIGN;
+    const GptqPlan plan = plan_gptq(N, K);
+    if (!workspace || ws_bytes < plan.bytes) return Q8_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    int* status = nullptr;
+    Q8_TRY(current_device(sms, &status));
+    return launched(launch_gptq_int8(W, H, N, (int)K, damp, (int)block, q, s_w, wsum, workspace,
+                                     (cudaStream_t)stream, sms, status));
 }
 
 q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* second,

@@ -179,6 +179,7 @@ namespace q8 {
 
 // Device status codes written to the caller-visible status word.
 constexpr int kStatusWaitTimeout = 1;
+constexpr int kStatusNotPositiveDefinite = 2;   // a Cholesky pivot was not positive
 // Bounded waits give up after this many nanoseconds of %globaltimer (a correct kernel
 // never waits more than microseconds; the limit only turns a logic error into an error
 // status instead of a hang).

@@ -104,6 +104,18 @@ cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const floa
                               const float* s, float* y, int G, int64_t M, int64_t N, int K,
                               cudaStream_t st, int num_sms, int* status);
 
+// k_gptq.cu
+struct GptqPlan {
+    size_t buf0, buf1, buf2, w, err, col, dead, bytes;   // byte offsets in the workspace
+};
+GptqPlan plan_gptq(int64_t N, int64_t K);
+bool gptq_block_ok(int64_t block);
+cudaError_t launch_hessian_accumulate(const float* x, int64_t R, int K, double* H, int reset,
+                                      cudaStream_t st);
+cudaError_t launch_gptq_int8(const float* W, const double* H, int64_t N, int K, double damp,
+                             int block, int8_t* q, float* s_w, int32_t* wsum, void* ws,
+                             cudaStream_t st, int num_sms, int* status);
+
 // k_gemv.cu
 cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w,
                               const float* bias, void* y, int y_bf16, int64_t M, int64_t N, int K,

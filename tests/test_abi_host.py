@@ -112,6 +112,27 @@ def test_argument_validation_before_device(L):
                                  1024, None) == q8.Q8_ERR_ALIGN
     assert L.q8_linear_w8a8_bias(good, bad_qp, None, good, good, good, good, good, 1, 16, 64,
                                  good, 1024, None) == q8.Q8_ERR_ARG
+    # GPTQ and the calibration Hessian
+    assert L.q8_hessian_accumulate(good, -1, 64, good, 1, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_hessian_accumulate(good, 4, 60, good, 1, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_hessian_accumulate(good, 0, 64, good, 0, None) == q8.Q8_OK
+    assert L.q8_hessian_accumulate(odd, 4, 64, good, 1, None) == q8.Q8_ERR_ALIGN
+    ws_g = q8.q8_workspace_bytes(q8.Q8_OP_GPTQ_INT8, 0, 8, 64, 128)
+    assert ws_g >= 3 * 64 * 64 * 8 + 8 * 64 * 8
+    assert q8.q8_workspace_bytes(q8.Q8_OP_GPTQ_INT8, 0, 8, 64, 0) == 0
+    assert q8.q8_workspace_bytes(q8.Q8_OP_GPTQ_INT8, 0, 8, 16384 + 16, 128) == 0
+    assert L.q8_gptq_int8(good, good, 8, 64, 0.01, 0, good, good, None, good, ws_g,
+                          None) == q8.Q8_ERR_ARG
+    assert L.q8_gptq_int8(good, good, 8, 64, -1.0, 128, good, good, None, good, ws_g,
+                          None) == q8.Q8_ERR_ARG
+    assert L.q8_gptq_int8(good, good, 8, 64, float("nan"), 128, good, good, None, good, ws_g,
+                          None) == q8.Q8_ERR_ARG
+    assert L.q8_gptq_int8(good, good, 8, 16400, 0.01, 128, good, good, None, good, ws_g,
+                          None) == q8.Q8_ERR_SHAPE
+    assert L.q8_gptq_int8(good, good, 8, 64, 0.01, 128, good, good, None, good, ws_g - 8,
+                          None) == q8.Q8_ERR_WORKSPACE
+    assert L.q8_gptq_int8(good, None, 8, 64, 0.01, 128, good, good, None, good, ws_g,
+                          None) == q8.Q8_ERR_NULL
     mmp = _p(0x10000)
     assert L.q8_observe_residual_minmax(good, 64, bad_qp, mmp, 1, None) == q8.Q8_ERR_ARG
     assert L.q8_observe_residual_minmax(good, -1, qp, mmp, 1, None) == q8.Q8_ERR_SHAPE
