@@ -13,7 +13,7 @@
 //
 //     x[m, k]               = 2^(b_m - 134) * sum_j 128^j d_j[m, k]
 //     sum_k x[m, k] q[n, k] = 2^(b_m - 134) * sum_j 128^j P_j[m, n],
-//     P_j[m, n]             = sum_k d_j[m, k] q[n, k]   (int32, exact: |P| <= 127*127*K < 2^31)
+//     P_j[m, n]             = sum_k d_j[m, k] q[n, k]   (int32, exact: |P| <= 127*128*K < 2^31)
 //
 // Every P_j is one column of an int8 GEMM whose B operand is the plane matrix with rows
 // (j, m) (row index j*M + m).  The epilogue recombines a row's columns in fp64 (Horner in

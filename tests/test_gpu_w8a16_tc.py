@@ -210,3 +210,20 @@ def test_w8a16_tc_graph_replay():
         torch.cuda.synchronize()
         y64, absum = oracle.linear_w8a16(wl.bf16_bits(x), rq, rs)
         _tight(y.cpu().numpy(), y64, absum, f"graph replay {r}")
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_w8a16_tc_full_int8_grid(M):
+    """Weights on the observer grid (codes down to -128, weight_int8 of the SmolVLM q8 page):
+    the digit-plane products stay exact in int32 (|P| <= 127 * 128 * K)."""
+    N, K = 2560, 960
+    W = wl.weight(N, K, seed=80)
+    W[3:, 0] = -W[3:].abs().amax(dim=1) * 1.01
+    q, s, _ = q8.q8_quantize_weight(W.to(DEV), want_wsum=False, grid="full128")
+    x = wl.normal_bf16((M, K), 1.0, seed=81)
+    y = q8.q8_linear_w8a16_planes(x.to(DEV), q, s, _ws(M, N, K), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rq, rs, _ = oracle.quantize_weight(W.numpy(), grid="full128")
+    assert (rq == -128).any()
+    y64, absum = oracle.linear_w8a16(wl.bf16_bits(x), rq, rs)
+    _tight(y.cpu().numpy(), y64, absum, f"planes on the full grid M={M}")
