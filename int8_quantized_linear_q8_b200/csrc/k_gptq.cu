@@ -18,7 +18,7 @@
 // is O(K^3) for the factorisations and O(N K^2) for the updates, offline, once per layer.
 //
 //   * Cholesky factorisations and the triangular inverse are right-looking: one launch per
-//     pivot k updates the whole trailing region.  An entry then receives its subtractions
+//     pivot k finalises the pivot column (row) and updates the whole trailing region.  An entry then receives its subtractions
 //     in ascending k -- the order of the left-looking dot products -- while every launch
 //     has (K - k)^2 / 2 independent entries instead of a long per-thread chain.
 //   * Row n of W is independent of every other row once U exists: the in-block column loop
@@ -115,62 +115,84 @@ __global__ void k_gptq_diag(const double* __restrict__ H, int K, double damp,
 
 // ---------------------------------------------------------------- Cholesky, step k
 // T holds A with the subtractions of pivots < k applied (row-major, lower triangle used).
-// Step k, first kernel (column k):  L[k, k] = d = sqrt(T[k, k]),  L[i, k] = T[i, k] / d
-// (also copied to the contiguous vector col[i]); second kernel (trailing triangle):
-// T[i, j] = T[i, j] - L[i, k] * L[j, k] for k < j <= i.  Each entry of L is the left-looking
-// sequential formula of the reference: its subtractions arrive in ascending k.
-__global__ __launch_bounds__(256) void k_chol_col(const double* __restrict__ T,
-                                                  double* __restrict__ L,
-                                                  double* __restrict__ col, int K, int k,
-                                                  int* status) {
+// Step k, one launch over 32 x 32 tiles of the trailing triangle {(i, j): k < j <= i < K}:
+//   L[k, k] = d = sqrt(T[k, k]),  L[i, k] = T[i, k] / d   (written by the first tile column)
+//   T[i, j] = T[i, j] - L[i, k] * L[j, k]
+// Each tile divides its own 32 + 32 entries of column k into shared memory (the same
+// correctly rounded divisions wherever they are repeated, so the same bits).  Every entry of
+// L is the left-looking sequential formula of the reference: its subtractions arrive in
+// ascending k.  Column k of T is only read in step k.
+__global__ __launch_bounds__(256) void k_chol_step(double* __restrict__ T, double* __restrict__ L,
+                                                   int K, int k, int* status) {
+    __shared__ double li[32], lj[32];
+    const int i0 = k + 1 + blockIdx.y * 32, j0 = k + 1 + blockIdx.x * 32;
+    if (j0 > i0 + 31) return;                            // tile above the diagonal
     const double tkk = T[(int64_t)k * K + k];
     const double d = __dsqrt_rn(tkk);
-    if (!(tkk > 0.0) && blockIdx.x == 0 && threadIdx.x == 0 && status)
-        atomicExch(status, kStatusNotPositiveDefinite);
-    for (int i = k + blockIdx.x * blockDim.x + threadIdx.x; i < K; i += gridDim.x * blockDim.x) {
-        const double v = (i == k) ? d : __ddiv_rn(T[(int64_t)i * K + k], d);
-        L[(int64_t)i * K + k] = v;
-        col[i] = v;
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        L[(int64_t)k * K + k] = d;
+        if (!(tkk > 0.0) && status) atomicExch(status, kStatusNotPositiveDefinite);
     }
-}
-
-// 32 x 8 threads per CTA: x over j (consecutive addresses of a row), y over i.
-__global__ __launch_bounds__(256) void k_chol_update(double* __restrict__ T,
-                                                     const double* __restrict__ col, int K,
-                                                     int k) {
-    const int j0 = k + 1 + blockIdx.x * 32, i0 = k + 1 + blockIdx.y * 32;
-    if (j0 > i0 + 31) return;                            // tile above the diagonal
-    const int j = j0 + (threadIdx.x & 31);
+    if (threadIdx.x < 32) {
+        const int i = i0 + threadIdx.x;
+        if (i < K) {
+            li[threadIdx.x] = __ddiv_rn(T[(int64_t)i * K + k], d);
+            if (blockIdx.x == 0) L[(int64_t)i * K + k] = li[threadIdx.x];
+        }
+    } else if (threadIdx.x < 64) {
+        const int j = j0 + threadIdx.x - 32;
+        if (j < K) lj[threadIdx.x - 32] = __ddiv_rn(T[(int64_t)j * K + k], d);
+    }
+    __syncthreads();
+    const int c = threadIdx.x & 31, j = j0 + c;
     if (j >= K) return;
-    const double cj = col[j];
-    for (int i = i0 + (threadIdx.x >> 5); i < i0 + 32 && i < K; i += 8)
-        if (j <= i) T[(int64_t)i * K + j] = dsub_mul(T[(int64_t)i * K + j], col[i], cj);
+    for (int r = threadIdx.x >> 5; r < 32; r += 8) {
+        const int i = i0 + r;
+        if (i < K && j <= i) T[(int64_t)i * K + j] = dsub_mul(T[(int64_t)i * K + j], li[r], lj[c]);
+    }
 }
 
 // ------------------------------------------------------- inverse of L, step k
 // Column-oriented forward substitution for every column j at once.  S holds the running
 // sums t[i, j] = 0 - sum_{k' < k} L[i, k'] Li[k', j] (row-major; zero-initialised).
-// Step k, first kernel (row k):  Li[k, j] = S[k, j] / L[k, k] (j < k),  Li[k, k] = 1 / L[k, k];
-// second kernel:  S[i, j] = S[i, j] - L[i, k] * Li[k, j]  for i > k, j <= k.
-__global__ __launch_bounds__(256) void k_trinv_row(const double* __restrict__ L,
-                                                   const double* __restrict__ S,
-                                                   double* __restrict__ Li, int K, int k) {
+// Step k, one launch over 32 x 32 tiles of {(i, j): k < i < K, j <= k} (at least one tile
+// row, so that row k is written even when k = K - 1):
+//   Li[k, j] = S[k, j] / L[k, k] (j < k),  Li[k, k] = 1 / L[k, k]  (first tile row writes)
+//   S[i, j] = S[i, j] - L[i, k] * Li[k, j]
+__global__ __launch_bounds__(256) void k_trinv_step(const double* __restrict__ L,
+                                                    double* __restrict__ S,
+                                                    double* __restrict__ Li, int K, int k) {
+    __shared__ double y[32];
+    const int j0 = blockIdx.x * 32, i0 = k + 1 + blockIdx.y * 32;
     const double lkk = L[(int64_t)k * K + k];
-    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j <= k; j += gridDim.x * blockDim.x)
-        Li[(int64_t)k * K + j] =
-            (j == k) ? __ddiv_rn(1.0, lkk) : __ddiv_rn(S[(int64_t)k * K + j], lkk);
+    if (threadIdx.x < 32) {
+        const int j = j0 + threadIdx.x;
+        if (j <= k) {
+            y[threadIdx.x] =
+                (j == k) ? __ddiv_rn(1.0, lkk) : __ddiv_rn(S[(int64_t)k * K + j], lkk);
+            if (blockIdx.y == 0) Li[(int64_t)k * K + j] = y[threadIdx.x];
+        }
+    }
+    __syncthreads();
+    const int c = threadIdx.x & 31, j = j0 + c;
+    if (j > k) return;
+    for (int r = threadIdx.x >> 5; r < 32; r += 8) {
+        const int i = i0 + r;
+        if (i < K) S[(int64_t)i * K + j] = dsub_mul(S[(int64_t)i * K + j], L[(int64_t)i * K + k], y[c]);
+    }
 }
 
-__global__ __launch_bounds__(256) void k_trinv_update(const double* __restrict__ L,
-                                                      double* __restrict__ S,
-                                                      const double* __restrict__ Li, int K,
-                                                      int k) {
-    const int j = blockIdx.x * 32 + (threadIdx.x & 31);
-    if (j > k) return;
-    const double y = Li[(int64_t)k * K + j];
-    for (int i = k + 1 + blockIdx.y * 32 + (threadIdx.x >> 5);
-         i < k + 1 + (blockIdx.y + 1) * 32 && i < K; i += 8)
-        S[(int64_t)i * K + j] = dsub_mul(S[(int64_t)i * K + j], L[(int64_t)i * K + k], y);
+// U = LA^T (exact copies), so that the block updates read rows of U: coalesced across the
+// later columns j.
+__global__ __launch_bounds__(256) void k_transpose(const double* __restrict__ A, int K,
+                                                   double* __restrict__ B) {
+    __shared__ double t[32][33];
+    const int i0 = blockIdx.y * 32, j0 = blockIdx.x * 32, c = threadIdx.x & 31;
+    for (int r = threadIdx.x >> 5; r < 32; r += 8)
+        if (i0 + r < K && j0 + c < K) t[r][c] = A[(int64_t)(i0 + r) * K + j0 + c];
+    __syncthreads();
+    for (int r = threadIdx.x >> 5; r < 32; r += 8)
+        if (j0 + r < K && i0 + c < K) B[(int64_t)(j0 + r) * K + i0 + c] = t[c][r];
 }
 
 // -------------------------------------------------------- H^-1 = Li^T Li
@@ -228,11 +250,11 @@ __global__ void k_gptq_init_w(const float* __restrict__ W, const unsigned char* 
         w[e] = dead[e % K] ? 0.0 : (double)W[e];
 }
 
-// The block [i1, i2): one thread per row, the block's columns in order.  LA is the lower
-// factor of H^-1 (U[i, j] = LA[j, i]).  Codes go to q, the scaled errors to err[n, 0..B),
-// and the code sum accumulates in wsum (initialised by the first block).
+// The block [i1, i2): one thread per row, the block's columns in order.  U is the upper
+// factor of H^-1 (row-major).  Codes go to q, the scaled errors to err[n, 0..B), and the code
+// sum accumulates in wsum (initialised by the first block).
 __global__ __launch_bounds__(GQ_ROW_THREADS) void k_gptq_block(
-    double* __restrict__ w, const double* __restrict__ LA, const float* __restrict__ s_w,
+    double* __restrict__ w, const double* __restrict__ U, const float* __restrict__ s_w,
     int64_t N, int K, int i1, int i2, int8_t* __restrict__ q, double* __restrict__ err,
     int32_t* __restrict__ wsum) {
     extern __shared__ double w1s[];                      // [GQ_ROW_THREADS][B + 1]
@@ -251,8 +273,8 @@ __global__ __launch_bounds__(GQ_ROW_THREADS) void k_gptq_block(
         qc = fmin(fmax(qc, -128.0), 127.0);
         q[n * K + i] = (int8_t)(int)qc;
         sum += (int)qc;
-        const double e = __ddiv_rn(__dsub_rn(col, __dmul_rn(qc, s)), LA[(int64_t)i * K + i]);
-        for (int u = t; u < B; ++u) w1[u] = dsub_mul(w1[u], e, LA[(int64_t)(i1 + u) * K + i]);
+        const double e = __ddiv_rn(__dsub_rn(col, __dmul_rn(qc, s)), U[(int64_t)i * K + i]);
+        for (int u = t; u < B; ++u) w1[u] = dsub_mul(w1[u], e, U[(int64_t)i * K + i1 + u]);
         err[n * GQ_BLOCK_MAX + t] = e;
     }
     if (wsum) wsum[n] = (i1 == 0 ? 0 : wsum[n]) + sum;
@@ -260,20 +282,20 @@ __global__ __launch_bounds__(GQ_ROW_THREADS) void k_gptq_block(
 
 // w[n, j] -= sum_{t ascending} err[n, t] * U[i1 + t, j] for j >= i2.
 __global__ __launch_bounds__(128) void k_gptq_update(double* __restrict__ w,
-                                                     const double* __restrict__ LA,
+                                                     const double* __restrict__ U,
                                                      const double* __restrict__ err, int64_t N,
                                                      int K, int i1, int i2) {
     const int j = i2 + blockIdx.x * 128 + threadIdx.x;
     __shared__ double e[GQ_BLOCK_MAX];
     const int B = i2 - i1;
-    const double* la = LA + (int64_t)(j < K ? j : 0) * K + i1;   // U[i1 + t, j] = LA[j, i1 + t]
+    const double* ut = U + (int64_t)i1 * K + (j < K ? j : 0);    // U[i1 + t, j] at ut[t * K]
     for (int64_t n = blockIdx.y; n < N; n += gridDim.y) {
         __syncthreads();                                 // e[] of the previous row is consumed
         for (int t = threadIdx.x; t < B; t += 128) e[t] = err[n * GQ_BLOCK_MAX + t];
         __syncthreads();
         if (j >= K) continue;
         double p = 0.0;
-        for (int t = 0; t < B; ++t) p = __dadd_rn(p, __dmul_rn(e[t], la[t]));
+        for (int t = 0; t < B; ++t) p = __dadd_rn(p, __dmul_rn(e[t], ut[(int64_t)t * K]));
         w[n * K + j] = __dsub_rn(w[n * K + j], p);
     }
 }
@@ -301,23 +323,19 @@ GptqPlan plan_gptq(int64_t N, int64_t K) {
     p.buf2 = up(p.buf1 + kk);
     p.w = up(p.buf2 + kk);
     p.err = up(p.w + (size_t)N * K * sizeof(double));
-    p.col = up(p.err + (size_t)N * GQ_BLOCK_MAX * sizeof(double));
-    p.dead = up(p.col + (size_t)K * sizeof(double));
+    p.dead = up(p.err + (size_t)N * GQ_BLOCK_MAX * sizeof(double));
     p.bytes = up(p.dead + (size_t)K);
     return p;
 }
 
 bool gptq_block_ok(int64_t block) { return block >= 1 && block <= GQ_BLOCK_MAX; }
 
-// Lower Cholesky factor of T (consumed) into L; `col` is a K-vector of scratch.
-static cudaError_t chol(double* T, double* L, double* col, int K, cudaStream_t st, int* status) {
+// Lower Cholesky factor of T (consumed) into L: one launch per pivot.
+static cudaError_t chol(double* T, double* L, int K, cudaStream_t st, int* status) {
     for (int k = 0; k < K; ++k) {
-        k_chol_col<<<(unsigned)((K - k + 255) / 256), 256, 0, st>>>(T, L, col, K, k, status);
         const int m = K - k - 1;
-        if (m > 0) {
-            const unsigned t = (unsigned)((m + 31) / 32);
-            k_chol_update<<<dim3(t, t), 256, 0, st>>>(T, col, K, k);
-        }
+        const unsigned t = (unsigned)(m > 0 ? (m + 31) / 32 : 1);
+        k_chol_step<<<dim3(t, t), 256, 0, st>>>(T, L, K, k, status);
     }
     return cudaGetLastError();
 }
@@ -333,7 +351,6 @@ cudaError_t launch_gptq_int8(const float* W, const double* H, int64_t N, int K, 
     double* w = reinterpret_cast<double*>(base + p.w);
     double* err = reinterpret_cast<double*>(base + p.err);
     unsigned char* dead = base + p.dead;
-    double* col = reinterpret_cast<double*>(base + p.col);
     const int64_t kk = (int64_t)K * K;
     const int cap = 8 * num_sms;
     // scales of the original rows (weight_int8's grid); q and wsum are rewritten below
@@ -342,20 +359,21 @@ cudaError_t launch_gptq_int8(const float* W, const double* H, int64_t N, int K, 
     // A = damped H in b0; L = chol(A) in b1 (A is consumed as the trailing matrix)
     k_gptq_copy<<<grid_for(kk, 256, cap), 256, 0, st>>>(H, K, b0);
     k_gptq_diag<<<1, 256, 0, st>>>(H, K, damp, b0, dead);
-    if ((e = chol(b0, b1, col, K, st, status)) != cudaSuccess) return e;
+    if ((e = chol(b0, b1, K, st, status)) != cudaSuccess) return e;
     // Li = L^-1 in b2, running sums in b0 (zeroed)
     if ((e = cudaMemsetAsync(b0, 0, (size_t)kk * sizeof(double), st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(b2, 0, (size_t)kk * sizeof(double), st)) != cudaSuccess) return e;
     for (int k = 0; k < K; ++k) {
-        k_trinv_row<<<(unsigned)((k + 256) / 256), 256, 0, st>>>(b1, b0, b2, K, k);
-        if (k + 1 < K)
-            k_trinv_update<<<dim3((unsigned)((k + 32) / 32), (unsigned)((K - k - 1 + 31) / 32)),
-                             256, 0, st>>>(b1, b0, b2, K, k);
+        const int rows = K - k - 1;
+        k_trinv_step<<<dim3((unsigned)((k + 32) / 32), (unsigned)(rows > 0 ? (rows + 31) / 32 : 1)),
+                       256, 0, st>>>(b1, b0, b2, K, k);
     }
     // H^-1 = Li^T Li in b1, then its lower factor LA in b0 (U = LA^T)
     const unsigned t = (unsigned)((K + GQ_TILE - 1) / GQ_TILE);
     k_inv_gram<<<dim3(t, t), GQ_TILE * GQ_ROWS, 0, st>>>(b2, K, b1);
-    if ((e = chol(b1, b0, col, K, st, status)) != cudaSuccess) return e;
+    if ((e = chol(b1, b0, K, st, status)) != cudaSuccess) return e;
+    // U = LA^T in b2 (Li is no longer needed)
+    k_transpose<<<dim3(t, t), 256, 0, st>>>(b0, K, b2);
     // the column blocks
     k_gptq_init_w<<<grid_for(N * K, 256, cap), 256, 0, st>>>(W, dead, N, K, w);
     const size_t smem = (size_t)GQ_ROW_THREADS * (block + 1) * sizeof(double);
@@ -363,11 +381,11 @@ cudaError_t launch_gptq_int8(const float* W, const double* H, int64_t N, int K, 
     for (int i1 = 0; i1 < K; i1 += block) {
         const int i2 = i1 + block < K ? i1 + block : K;
         k_gptq_block<<<(unsigned)((N + GQ_ROW_THREADS - 1) / GQ_ROW_THREADS), GQ_ROW_THREADS,
-                       smem, st>>>(w, b0, s_w, N, K, i1, i2, q, err, wsum);
+                       smem, st>>>(w, b2, s_w, N, K, i1, i2, q, err, wsum);
         if (i2 < K)
             k_gptq_update<<<dim3((unsigned)((K - i2 + 127) / 128),
                                  (unsigned)(N < 65535 ? N : 65535)),
-                            128, 0, st>>>(w, b0, err, N, K, i1, i2);
+                            128, 0, st>>>(w, b2, err, N, K, i1, i2);
     }
     return cudaGetLastError();
 }

@@ -106,7 +106,7 @@ cudaError_t launch_q4_gemm_tc(const uint16_t* wb, const uint16_t* xz, const floa
 
 // k_gptq.cu
 struct GptqPlan {
-    size_t buf0, buf1, buf2, w, err, col, dead, bytes;   // byte offsets in the workspace
+    size_t buf0, buf1, buf2, w, err, dead, bytes;     // byte offsets in the workspace
 };
 GptqPlan plan_gptq(int64_t N, int64_t K);
 bool gptq_block_ok(int64_t block);
