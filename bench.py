@@ -784,9 +784,7 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 activations; N(0,0.02^2) fp32 weights "
                 "quantized per channel on the GPU)",
-        "config": {"workload": "W8A16 decode sweep: bf16 x [M,K] (M in 1,4,16) times int8 "
-                               "W [N,K], (K,N) in (960,2560),(2048,8192),(4096,11008),"
-                               "(4096,32000); bf16 out",
+        "config": {"workload": SWEEP_WORKLOAD,
                    "step": "12 GEMV launches (every shape x M), " +
                            ("launched eagerly" if args.eager else "one CUDA graph"),
                    "bytes_per_step": sweep.step_bytes,
@@ -825,6 +823,10 @@ def run_ours(args):
     dist.close()
 
 
+SWEEP_WORKLOAD = ("W8A16 decode sweep: bf16 x [M,K] (M in 1,4,16) times int8 W [N,K], (K,N) in "
+                  "(960,2560),(2048,8192),(4096,11008),(4096,32000); bf16 out")
+
+
 def run_reference(args):
     """The reference arm: the CPU oracle as it stands, on the host cores, on the same metric
     (W8A16 decode GB/s).  Each step is a bounded sample of the workload: the M = 1 case of
@@ -861,8 +863,9 @@ def run_reference(args):
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(el * 1e3 / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": "W8A16 decode sweep (M=1 sample)",
-                                        "bytes_per_step": step_bytes},
+        "data": "synthetic", "config": {"workload": SWEEP_WORKLOAD, "sample": sample,
+                                        "bytes_per_step": step_bytes,
+                                        "parallelism": "replicas x1 (rank 0 only)"},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
