@@ -649,3 +649,12 @@ def test_gptq_dead_columns_and_error_reduction():
         d = W.astype(np.float64) - codes.astype(np.float64) * sc.astype(np.float64)[:, None]
         return float(np.einsum("nk,kl,nl->", d, H, d))
     assert qerr(q, s) < 0.8 * qerr(rq, rs)
+
+
+def test_minmax_is_numpy_min_max():
+    """act_observer's statistics (SmolVLM q8 page): the min and max of everything observed."""
+    x = wl.normal((37, 51), 3.0, seed=48).numpy()
+    x[5, 7] = -1e30
+    x[36, 50] = 7e29
+    assert oracle.minmax(x) == (float(x.min()), float(x.max()))
+    assert oracle.minmax(np.full((3,), 2.5, np.float32)) == (2.5, 2.5)
