@@ -133,6 +133,60 @@ def test_argument_validation_before_device(L):
                           None) == q8.Q8_ERR_WORKSPACE
     assert L.q8_gptq_int8(good, None, 8, 64, 0.01, 128, good, good, None, good, ws_g,
                           None) == q8.Q8_ERR_NULL
+    # static activation codes, the first-pass observer
+    qpp = ctypes.byref(qp)
+    bad_qpp = ctypes.byref(bad_qp)
+    assert L.q8_quantize_static(good, -1, 64, qp, None, good, None, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_quantize_static(good, 4, 60, qp, None, good, None, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_quantize_static(good, 4, 64, bad_qp, None, good, None, None) == q8.Q8_ERR_ARG
+    assert L.q8_quantize_static(good, 4, 64, qp, bad_qpp, good, good, None) == q8.Q8_ERR_ARG
+    assert L.q8_quantize_static(good, 0, 64, qp, None, None, None, None) == q8.Q8_OK
+    assert L.q8_quantize_static(good, 4, 64, qp, qpp, good, None, None) == q8.Q8_ERR_NULL
+    assert L.q8_quantize_static(odd, 4, 64, qp, None, good, None, None) == q8.Q8_ERR_ALIGN
+    assert L.q8_observe_minmax(good, -1, good, 1, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_observe_minmax(good, 8, None, 1, None) == q8.Q8_ERR_NULL
+    assert L.q8_observe_minmax(None, 8, good, 1, None) == q8.Q8_ERR_NULL
+    assert L.q8_observe_minmax(None, 0, good, 0, None) == q8.Q8_OK
+    assert L.q8_observe_minmax(odd, 8, good, 1, None) == q8.Q8_ERR_ALIGN
+    # 8da4w linear
+    assert L.q8_linear_dq8ca_q4gsw(good, good, good, 48, good, 1, 16, 256, good, 1 << 20,
+                                   None) == q8.Q8_ERR_ARG
+    assert L.q8_linear_dq8ca_q4gsw(good, good, good, 128, good, 1, 0, 256, good, 1 << 20,
+                                   None) == q8.Q8_ERR_SHAPE
+    assert L.q8_linear_dq8ca_q4gsw(good, good, good, 64, good, 1, 16, 192, good, 1 << 20,
+                                   None) == q8.Q8_ERR_SHAPE
+    assert L.q8_linear_dq8ca_q4gsw(good, good, good, 256, good, 1, 16, 384, good, 1 << 20,
+                                   None) == q8.Q8_ERR_SHAPE
+    assert L.q8_linear_dq8ca_q4gsw(good, good, good, 128, good, 0, 16, 256, None, 0,
+                                   None) == q8.Q8_OK
+    assert L.q8_linear_dq8ca_q4gsw(None, good, good, 128, good, 1, 16, 256, good, 1 << 20,
+                                   None) == q8.Q8_ERR_NULL
+    assert L.q8_linear_dq8ca_q4gsw(good, good, good, 128, odd, 1, 16, 256, good, 1 << 20,
+                                   None) == q8.Q8_ERR_ALIGN
+    # int8 GEMM test export
+    assert L.q8_gemm_s8s8_s32(good, good, good, 4, 0, 256, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_gemm_s8s8_s32(good, good, good, 4, 16, 64, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_gemm_s8s8_s32(good, good, good, 0, 16, 256, None) == q8.Q8_OK
+    assert L.q8_gemm_s8s8_s32(good, None, good, 4, 16, 256, None) == q8.Q8_ERR_NULL
+    assert L.q8_gemm_s8s8_s32(good, good, odd, 4, 16, 256, None) == q8.Q8_ERR_ALIGN
+    # built-in scratch too small for these codes (decided on the host)
+    assert L.q8_linear_w8a8_noalloc(good, qp, None, good, good, good, good, 8192, 16, 4096,
+                                    None) == q8.Q8_ERR_WORKSPACE
+    # digit-plane W8A16
+    assert L.q8_linear_w8a16_planes(good, good, good, good, 7, 1, 16, 64, good, 1 << 20,
+                                    None) == q8.Q8_ERR_ARG
+    assert L.q8_linear_w8a16_planes(good, good, good, good, q8.Q8_F32, 1, 16, 40, good,
+                                    1 << 20, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_linear_w8a16_planes(good, good, good, good, q8.Q8_F32, 0, 16, 64, None, 0,
+                                    None) == q8.Q8_OK
+    assert L.q8_linear_w8a16_planes(good, None, good, good, q8.Q8_F32, 1, 16, 64, good,
+                                    1 << 20, None) == q8.Q8_ERR_NULL
+    assert L.q8_linear_w8a16_planes(odd, good, good, good, q8.Q8_F32, 1, 16, 64, good,
+                                    1 << 20, None) == q8.Q8_ERR_ALIGN
+    # bounded-wait self-test
+    assert L.q8_selftest_bounded_wait(100000, None, None) == q8.Q8_ERR_NULL
+    assert L.q8_selftest_bounded_wait(10, good, None) == q8.Q8_ERR_ARG
+    assert L.q8_selftest_bounded_wait(3000000000, good, None) == q8.Q8_ERR_ARG
     mmp = _p(0x10000)
     assert L.q8_observe_residual_minmax(good, 64, bad_qp, mmp, 1, None) == q8.Q8_ERR_ARG
     assert L.q8_observe_residual_minmax(good, -1, qp, mmp, 1, None) == q8.Q8_ERR_SHAPE
