@@ -49,6 +49,7 @@ def lib() -> ctypes.CDLL:
         L.q8o_quantize_weight_q4gs.argtypes = [_vp, _i64, _i64, ctypes.c_int, _vp, _vp]
         L.q8o_linear_dq8ca_q4gsw.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_int,
                                              _i64, _i64, _i64, _vp, _i64, _vp, _vp]
+        L.q8o_q4gs_zero_fold.argtypes = [_vp, _vp, ctypes.c_int, _i64, _i64, _vp]
         L.q8o_gemm_s8s8_s32.argtypes = [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp]
         L.q8o_gram_rows.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp]
         L.q8o_gptq_hinv.restype = ctypes.c_int
@@ -256,6 +257,17 @@ def linear_dq8ca_q4gsw(xq, s, z, q4, gs, G, rows=None):
     lib().q8o_linear_dq8ca_q4gsw(_p(xq), _p(s), _p(z), _p(q4), _p(gs), int(G), M, N, K,
                                  _p(r), R, _p(y), _p(a))
     return y, a
+
+
+def q4gs_zero_fold(q4, gs, G):
+    """Zero-point fold of an 8da4w weight: c [N] fp32, the row sums of the dequantized
+    weight (sum_g gs[n,g] * sum_{k in g} q4[n,k], fp64 over g ascending, one fp32 rounding)."""
+    q4 = _c(q4, np.uint8)
+    gs = _c(gs, np.float32)
+    N, K2 = q4.shape
+    c = np.empty(N, np.float32)
+    lib().q8o_q4gs_zero_fold(_p(q4), _p(gs), int(G), N, 2 * K2, _p(c))
+    return c
 
 
 def gemm_s8s8_s32(a, b, rows=None):

@@ -436,6 +436,29 @@ void q8o_linear_dq8ca_q4gsw(const int8_t* xq, const float* s, const int32_t* z,
     }
 }
 
+/* Zero-point fold of the 8da4w weight.  In [ET-21229]'s
+ *     out[m,n] = s[m] * sum_k (xq[m,k] - z[m]) * dequant(w)[n,k]
+ * the zero-point part separates as z[m] * c[n] with c[n] = sum_k dequant(w)[n,k], the row
+ * sum of the dequantized weight:
+ *     c[n] = sum_g gs[n,g] * (sum_{k in g} q4[n,k])
+ * Inner sums exact (int64); each product gs * S is exact in fp64 (24 + 12 bits); the outer
+ * sum runs over g ascending in fp64, rounded once to fp32 at the end. */
+void q8o_q4gs_zero_fold(const uint8_t* q4, const float* gs, int G, int64_t N, int64_t K,
+                        float* c) {
+    int64_t ng = K / G;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const uint8_t* wr = q4 + n * (K / 2);
+        double acc = 0.0;
+        for (int64_t g = 0; g < ng; ++g) {
+            int64_t part = 0;
+            for (int64_t k = g * G; k < (g + 1) * G; ++k) part += q4_code(wr, k);
+            acc += (double)part * (double)gs[n * ng + g];
+        }
+        c[n] = (float)acc;
+    }
+}
+
 /* ------------------------------------------------ int8 GEMM, int32 out (a8)
  * acc[m,n] = sum_k a[m,k] * b[n,k], exact. */
 void q8o_gemm_s8s8_s32(const int8_t* a, const int8_t* b,

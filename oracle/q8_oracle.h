@@ -44,6 +44,8 @@ void q8o_linear_dq8ca_q4gsw(const int8_t* xq, const float* s, const int32_t* z,
                             int64_t M, int64_t N, int64_t K,
                             const int64_t* rows, int64_t nrows,
                             double* y, double* absum);
+void q8o_q4gs_zero_fold(const uint8_t* q4, const float* gs, int G, int64_t N, int64_t K,
+                        float* c);
 void q8o_gemm_s8s8_s32(const int8_t* a, const int8_t* b,
                        int64_t M, int64_t N, int64_t K,
                        const int64_t* rows, int64_t nrows, int32_t* acc);

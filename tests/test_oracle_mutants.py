@@ -45,6 +45,11 @@ MUTANTS = [
      "acc += (double)gs[n * ng] * (double)part;", ["test_dq8ca_q4gsw_reductions"]),
     ("q4 zero point dropped", "int64_t p = ((int64_t)xr[k] - z[m]) * q4_code(wr, k);",
      "int64_t p = ((int64_t)xr[k]) * q4_code(wr, k);", ["test_dq8ca_q4gsw_reductions"]),
+    ("zero fold drops the group scale", "acc += (double)part * (double)gs[n * ng + g];",
+     "acc += (double)part;", ["test_golden_q4gs_zero_fold"]),
+    ("zero fold skips the last group", "for (int64_t g = 0; g < ng; ++g) {\n            int64_t part = 0;\n            for (int64_t k = g * G; k < (g + 1) * G; ++k) part +=",
+     "for (int64_t g = 0; g < ng - 1; ++g) {\n            int64_t part = 0;\n            for (int64_t k = g * G; k < (g + 1) * G; ++k) part +=",
+     ["test_q4gs_zero_fold_exact_row_sums"]),
     ("bf16 rounding truncates", "double r = nearbyint(ldexp(m, 8));",
      "double r = trunc(ldexp(m, 8));", ["test_round_bf16"]),
     ("full grid clamps at -127",

@@ -73,6 +73,38 @@ def test_golden_q4_groups():
     assert gs[0].tolist() == [float(r[1][0]) for r in rows]
 
 
+def test_golden_q4gs_zero_fold():
+    """The 8da4w zero-point fold c[n] (row sum of the dequantized weight) on hand-worked
+    rows, including a zero group, a negative sum and the final fp32 rounding."""
+    rows = _parse("q4gs_zero_fold_rows.txt")
+    W = np.array([[float(v) for v in r[0]] for r in rows], np.float32)
+    q4, gs = oracle.quantize_weight_q4gs(W, 4)
+    c = oracle.q4gs_zero_fold(q4, gs, 4)
+    for i, r in enumerate(rows):
+        assert Fraction(float(c[i])) == Fraction(r[1][0]), f"row {i}"
+
+
+def test_q4gs_zero_fold_exact_row_sums():
+    """c[n] is the nearest fp32 to the exact rational row sum of gs * code (codes decoded
+    here from the packed bytes), for random weights, both group sizes and zero groups."""
+    W = wl.weight(24, 512, seed=35).numpy()
+    W[3, 64:192] = 0.0
+    W[5] *= 1e-20
+    for G in (32, 128):
+        q4, gs = oracle.quantize_weight_q4gs(W, G)
+        c = oracle.q4gs_zero_fold(q4, gs, G)
+        for n in range(W.shape[0]):
+            exact = Fraction(0)
+            for g in range(512 // G):
+                S = 0
+                for k in range(g * G, (g + 1) * G):
+                    b = int(q4[n, k // 2])
+                    nib = (b >> 4) if k & 1 else (b & 0xF)
+                    S += nib - 16 if nib >= 8 else nib
+                exact += Fraction(float(gs[n, g])) * S
+            assert Fraction(float(c[n])) == rn32(exact), f"G={G} row {n}"
+
+
 # ------------------------------------------------------ weight codes, brute force
 
 
