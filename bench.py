@@ -513,26 +513,6 @@ def bench_w8a8_prefill(dev, peaks, reps=5):
     return out
 
 
-def planes_case_times(sweep: W8A16Sweep):
-    """The sweep's cases through q8_linear_w8a16_planes (int8 tensor cores over exact digit
-    planes of the activations), timed like the headline's per-case times."""
-    q8 = sweep.q8
-    ws = {}
-
-    def launch(i, M, copy):
-        sh, copies, s = sweep.shapes[i]
-        if (i, M) not in ws:
-            n = q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A16_PLANES, M, sh.N, sh.K)
-            ws[(i, M)] = torch.zeros(max(n, 16), dtype=torch.uint8, device=copies[0].device)
-        q8.q8_linear_w8a16_planes(sweep.xs[(i, M)], copies[copy], s, ws[(i, M)],
-                                  y=sweep.ys[(i, M)])
-
-    out = per_case_times(sweep, launch=launch)
-    total_b = sum(w8a16_bytes(c["M"], c["N"], c["K"]) for c in out)
-    total_us = sum(c["us"] for c in out)
-    return {"cases": out, "GBps_sum_of_cases": round(total_b / total_us / 1e3, 1)}
-
-
 def bias_case_times(sweep: W8A16Sweep):
     """The sweep's cases through q8_linear_w8a16 with an fp32 bias [N] (4 N more bytes),
     timed like the headline's per-case times."""
@@ -808,7 +788,6 @@ def run_ours(args):
         result["cpu_baseline"] = cpu_baseline_w8a16(sweep)
     if dist.rank == 0 and not args.no_paths:
         result["paths"] = {
-            "w8a16_planes": planes_case_times(sweep),
             "w8a16_bias": bias_case_times(sweep),
             "w8a8_static_k960": bench_w8a8_paths(dev),
             "w8a8_prefill_m4096": bench_w8a8_prefill(dev, peaks),

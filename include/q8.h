@@ -36,6 +36,11 @@
  *   - The device must be sm_100 (B200); other devices return
  *     Q8_ERR_UNSUPPORTED_ARCH.  There is no CPU fallback.
  *   - Calls that overlap on the GPU may share nothing they write.
+ *   - Per device, the first call made with that device current records the device's
+ *     architecture and SM count and the device addresses of the library's own device
+ *     variables (its status word, the built-in scratch of q8_linear_w8a8_noalloc); later
+ *     calls reuse them.  After cudaDeviceReset those addresses are stale: do not call the
+ *     library again in a process that has reset a device it used.
  */
 #ifndef Q8_H
 #define Q8_H
@@ -59,6 +64,11 @@ typedef enum {
     Q8_ERR_DEVICE = 8             /* a kernel recorded a device-side failure           */
 } q8_status;
 
+/* Names of the same two codes in the boundary table this header implements: an invalid
+ * dtype is one case of Q8_ERR_ARG, an expired bounded wait one case of Q8_ERR_DEVICE. */
+#define Q8_ERR_DTYPE Q8_ERR_ARG
+#define Q8_ERR_DEVICE_TIMEOUT Q8_ERR_DEVICE
+
 typedef enum { Q8_F32 = 0, Q8_BF16 = 1 } q8_dtype;
 
 /* Static per-tensor affine activation parameters: real x ~ (code - zero_point) * scale,
@@ -72,7 +82,6 @@ typedef struct {
 typedef enum {
     Q8_OP_LINEAR_W8A8 = 0,
     Q8_OP_LINEAR_DQ8CA_Q4GSW = 1,
-    Q8_OP_LINEAR_W8A16_PLANES = 2,  /* q8_linear_w8a16_planes */
     Q8_OP_GPTQ_INT8 = 3             /* q8_gptq_int8 (M unused, extra = block) */
 } q8_op;
 
@@ -173,10 +182,18 @@ q8_status q8_qparams_from_minmax(float mn, float mx, q8_qparams* out);
  *     code    = clamp(round(W / gs[n,g]), -7, 7)   (a zero-scale group: gs = 1, codes 0)
  * packed two per byte: byte k/2 of row n holds code k in its low nibble (k even)
  * or its high nibble (k odd).
- *   W device fp32 [N, K]; q4 device uint8 [N, K/2]; gs device fp32 [N, K/G].
- *   G in {32, 64, 128, 256} and K % G == 0. */
+ * When c != NULL it also receives the zero-point fold of each row: [ET-21229] defines
+ * out[m,n] = s[m] * sum_k (xq[m,k] - z[m]) * dequant(w)[n,k], whose zero-point part is
+ * z[m] * c[n] with c[n] the row sum of the dequantized weight,
+ *     c[n] = sum_g gs[n,g] * sum_{k in g} code[n,k]
+ * (exact products, an fp64 sum over g in ascending order, one rounding to fp32), so a
+ * caller can apply the zero point once per output instead of per element.
+ *   W device fp32 [N, K]; q4 device uint8 [N, K/2]; gs device fp32 [N, K/G];
+ *   c device fp32 [N] (nullable; 4-byte aligned).
+ *   G in {32, 64, 128, 256} and K % G == 0.
+ * Codes, scales and c are bit-identical to the CPU reference definition. */
 q8_status q8_quantize_weight_q4gs(const float* W, int64_t N, int64_t K, int G,
-                                  uint8_t* q4, float* gs, void* stream);
+                                  uint8_t* q4, float* gs, float* c, void* stream);
 
 /* -------------------------------------------------------------------- linears */
 
@@ -201,31 +218,6 @@ q8_status q8_linear_w8a16_bias(const void* x, const int8_t* q, const float* s_w,
                                const float* bias, void* y, q8_dtype yt, int64_t M, int64_t N,
                                int64_t K, void* stream);
 
-/* W8A16, same definition and arguments as q8_linear_w8a16, computed on the int8 tensor
- * cores for decode-sized M (1..16): the bf16 activations are rewritten once per call as
- * exact int8 digit planes (per row: base-128 digits of the values on a common power of
- * two), every plane is multiplied with the int8 weight by tcgen05.mma.kind::i8 (exact
- * int32), and the planes are recombined in fp64 before the scale -- the dot product is
- * rounded about once, so the result meets the same bound as q8_linear_w8a16 with room
- * to spare.  A row whose values span more than the plane budget (jcap planes of 7 bits:
- * 80 for M = 1, 20 for M = 4, 10 for M = 16) keeps its smallest elements, and any
- * non-finite ones, out of the planes and adds their products in the epilogue (slower,
- * same accuracy; infinities and NaNs propagate as in IEEE arithmetic).  Its weight stream
- * is conversion-free, but building the planes costs a grid-wide handshake per call, so
- * q8_linear_w8a16 is faster at the sizes measured; this form is for callers that want
- * the tighter rounding.
- *   workspace: at least q8_workspace_bytes(Q8_OP_LINEAR_W8A16_PLANES, M, N, K, 0) bytes,
- *   16-byte aligned, ZERO-FILLED before its first use and then left to this function (it
- *   keeps a call counter and per-call flags there, so calls captured in a CUDA graph may be
- *   replayed); one workspace must not serve two calls that may run at the same time, nor
- *   any other operation.  After a call that returned an error status, zero-fill it again.  The kernel keeps one CTA per SM resident and its CTAs wait on each
- *   other (bounded): it must not share the GPU with a limit on SMs.
- *   Q8_ERR_WORKSPACE if the workspace is NULL or too small.  M > 16 (workspace size 0)
- *   runs q8_linear_w8a16. */
-q8_status q8_linear_w8a16_planes(const void* x, const int8_t* q, const float* s_w,
-                                 void* y, q8_dtype yt, int64_t M, int64_t N, int64_t K,
-                                 void* workspace, size_t ws_bytes, void* stream);
-
 /* W8A8: static per-tensor int8 activations times per-channel int8 weights
  * ([SmolVLM-Q8] Q8Linear.forward; the delegated op takes weight_sums):
  *     acc1[m,n] = sum_k xq1[m,k] q[n,k]     (int32, exact)
@@ -238,9 +230,10 @@ q8_status q8_linear_w8a16_planes(const void* x, const int8_t* q, const float* s_
  *   workspace: device scratch of at least q8_workspace_bytes(Q8_OP_LINEAR_W8A8, M, N,
  *   K, second != NULL) bytes (may be NULL when that is 0); its contents on entry do not
  *   matter and are overwritten.
- * Decode-sized M runs as a GEMV with the activation codes computed in-kernel; larger M
- * quantizes x into the workspace and runs a tcgen05 int8 GEMM (int32 accumulators in
- * tensor memory) with the zero-point term and both scales in its epilogue. */
+ * A first kernel writes the activation codes (q8_quantize_static) to the workspace; then
+ * decode-sized M (<= 16) runs as a GEMV on the warp-level int8 MMA, larger M as a tcgen05
+ * int8 GEMM (int32 accumulators in tensor memory) with the zero-point term and both
+ * scales in its epilogue. */
 q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* second,
                          const int8_t* q, const int32_t* wsum, const float* s_w,
                          float* y, int64_t M, int64_t N, int64_t K,
@@ -306,9 +299,9 @@ q8_status q8_gptq_int8(const float* W, const double* H, int64_t N, int64_t K, do
                        size_t ws_bytes, void* stream);
 
 /* Host.  Workspace bytes a linear needs for these sizes (0 if none).  `extra` is
- * "two-pass" (0/1) for Q8_OP_LINEAR_W8A8, G for Q8_OP_LINEAR_DQ8CA_Q4GSW and unused (0)
- * for Q8_OP_LINEAR_W8A16_PLANES (whose size also depends on the current device's SM
- * count).
+ * "two-pass" (0/1) for Q8_OP_LINEAR_W8A8, G for Q8_OP_LINEAR_DQ8CA_Q4GSW and the block
+ * size for Q8_OP_GPTQ_INT8.  The 8da4w size for 17..64 rows also depends on the current
+ * device's SM count.
  * Returns 0 for invalid arguments as well; the linear then reports the error. */
 size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra);
 

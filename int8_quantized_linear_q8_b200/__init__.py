@@ -24,7 +24,7 @@ Q8_OK = 0
 Q8_ERR_NULL, Q8_ERR_SHAPE, Q8_ERR_ALIGN, Q8_ERR_ARG = 1, 2, 3, 4
 Q8_ERR_UNSUPPORTED_ARCH, Q8_ERR_LAUNCH, Q8_ERR_WORKSPACE, Q8_ERR_DEVICE = 5, 6, 7, 8
 Q8_F32, Q8_BF16 = 0, 1
-Q8_OP_LINEAR_W8A8, Q8_OP_LINEAR_DQ8CA_Q4GSW, Q8_OP_LINEAR_W8A16_PLANES = 0, 1, 2
+Q8_OP_LINEAR_W8A8, Q8_OP_LINEAR_DQ8CA_Q4GSW = 0, 1
 Q8_OP_GPTQ_INT8 = 3
 Q8_GRID_SYM127, Q8_GRID_FULL128 = 0, 1
 _GRIDS = {"sym127": Q8_GRID_SYM127, "full128": Q8_GRID_FULL128}
@@ -35,7 +35,7 @@ SYMBOLS = (
     "q8_quantize_static", "q8_observe_minmax", "q8_qparams_from_minmax",
     "q8_quantize_weight_q4gs", "q8_linear_w8a16", "q8_linear_w8a8", "q8_linear_dq8ca_q4gsw",
     "q8_workspace_bytes", "q8_gemm_s8s8_s32", "q8_last_device_status",
-    "q8_linear_w8a8_noalloc", "q8_selftest_bounded_wait", "q8_linear_w8a16_planes",
+    "q8_linear_w8a8_noalloc", "q8_selftest_bounded_wait",
     "q8_quantize_weight_grid", "q8_linear_w8a16_bias", "q8_linear_w8a8_bias",
     "q8_observe_residual_minmax", "q8_hessian_accumulate", "q8_gptq_int8",
 )
@@ -92,14 +92,11 @@ def _lib() -> ctypes.CDLL:
     L.q8_qparams_from_minmax.argtypes = [ctypes.c_float, ctypes.c_float,
                                          ctypes.POINTER(q8_qparams)]
     L.q8_quantize_weight_q4gs.restype = st
-    L.q8_quantize_weight_q4gs.argtypes = [_vp, _i64, _i64, st, _vp, _vp, _vp]
+    L.q8_quantize_weight_q4gs.argtypes = [_vp, _i64, _i64, st, _vp, _vp, _vp, _vp]
     L.q8_linear_w8a16.restype = st
     L.q8_linear_w8a16.argtypes = [_vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp]
     L.q8_linear_w8a16_bias.restype = st
     L.q8_linear_w8a16_bias.argtypes = [_vp, _vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp]
-    L.q8_linear_w8a16_planes.restype = st
-    L.q8_linear_w8a16_planes.argtypes = [_vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp, _sz,
-                                         _vp]
     L.q8_linear_w8a8.restype = st
     L.q8_linear_w8a8.argtypes = [_vp, q8_qparams, ctypes.POINTER(q8_qparams), _vp, _vp, _vp,
                                  _vp, _i64, _i64, _i64, _vp, _sz, _vp]
@@ -256,17 +253,24 @@ def q8_qparams_from_minmax(mn: float, mx: float) -> Tuple[float, int]:
     return float(out.scale), int(out.zero_point)
 
 
-def q8_quantize_weight_q4gs(W: torch.Tensor, G: int, q4=None, gs=None, stream=None):
-    """int4 group-symmetric codes (packed, low nibble = even k) -> (q4 [N,K/2], gs [N,K/G])."""
+def q8_quantize_weight_q4gs(W: torch.Tensor, G: int, q4=None, gs=None, stream=None,
+                            c=None, want_c: bool = False):
+    """int4 group-symmetric codes (packed, low nibble = even k) -> (q4 [N,K/2], gs [N,K/G]);
+    with want_c (or a `c` tensor) also the zero-point fold c [N] (row sums of the
+    dequantized weight) -> (q4, gs, c)."""
     N, K = W.shape
     _need(W, "W", torch.float32, (N, K))
     if G <= 0 or K % G or K % 2:
         raise ValueError("K must be a multiple of G")
     q4 = _out(q4, "q4", torch.uint8, (N, K // 2), W.device)
     gs = _out(gs, "gs", torch.float32, (N, K // G), W.device)
+    fold = want_c or c is not None
+    if fold:
+        c = _out(c, "c", torch.float32, (N,), W.device)
     _check(_lib().q8_quantize_weight_q4gs(_ptr(W), N, K, int(G), _ptr(q4), _ptr(gs),
-                                          _stream(stream)), "q8_quantize_weight_q4gs")
-    return q4, gs
+                                          _ptr(c) if fold else None, _stream(stream)),
+           "q8_quantize_weight_q4gs")
+    return (q4, gs, c) if fold else (q4, gs)
 
 
 # ---------------------------------------------------------------------------- linears
@@ -306,36 +310,6 @@ def q8_linear_w8a16(x: torch.Tensor, q: torch.Tensor, s_w: torch.Tensor, y=None,
     else:
         _check(_lib().q8_linear_w8a16_bias(_ptr(x), _ptr(q), _ptr(s_w), _ptr(bias), _ptr(y), yt,
                                            M, N, K, _stream(stream)), "q8_linear_w8a16_bias")
-    return y
-
-
-def q8_w8a16_planes_workspace(M: int, N: int, K: int, device=None) -> Optional[torch.Tensor]:
-    """A zero-filled workspace for q8_linear_w8a16_planes (None when the sizes need none).
-    Keep one per stream: the call leaves per-call flags in it."""
-    nbytes = q8_workspace_bytes(Q8_OP_LINEAR_W8A16_PLANES, M, N, K)
-    if nbytes == 0:
-        return None
-    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
-
-
-def q8_linear_w8a16_planes(x: torch.Tensor, q: torch.Tensor, s_w: torch.Tensor, workspace,
-                           y=None, out_dtype: torch.dtype = torch.bfloat16,
-                           stream=None) -> torch.Tensor:
-    """q8_linear_w8a16 on the int8 tensor cores over exact digit planes of x; `workspace`
-    from q8_w8a16_planes_workspace (zero-filled once, not shared by concurrent calls)."""
-    M, K = x.shape
-    N = q.shape[0]
-    _need(x, "x", torch.bfloat16, (M, K))
-    _need(q, "q", torch.int8, (N, K))
-    _need(s_w, "s_w", torch.float32, (N,))
-    if out_dtype not in (torch.bfloat16, torch.float32):
-        raise ValueError("out_dtype must be bfloat16 or float32")
-    y = _out(y, "y", out_dtype, (M, N), x.device)
-    yt = Q8_BF16 if y.dtype == torch.bfloat16 else Q8_F32
-    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_lib().q8_linear_w8a16_planes(_ptr(x), _ptr(q), _ptr(s_w), _ptr(y), yt, M, N, K,
-                                         _ptr(workspace), wsb, _stream(stream)),
-           "q8_linear_w8a16_planes")
     return y
 
 

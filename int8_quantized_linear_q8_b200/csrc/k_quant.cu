@@ -366,6 +366,49 @@ __global__ __launch_bounds__(256) void k_quantize_weight_q4gs(const float* __res
     if (lane == 0) gs[g] = scale;
 }
 
+// Zero-point fold of the 8da4w weight (pytorch/executorch PR #21229, linear_dq8ca_q4gsw:
+// out = s * sum_k (xq - z) * dequant(w), whose zero-point part is z * c[n] with c[n] the
+// row sum of the dequantized weight):
+//     c[n] = sum_g gs[n,g] * S[n,g],   S[n,g] = sum of the group's signed 4-bit codes.
+// One warp per row.  Lane j computes the exact fp64 product for group base + j (24-bit
+// scale times a code sum of at most 12 bits); the warp then adds the 32 products in group
+// order (every lane runs the same sequential chain), so the fp64 sum runs over g ascending
+// and is rounded once to fp32.
+__global__ __launch_bounds__(256) void k_q4gs_zero_fold(const uint8_t* __restrict__ q4,
+                                                        const float* __restrict__ gs, int G,
+                                                        int64_t N, int K,
+                                                        float* __restrict__ c) {
+    const int lane = threadIdx.x & 31;
+    const int64_t n = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (n >= N) return;
+    const int ng = K / G;
+    const uint8_t* row = q4 + n * (int64_t)(K / 2);
+    const float* grow = gs + n * (int64_t)ng;
+    double acc = 0.0;
+    for (int base = 0; base < ng; base += 32) {
+        const int g = base + lane;
+        double p = 0.0;
+        if (g < ng) {
+            // G / 2 bytes per group, a multiple of 16: whole 16-byte loads
+            const uint4* src = reinterpret_cast<const uint4*>(row + (int64_t)g * (G / 2));
+            int S = 0;
+            for (int i = 0; i < G / 32; ++i) {
+                const uint4 v = __ldg(src + i);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int b = 0; b < 8; ++b)
+                        S += (int)(w[j] << (28 - 4 * b)) >> 28;     // sign-extended nibble
+            }
+            p = (double)__ldg(grow + g) * (double)S;                 // exact
+        }
+        const int cnt = ng - base < 32 ? ng - base : 32;
+        for (int j = 0; j < cnt; ++j) acc = __dadd_rn(acc, __shfl_sync(0xffffffffu, p, j));
+    }
+    if (lane == 0) c[n] = __double2float_rn(acc);
+}
+
 // ---------------------------------------------------------------------- launchers
 cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int full, int8_t* q,
                                    float* s_w, int32_t* wsum, cudaStream_t st) {
@@ -425,6 +468,12 @@ cudaError_t launch_quantize_weight_q4gs(const float* W, int64_t N, int K, int G,
         case 256: k_quantize_weight_q4gs<8><<<blocks, 256, 0, st>>>(W, groups, K, q4, gs); break;
         default: return cudaErrorInvalidValue;
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_q4gs_zero_fold(const uint8_t* q4, const float* gs, int G, int64_t N, int K,
+                                  float* c, cudaStream_t st) {
+    k_q4gs_zero_fold<<<(unsigned)((N + 7) / 8), 256, 0, st>>>(q4, gs, G, N, K, c);
     return cudaGetLastError();
 }
 

@@ -102,6 +102,27 @@ static inline q8_status launched(cudaError_t e) {
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Host-side checks of the W8A8 linear's arguments other than the workspace (shared by the
+// workspace and the allocation-free entry points, so both report the same status codes).
+q8_status w8a8_check_args(const float* x, const q8_qparams& first, const q8_qparams* second,
+                          const int8_t* q, const int32_t* wsum, const float* s_w,
+                          const float* bias, const float* y, int64_t M, int64_t N, int64_t K) {
+    if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    Q8_TRY(check_qparams(first));
+    if (second) Q8_TRY(check_qparams(*second));
+    if (M == 0) return Q8_OK;
+    if (!x || !q || !wsum || !s_w || !y) return Q8_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(y) || !aligned4(bias)) return Q8_ERR_ALIGN;
+    return Q8_OK;
+}
+
+// The current device's arch check, for entry points in other files.
+q8_status check_current_device() {
+    int sms = 0;
+    return current_device(sms);
+}
+
 // Activation rows up to which the W8A8 linear runs as a GEMV (weights streamed once per
 // 16 rows); above it the tensor-core GEMM takes over.  The tensor-core path loads K in
 // 128-byte steps and needs at least one whole step.
@@ -286,16 +307,19 @@ q8_status q8_qparams_from_minmax(float mn, float mx, q8_qparams* out) {
 }
 
 q8_status q8_quantize_weight_q4gs(const float* W, int64_t N, int64_t K, int G, uint8_t* q4,
-                                  float* gs, void* stream) {
+                                  float* gs, float* c, void* stream) {
     if (!W || !q4 || !gs) return Q8_ERR_NULL;
     if (G != 32 && G != 64 && G != 128 && G != 256) return Q8_ERR_ARG;
     if (N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
     Q8_TRY(check_k(K));
     if (K % G) return Q8_ERR_SHAPE;
-    if (!aligned16(W) || !aligned16(q4) || !aligned16(gs)) return Q8_ERR_ALIGN;
+    if (!aligned16(W) || !aligned16(q4) || !aligned16(gs) || !aligned4(c)) return Q8_ERR_ALIGN;
     int sms = 0;
     Q8_TRY(current_device(sms));
-    return launched(launch_quantize_weight_q4gs(W, N, (int)K, G, q4, gs, (cudaStream_t)stream));
+    cudaStream_t st = (cudaStream_t)stream;
+    Q8_TRY(launched(launch_quantize_weight_q4gs(W, N, (int)K, G, q4, gs, st)));
+    if (!c) return Q8_OK;
+    return launched(launch_q4gs_zero_fold(q4, gs, G, N, (int)K, c, st));
 }
 
 q8_status q8_linear_w8a16(const void* x, const int8_t* q, const float* s_w, void* y,
@@ -322,34 +346,9 @@ q8_status q8_linear_w8a16_bias(const void* x, const int8_t* q, const float* s_w,
                                       (int)K, (cudaStream_t)stream, sms));
 }
 
-q8_status q8_linear_w8a16_planes(const void* x, const int8_t* q, const float* s_w, void* y,
-                                 q8_dtype yt, int64_t M, int64_t N, int64_t K, void* workspace,
-                                 size_t ws_bytes, void* stream) {
-    if (yt != Q8_F32 && yt != Q8_BF16) return Q8_ERR_ARG;
-    if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
-    Q8_TRY(check_k(K));
-    if (M == 0) return Q8_OK;
-    if (!x || !q || !s_w || !y) return Q8_ERR_NULL;
-    if (!aligned16(x) || !aligned16(q)) return Q8_ERR_ALIGN;
-    int sms = 0;
-    int* status = nullptr;
-    Q8_TRY(current_device(sms, &status));
-    const size_t need = w8a16_tc_workspace_bytes(M, K, sms);
-    if (need == 0) return q8_linear_w8a16(x, q, s_w, y, yt, M, N, K, stream);
-    if (!workspace || ws_bytes < need) return Q8_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return Q8_ERR_ALIGN;
-    return launched(launch_w8a16_tc((const uint16_t*)x, q, s_w, y, yt == Q8_BF16, M, N, (int)K,
-                                    workspace, (cudaStream_t)stream, sms, status));
-}
-
 size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) {
     if (M < 0 || N < 1 || check_k(K) != Q8_OK) return 0;
     switch (op) {
-        case Q8_OP_LINEAR_W8A16_PLANES: {
-            int sms = 0;
-            if (current_device(sms) != Q8_OK) return 0;
-            return w8a16_tc_workspace_bytes(M, K, sms);
-        }
         case Q8_OP_LINEAR_W8A8: return plan_w8a8(M, K, extra != 0).bytes;
         case Q8_OP_GPTQ_INT8:
             if (K > kGptqMaxK || !gptq_block_ok(extra)) return 0;
@@ -407,13 +406,8 @@ q8_status q8_linear_w8a8_bias(const float* x, q8_qparams first, const q8_qparams
                               const int8_t* q, const int32_t* wsum, const float* s_w,
                               const float* bias, float* y, int64_t M, int64_t N, int64_t K,
                               void* workspace, size_t ws_bytes, void* stream) {
-    if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
-    Q8_TRY(check_k(K));
-    Q8_TRY(check_qparams(first));
-    if (second) Q8_TRY(check_qparams(*second));
+    Q8_TRY(w8a8_check_args(x, first, second, q, wsum, s_w, bias, y, M, N, K));
     if (M == 0) return Q8_OK;
-    if (!x || !q || !wsum || !s_w || !y) return Q8_ERR_NULL;
-    if (!aligned16(x) || !aligned16(q) || !aligned16(y) || !aligned4(bias)) return Q8_ERR_ALIGN;
     const int two = second != nullptr;
     const W8A8Plan plan = plan_w8a8(M, K, two);
     if (plan.bytes > 0 && (!workspace || ws_bytes < plan.bytes)) return Q8_ERR_WORKSPACE;

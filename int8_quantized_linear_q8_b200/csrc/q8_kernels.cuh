@@ -36,6 +36,12 @@ __device__ __forceinline__ void static_codes16(const float (&v)[16], float s1, f
     }
 }
 
+// q8_abi.cu: host checks shared with the allocation-free entry point
+q8_status w8a8_check_args(const float* x, const q8_qparams& first, const q8_qparams* second,
+                          const int8_t* q, const int32_t* wsum, const float* s_w,
+                          const float* bias, const float* y, int64_t M, int64_t N, int64_t K);
+q8_status check_current_device();
+
 // k_quant.cu
 // full: 0 = amax/127 on +-127, 1 = max(amax/127.5, FLT_EPSILON) on [-128, 127]
 cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int full, int8_t* q,
@@ -52,6 +58,8 @@ cudaError_t launch_observe_minmax(const float* x, int64_t n, float* mm, int rese
                                   float s1, int z1, cudaStream_t st, int num_sms);
 cudaError_t launch_quantize_weight_q4gs(const float* W, int64_t N, int K, int G, uint8_t* q4,
                                         float* gs, cudaStream_t st);
+cudaError_t launch_q4gs_zero_fold(const uint8_t* q4, const float* gs, int G, int64_t N, int K,
+                                  float* c, cudaStream_t st);
 
 // k_gemv_tma.cu
 bool make_tmap_u8_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
@@ -61,12 +69,6 @@ bool w8a16_tma_fits(int64_t M, int64_t K, bool bias = false);
 cudaError_t launch_w8a16_tma(const uint16_t* x, const int8_t* q, const float* s_w,
                              const float* bias, void* y, int y_bf16, int64_t M, int64_t N, int K,
                              cudaStream_t st, int num_sms, int* status);
-
-// k_w8a16_tc.cu
-size_t w8a16_tc_workspace_bytes(int64_t M, int64_t K, int num_sms);
-cudaError_t launch_w8a16_tc(const uint16_t* x, const int8_t* q, const float* s_w, void* y,
-                            int y_bf16, int64_t M, int64_t N, int K, void* ws,
-                            cudaStream_t st, int num_sms, int* status);
 
 // k_gemm_tc.cu
 cudaError_t launch_gemm_s8s8_s32_tc(const int8_t* a, const int8_t* b, int32_t* acc, int64_t M,

@@ -59,11 +59,17 @@ extern "C" q8_status q8_linear_w8a8_noalloc(const float* x, q8_qparams first,
                                             const q8_qparams* second, const int8_t* q,
                                             const int32_t* wsum, const float* s_w, float* y,
                                             int64_t M, int64_t N, int64_t K, void* stream) {
+    // The same argument checks, in the same order, as q8_linear_w8a8 (so both report the
+    // same status for the same mistake), then the device, then the built-in size limit.
+    q8_status st = q8::w8a8_check_args(x, first, second, q, wsum, s_w, nullptr, y, M, N, K);
+    if (st != Q8_OK || M == 0) return st;
+    st = q8::check_current_device();
+    if (st != Q8_OK) return st;
     const size_t need =
         q8_workspace_bytes(Q8_OP_LINEAR_W8A8, M, N, K, second != nullptr ? 1 : 0);
     if (need > q8::kNoAllocScratchBytes) return Q8_ERR_WORKSPACE;
     void* scratch = nullptr;
-    const q8_status st = q8::noalloc_scratch(&scratch);
+    st = q8::noalloc_scratch(&scratch);
     if (st != Q8_OK) return st;
     // Every step after this is q8_linear_w8a8 itself, with the built-in array as workspace.
     return q8_linear_w8a8(x, first, second, q, wsum, s_w, y, M, N, K, scratch,

@@ -93,8 +93,10 @@ def test_argument_validation_before_device(L):
                             None) == q8.Q8_ERR_WORKSPACE
     assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 4, 16, 64, good, 10,
                             None) == q8.Q8_ERR_WORKSPACE
-    assert L.q8_quantize_weight_q4gs(good, 4, 64, 48, good, good, None) == q8.Q8_ERR_ARG
-    assert L.q8_quantize_weight_q4gs(good, 4, 96, 64, good, good, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_quantize_weight_q4gs(good, 4, 64, 48, good, good, None, None) == q8.Q8_ERR_ARG
+    assert L.q8_quantize_weight_q4gs(good, 4, 96, 64, good, good, None, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_quantize_weight_q4gs(good, 4, 128, 64, good, good, _p(0x10002), None) == \
+        q8.Q8_ERR_ALIGN
     # weight grid option and bias entry points
     assert L.q8_quantize_weight_grid(good, 4, 64, 2, good, good, None, None) == q8.Q8_ERR_ARG
     assert L.q8_quantize_weight_grid(good, 4, 60, q8.Q8_GRID_FULL128, good, good, None,
@@ -169,20 +171,17 @@ def test_argument_validation_before_device(L):
     assert L.q8_gemm_s8s8_s32(good, good, good, 0, 16, 256, None) == q8.Q8_OK
     assert L.q8_gemm_s8s8_s32(good, None, good, 4, 16, 256, None) == q8.Q8_ERR_NULL
     assert L.q8_gemm_s8s8_s32(good, good, odd, 4, 16, 256, None) == q8.Q8_ERR_ALIGN
-    # built-in scratch too small for these codes (decided on the host)
-    assert L.q8_linear_w8a8_noalloc(good, qp, None, good, good, good, good, 8192, 16, 4096,
-                                    None) == q8.Q8_ERR_WORKSPACE
-    # digit-plane W8A16
-    assert L.q8_linear_w8a16_planes(good, good, good, good, 7, 1, 16, 64, good, 1 << 20,
+    # the allocation-free W8A8 reports argument mistakes exactly as q8_linear_w8a8 does
+    assert L.q8_linear_w8a8_noalloc(None, qp, None, good, good, good, good, 4, 16, 64,
+                                    None) == q8.Q8_ERR_NULL
+    assert L.q8_linear_w8a8_noalloc(good, qp, None, good, good, good, good, 1 << 33, 16, 64,
+                                    None) == q8.Q8_ERR_SHAPE
+    assert L.q8_linear_w8a8_noalloc(good, bad_qp, None, good, good, good, good, 4, 16, 64,
                                     None) == q8.Q8_ERR_ARG
-    assert L.q8_linear_w8a16_planes(good, good, good, good, q8.Q8_F32, 1, 16, 40, good,
-                                    1 << 20, None) == q8.Q8_ERR_SHAPE
-    assert L.q8_linear_w8a16_planes(good, good, good, good, q8.Q8_F32, 0, 16, 64, None, 0,
+    assert L.q8_linear_w8a8_noalloc(odd, qp, None, good, good, good, good, 4, 16, 64,
+                                    None) == q8.Q8_ERR_ALIGN
+    assert L.q8_linear_w8a8_noalloc(good, qp, None, good, good, good, good, 0, 16, 64,
                                     None) == q8.Q8_OK
-    assert L.q8_linear_w8a16_planes(good, None, good, good, q8.Q8_F32, 1, 16, 64, good,
-                                    1 << 20, None) == q8.Q8_ERR_NULL
-    assert L.q8_linear_w8a16_planes(odd, good, good, good, q8.Q8_F32, 1, 16, 64, good,
-                                    1 << 20, None) == q8.Q8_ERR_ALIGN
     # bounded-wait self-test
     assert L.q8_selftest_bounded_wait(100000, None, None) == q8.Q8_ERR_NULL
     assert L.q8_selftest_bounded_wait(10, good, None) == q8.Q8_ERR_ARG
@@ -199,6 +198,9 @@ def test_argument_validation_before_device(L):
 def test_valid_call_without_gpu_fails_loudly(L):
     good = _p(0x10000)
     st = L.q8_quantize_weight(good, 4, 64, good, good, None, None)
+    assert st in (q8.Q8_ERR_LAUNCH, q8.Q8_ERR_UNSUPPORTED_ARCH)
+    qp = q8.q8_qparams(0.1, 0)
+    st = L.q8_linear_w8a8_noalloc(good, qp, None, good, good, good, good, 4, 16, 64, None)
     assert st in (q8.Q8_ERR_LAUNCH, q8.Q8_ERR_UNSUPPORTED_ARCH)
     with pytest.raises((q8.Q8Error, ValueError, RuntimeError)):
         q8.q8_linear_w8a16(torch.zeros(1, 64, dtype=torch.bfloat16),

@@ -149,14 +149,21 @@ def test_observe_minmax_accumulates():
 
 
 @pytest.mark.parametrize("N,K,G", [(11008, 4096, 32), (11008, 4096, 128), (19, 256, 64),
-                                   (7, 512, 256)])
+                                   (7, 512, 256), (5, 65024, 32), (3, 2048, 256)])
 def test_quantize_weight_q4gs_bit_exact(N, K, G):
+    """Codes, group scales and the zero-point fold c, bit for bit; 65024 / 32 = 2032 groups
+    per row exercise the fold's long fp64 chain across many 32-group rounds."""
     W = wl.weight(N, K, seed=300 + G)
     W[0, :G] = 0.0                                          # a zero group
+    W[1, G:3 * G] *= 1e-20                                  # groups far smaller than the rest
     q4, gs = q8.q8_quantize_weight_q4gs(W.to(DEV), G)
     rq4, rgs = oracle.quantize_weight_q4gs(W.numpy(), G)
     assert np.array_equal(q4.cpu().numpy(), rq4)
     assert np.array_equal(gs.cpu().numpy().view(np.uint32), rgs.view(np.uint32))
+    q4b, gsb, c = q8.q8_quantize_weight_q4gs(W.to(DEV), G, want_c=True)
+    assert torch.equal(q4b, q4) and torch.equal(gsb, gs)
+    rc = oracle.q4gs_zero_fold(rq4, rgs, G)
+    assert np.array_equal(c.cpu().numpy().view(np.uint32), rc.view(np.uint32))
 
 
 # ---------------------------------------------------------------------- W8A16 (a4)
@@ -230,10 +237,10 @@ def _range_edge_rows(M, K, e_small, seed):
 
 @pytest.mark.parametrize("M,N", [(16, 2000), (4, 32000)])
 @pytest.mark.parametrize("e_small", [-22, -23])
-def test_w8a16_fp16_range_boundary(M, N, e_small):
-    """2^10 and 2^-22 are 32 binades apart -- the widest range the fp16 path takes (its
-    smallest elements land exactly on the fp16 subnormal grid); at 2^-23 the kernel must
-    fall back to bf16.  Either way the small elements' sum must be exact to fp32 rounding."""
+def test_w8a16_wide_row_range(M, N, e_small):
+    """Rows whose elements span 32-33 binades (one 2^10 element on an all-zero weight
+    column, the rest near 2^-22 or 2^-23): the bf16 operands carry every element exactly,
+    so the output -- the small elements' sum alone -- must hold to fp32 rounding."""
     K = 4096
     x = _range_edge_rows(M, K, e_small, seed=90 + M)
     W = wl.weight(N, K, seed=91)
@@ -245,8 +252,8 @@ def test_w8a16_fp16_range_boundary(M, N, e_small):
 @pytest.mark.parametrize("M,N", [(16, 1000), (4, 32000)])
 @pytest.mark.parametrize("kind", ["wide", "tiny", "inf"])
 def test_w8a16_activation_ranges(M, N, kind):
-    """Rows the fp16 path cannot take (exponents spread over 2^-120..2^60, inf/NaN) and rows
-    it takes with a large scale (all values near the bf16 subnormal range)."""
+    """Extreme activation rows: exponents spread over 2^-120..2^60, values near the bf16
+    subnormal range, and rows holding inf / NaN (which must propagate as in IEEE)."""
     K = 4096
     g = torch.Generator().manual_seed(95)
     x = torch.randn(M, K, generator=g, dtype=torch.float64)
