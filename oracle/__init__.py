@@ -50,6 +50,18 @@ def lib() -> ctypes.CDLL:
         L.q8o_linear_dq8ca_q4gsw.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_int,
                                              _i64, _i64, _i64, _vp, _i64, _vp, _vp]
         L.q8o_q4gs_zero_fold.argtypes = [_vp, _vp, ctypes.c_int, _i64, _i64, _vp]
+        L.q8o_e2m1_value.restype = ctypes.c_float
+        L.q8o_e2m1_value.argtypes = [ctypes.c_int]
+        L.q8o_e4m3_value.restype = ctypes.c_float
+        L.q8o_e4m3_value.argtypes = [ctypes.c_int]
+        L.q8o_rn_e2m1.restype = ctypes.c_int
+        L.q8o_rn_e2m1.argtypes = [_f32]
+        L.q8o_rn_e4m3.restype = ctypes.c_int
+        L.q8o_rn_e4m3.argtypes = [_f32]
+        L.q8o_quantize_weight_nvfp4.restype = ctypes.c_int
+        L.q8o_quantize_weight_nvfp4.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
+        L.q8o_linear_w4a16_nvfp4.argtypes = [_vp, _vp, _vp, _f32, _i64, _i64, _i64, _vp, _i64,
+                                             _vp, _vp]
         L.q8o_gemm_s8s8_s32.argtypes = [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp]
         L.q8o_gram_rows.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp]
         L.q8o_gptq_hinv.restype = ctypes.c_int
@@ -268,6 +280,50 @@ def q4gs_zero_fold(q4, gs, G):
     c = np.empty(N, np.float32)
     lib().q8o_q4gs_zero_fold(_p(q4), _p(gs), int(G), N, 2 * K2, _p(c))
     return c
+
+
+def e2m1_value(code: int) -> float:
+    return float(lib().q8o_e2m1_value(int(code)))
+
+
+def e4m3_value(byte: int) -> float:
+    return float(lib().q8o_e4m3_value(int(byte)))
+
+
+def rn_e2m1(v: float) -> int:
+    return int(lib().q8o_rn_e2m1(float(v)))
+
+
+def rn_e4m3(v: float) -> int:
+    return int(lib().q8o_rn_e4m3(float(v)))
+
+
+def quantize_weight_nvfp4(W: np.ndarray):
+    """NVFP4 weight codes -> (q4 u8 [N,K/2], block scales u8 [N,K/16] (E4M3), gsc fp32)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    q4 = np.zeros((N, K // 2), np.uint8)
+    sf = np.zeros((N, K // 16), np.uint8)
+    g = np.zeros(1, np.float32)
+    lib().q8o_quantize_weight_nvfp4(_p(W), N, K, _p(q4), _p(sf), _p(g))
+    return q4, sf, np.float32(g[0])
+
+
+def linear_w4a16_nvfp4(x_bf16, q4, sf, gsc, rows=None):
+    """fp64 y [R,N] and magnitude sums for the NVFP4 weight-only linear."""
+    x = _c(x_bf16, np.uint16)
+    q4 = _c(q4, np.uint8)
+    sf = _c(sf, np.uint8)
+    M, K = x.shape
+    N = q4.shape[0]
+    r, R = _rows(rows, M)
+    y = np.empty((R, N), np.float64)
+    a = np.empty((R, N), np.float64)
+    lib().q8o_linear_w4a16_nvfp4(_p(x), _p(q4), _p(sf), float(gsc), M, N, K, _p(r), R,
+                                 _p(y), _p(a))
+    return y, a
 
 
 def gemm_s8s8_s32(a, b, rows=None):

@@ -459,6 +459,135 @@ void q8o_q4gs_zero_fold(const uint8_t* q4, const float* gs, int G, int64_t N, in
     }
 }
 
+/* ------------------------------------------------ NVFP4 weight-only twin (f4)
+ * flashrt-structures schemes.py, W4A16Decode: the weights are quantized per 16-element block
+ * at bind time to NVFP4 -- E2M1 codes packed two per byte plus block scale factors -- and the
+ * activations stay bf16.  The page prints neither the grid nor the scale rule; the reading
+ * taken is NVIDIA's NVFP4 layout, the format the name refers to:
+ *   E2M1 code: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0; magnitudes
+ *     {0, 0.5, 1, 1.5, 2, 3, 4, 6} for codes 0..7 (exponent field 0: 0 and the subnormal 0.5).
+ *   E4M3 block scale: sign bit 7, exponent bits 6..3 (bias 7), mantissa bits 2..0, no
+ *     infinity, 0x7F is NaN, largest finite 448, subnormals m/8 * 2^-6.
+ *   per-tensor fp32 scale gsc = amax(W) / (6 * 448)  (1.0 when W is all zero);
+ *   per block b of 16 consecutive k in a row:
+ *     sb = amax_b / 6;  e = rn_e4m3(sb / gsc);  d = e4m3(e) * gsc      (fp32 steps)
+ *     code = rn_e2m1(W / d)  (IEEE division; a block with d == 0 gets codes 0)
+ *   rn_* round to the nearest representable value, ties to the even code, and saturate at
+ *   the largest finite magnitude; a value that rounds to magnitude 0 gets code 0 (+0).
+ *   Packing: byte k/2 of row n holds code k in its low nibble (k even) or high nibble (k odd);
+ *   block scales are bytes [N, K/16].
+ *   Dequantized weight: e2m1(code) * e4m3(e) * gsc; the first product is exact (2 + 4
+ *   significant bits), so y = gsc * sum_k x * (e2m1 * e4m3). */
+static const float k_e2m1_mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+float q8o_e2m1_value(int code) {
+    const float m = k_e2m1_mag[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+float q8o_e4m3_value(int byte) {
+    const int e = (byte >> 3) & 15, m = byte & 7;
+    float v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexpf((float)m / 8.0f, -6);
+    else v = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+    return (byte & 0x80) ? -v : v;
+}
+
+/* Nearest E2M1 code of a finite v (ties to even code, saturating at 6, +0 for zero). */
+int q8o_rn_e2m1(float v) {
+    const float a = fabsf(v);
+    int best = 0;
+    for (int c = 1; c < 8; ++c) {
+        const float dc = fabsf(a - k_e2m1_mag[c]), db = fabsf(a - k_e2m1_mag[best]);
+        if (dc < db || (dc == db && (c & 1) == 0)) best = c;
+    }
+    if (a >= 6.0f) best = 7;
+    if (best == 0) return 0;
+    return (v < 0.0f ? 8 : 0) | best;
+}
+
+/* Nearest non-negative finite E4M3 byte of a finite v >= 0 (ties to even mantissa,
+ * saturating at 448). */
+int q8o_rn_e4m3(float v) {
+    int best = 0;
+    double bd = fabs((double)v);
+    for (int b = 1; b < 127; ++b) {             /* 0x7F is NaN */
+        const double d = fabs((double)v - (double)q8o_e4m3_value(b));
+        if (d < bd || (d == bd && (b & 1) == 0)) {
+            best = b;
+            bd = d;
+        }
+    }
+    if ((double)v >= 448.0) best = 0x7E;
+    return best;
+}
+
+int q8o_quantize_weight_nvfp4(const float* W, int64_t N, int64_t K, uint8_t* q4,
+                              uint8_t* sf, float* gsc_out) {
+    if (K % 16) return -1;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < N * K; ++i) {
+        const float a = fabsf(W[i]);
+        if (a > amax) amax = a;
+    }
+    float gsc = amax / 2688.0f;                 /* 6 * 448 */
+    if (gsc == 0.0f) gsc = 1.0f;
+    *gsc_out = gsc;
+    const int64_t nb = K / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const float* w = W + n * K + b * 16;
+            float bmax = 0.0f;
+            for (int j = 0; j < 16; ++j) {
+                const float a = fabsf(w[j]);
+                if (a > bmax) bmax = a;
+            }
+            const float sb = bmax / 6.0f;
+            const int e = q8o_rn_e4m3(sb / gsc);
+            const float d = q8o_e4m3_value(e) * gsc;
+            sf[n * nb + b] = (uint8_t)e;
+            for (int j = 0; j < 16; ++j) {
+                const int code = d == 0.0f ? 0 : q8o_rn_e2m1(w[j] / d);
+                const int64_t k = b * 16 + j;
+                uint8_t* byte = q4 + n * (K / 2) + k / 2;
+                if ((k & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | code);
+                else              *byte = (uint8_t)((*byte & 0x0F) | (code << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* W4A16 NVFP4 linear: y[m,n] = gsc * sum_k x[m,k] * (e2m1(q[n,k]) * e4m3(sf[n,k/16])),
+ * fp64 sum over k ascending; absum the same sum of magnitudes. */
+void q8o_linear_w4a16_nvfp4(const uint16_t* x, const uint8_t* q4, const uint8_t* sf, float gsc,
+                            int64_t M, int64_t N, int64_t K,
+                            const int64_t* rows, int64_t nrows, double* y, double* absum) {
+    int64_t R = rows ? nrows : M;
+    const int64_t nb = K / 16;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < R; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        const uint16_t* xr = x + m * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t* wr = q4 + n * (K / 2);
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const int code = (k & 1) ? (wr[k / 2] >> 4) & 0xF : wr[k / 2] & 0xF;
+                const double w = (double)q8o_e2m1_value(code) *
+                                 (double)q8o_e4m3_value(sf[n * nb + k / 16]);
+                const double p = (double)bf16_to_f32(xr[k]) * w;
+                acc += p;
+                mag += fabs(p);
+            }
+            y[i * N + n] = acc * (double)gsc;
+            if (absum) absum[i * N + n] = mag * fabs((double)gsc);
+        }
+    }
+}
+
 /* ------------------------------------------------ int8 GEMM, int32 out (a8)
  * acc[m,n] = sum_k a[m,k] * b[n,k], exact. */
 void q8o_gemm_s8s8_s32(const int8_t* a, const int8_t* b,

@@ -46,6 +46,15 @@ void q8o_linear_dq8ca_q4gsw(const int8_t* xq, const float* s, const int32_t* z,
                             double* y, double* absum);
 void q8o_q4gs_zero_fold(const uint8_t* q4, const float* gs, int G, int64_t N, int64_t K,
                         float* c);
+float q8o_e2m1_value(int code);
+float q8o_e4m3_value(int byte);
+int  q8o_rn_e2m1(float v);
+int  q8o_rn_e4m3(float v);
+int  q8o_quantize_weight_nvfp4(const float* W, int64_t N, int64_t K, uint8_t* q4, uint8_t* sf,
+                               float* gsc);
+void q8o_linear_w4a16_nvfp4(const uint16_t* x, const uint8_t* q4, const uint8_t* sf, float gsc,
+                            int64_t M, int64_t N, int64_t K, const int64_t* rows, int64_t nrows,
+                            double* y, double* absum);
 void q8o_gemm_s8s8_s32(const int8_t* a, const int8_t* b,
                        int64_t M, int64_t N, int64_t K,
                        const int64_t* rows, int64_t nrows, int32_t* acc);

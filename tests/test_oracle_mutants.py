@@ -39,7 +39,8 @@ MUTANTS = [
     ("w8a16 transposed weight index", "(double)bf16_to_f32(xr[k]) * (double)qr[k];",
      "(double)bf16_to_f32(xr[k]) * (double)q[k * N + n];",
      ["test_w8a16_factorisation_identity"]),
-    ("q4 nibble order swapped", "if ((k & 1) == 0) *byte", "if ((k & 1) == 1) *byte",
+    ("q4 nibble order swapped", "if ((k & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | nib);",
+     "if ((k & 1) == 1) *byte = (uint8_t)((*byte & 0xF0) | nib);",
      ["test_golden_q4_groups"]),
     ("q4 group scale index", "acc += (double)gs[n * ng + g] * (double)part;",
      "acc += (double)gs[n * ng] * (double)part;", ["test_dq8ca_q4gsw_reductions"]),
@@ -50,6 +51,19 @@ MUTANTS = [
     ("zero fold skips the last group", "for (int64_t g = 0; g < ng; ++g) {\n            int64_t part = 0;\n            for (int64_t k = g * G; k < (g + 1) * G; ++k) part +=",
      "for (int64_t g = 0; g < ng - 1; ++g) {\n            int64_t part = 0;\n            for (int64_t k = g * G; k < (g + 1) * G; ++k) part +=",
      ["test_q4gs_zero_fold_exact_row_sums"]),
+    ("e2m1 ties away from zero", "if (dc < db || (dc == db && (c & 1) == 0)) best = c;",
+     "if (dc <= db) best = c;", ["test_rn_e2m1_nearest_even_saturating"]),
+    ("e4m3 rounding truncates", "if (d < bd || (d == bd && (b & 1) == 0)) {",
+     "if ((double)q8o_e4m3_value(b) <= (double)v) {", ["test_rn_e4m3_nearest_even_saturating"]),
+    ("nvfp4 block scale amax/4", "const float sb = bmax / 6.0f;", "const float sb = bmax / 4.0f;",
+     ["test_golden_nvfp4_blocks"]),
+    ("nvfp4 tensor scale over 448", "float gsc = amax / 2688.0f;", "float gsc = amax / 448.0f;",
+     ["test_golden_nvfp4_blocks"]),
+    ("nvfp4 nibble order", "if ((k & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | code);",
+     "if ((k & 1) == 1) *byte = (uint8_t)((*byte & 0xF0) | code);", ["test_golden_nvfp4_blocks"]),
+    ("w4a16 scale of the next block", "(double)q8o_e4m3_value(sf[n * nb + k / 16]);",
+     "(double)q8o_e4m3_value(sf[n * nb + (k / 16 + 1) % nb]);",
+     ["test_w4a16_nvfp4_factorisation_identity"]),
     ("bf16 rounding truncates", "double r = nearbyint(ldexp(m, 8));",
      "double r = trunc(ldexp(m, 8));", ["test_round_bf16"]),
     ("full grid clamps at -127",

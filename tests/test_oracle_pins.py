@@ -690,3 +690,161 @@ def test_minmax_is_numpy_min_max():
     x[36, 50] = 7e29
     assert oracle.minmax(x) == (float(x.min()), float(x.max()))
     assert oracle.minmax(np.full((3,), 2.5, np.float32)) == (2.5, 2.5)
+
+
+# ------------------------------------------------------ NVFP4 weight-only twin (f4)
+# flashrt-structures schemes.py, W4A16Decode: E2M1 codes packed two per byte with a scale
+# per 16-element block, bf16 activations.  The format's fields are written out here from
+# their bit definitions (not from the oracle) and the oracle is held to them.
+
+
+def _e2m1_exact(code):
+    """E2M1 from its bits: sign 3, exponent 2..1 (bias 1), mantissa 0; exponent 0 is the
+    subnormal m * 0.5."""
+    s, e, m = (code >> 3) & 1, (code >> 1) & 3, code & 1
+    v = Fraction(m, 2) if e == 0 else Fraction(2) ** (e - 1) * (1 + Fraction(m, 2))
+    return -v if s else v
+
+
+def _e4m3_exact(b):
+    """E4M3 from its bits: sign 7, exponent 6..3 (bias 7), mantissa 2..0, subnormals
+    m/8 * 2^-6; exponent 15 with mantissa 7 is NaN (None here)."""
+    s, e, m = (b >> 7) & 1, (b >> 3) & 15, b & 7
+    if e == 15 and m == 7:
+        return None
+    v = Fraction(m, 8) * Fraction(1, 64) if e == 0 else Fraction(2) ** (e - 7) * (1 + Fraction(m, 8))
+    return -v if s else v
+
+
+def _nearest_code(a, values):
+    """Index of the value nearest to a (ties to the even index), saturating at the last."""
+    best = 0
+    for i, v in enumerate(values):
+        d, db = abs(a - v), abs(a - values[best])
+        if d < db or (d == db and i % 2 == 0):
+            best = i
+    if a >= values[-1]:
+        best = len(values) - 1
+    return best
+
+
+E2M1_POS = [_e2m1_exact(c) for c in range(8)]
+E4M3_POS = [_e4m3_exact(b) for b in range(127)]
+
+
+def test_e2m1_and_e4m3_tables_exhaustive():
+    assert E2M1_POS == [Fraction(v) for v in ("0", "1/2", "1", "3/2", "2", "3", "4", "6")]
+    for c in range(16):
+        assert Fraction(oracle.e2m1_value(c)) == _e2m1_exact(c), c
+    for b in range(256):
+        want = _e4m3_exact(b)
+        got = oracle.e4m3_value(b)
+        if want is None:
+            assert np.isnan(got), b
+        else:
+            assert Fraction(got) == want, b
+    assert max(E4M3_POS) == 448 and min(v for v in E4M3_POS if v > 0) == Fraction(1, 512)
+
+
+def _rn_e2m1_exact(v):
+    a = abs(Fraction(float(np.float32(v))))
+    c = _nearest_code(a, E2M1_POS)
+    return 0 if c == 0 else (8 if v < 0 else 0) | c
+
+
+def test_rn_e2m1_nearest_even_saturating():
+    rng = np.random.default_rng(40)
+    vals = list(rng.uniform(-8, 8, 4000).astype(np.float32))
+    mids = [(E2M1_POS[i] + E2M1_POS[i + 1]) / 2 for i in range(7)]
+    for mid in mids:                                  # exact ties and their neighbours
+        f = float(mid)
+        vals += [f, -f, np.nextafter(np.float32(f), np.float32(0)),
+                 np.nextafter(np.float32(f), np.float32(10))]
+    vals += [0.0, -0.0, 6.0, -6.0, 6.5, -100.0, 1e-30, -1e-30]
+    for v in vals:
+        assert oracle.rn_e2m1(float(v)) == _rn_e2m1_exact(v), v
+
+
+def test_rn_e4m3_nearest_even_saturating():
+    rng = np.random.default_rng(41)
+    vals = list(np.exp2(rng.uniform(-12, 10, 3000)).astype(np.float32))
+    for i in range(len(E4M3_POS) - 1):
+        mid = (E4M3_POS[i] + E4M3_POS[i + 1]) / 2
+        f = np.float32(float(mid))
+        if Fraction(float(f)) == mid:                 # exact ties (fp32 holds them all)
+            vals += [f, np.nextafter(f, np.float32(0)), np.nextafter(f, np.float32(1e4))]
+    vals += [0.0, 448.0, 449.0, 464.0, 1e6, 2.0 ** -10, 2.0 ** -9]
+    for v in vals:
+        a = Fraction(float(np.float32(v)))
+        assert oracle.rn_e4m3(float(v)) == _nearest_code(a, E4M3_POS), v
+
+
+def _nvfp4_golden():
+    rows = _parse("nvfp4_blocks.txt")
+    blocks = [([float(v) for v in r[0]], int(r[1][0], 16), [int(c, 16) for c in r[2]])
+              for r in rows]
+    W = np.array([sum((b[0] for b in blocks[0:4]), []), sum((b[0] for b in blocks[4:8]), [])],
+                 np.float32)
+    return W, blocks
+
+
+def _unpack_nibbles(q4):
+    codes = np.empty((q4.shape[0], 2 * q4.shape[1]), np.int64)
+    codes[:, 0::2] = q4 & 0xF
+    codes[:, 1::2] = q4 >> 4
+    return codes
+
+
+def test_golden_nvfp4_blocks():
+    """Hand-worked blocks: the scale byte and the 16 codes of every block, gsc = 1."""
+    W, blocks = _nvfp4_golden()
+    q4, sf, gsc = oracle.quantize_weight_nvfp4(W)
+    assert gsc == np.float32(1.0)
+    codes = _unpack_nibbles(q4)
+    for i, (_, e, want) in enumerate(blocks):
+        r, b = divmod(i, 4)
+        assert sf[r, b] == e, f"block {i} scale"
+        assert codes[r, 16 * b:16 * b + 16].tolist() == want, f"block {i} codes"
+
+
+def test_nvfp4_quantizer_follows_its_steps():
+    """Random weights (a zero block, a tiny block, mixed magnitudes): every fp32 step of the
+    reading re-done here in exact arithmetic -- the tensor scale, each block's E4M3 byte as
+    the nearest to fp32(fp32(amax_b / 6) / gsc), each code as the nearest E2M1 to
+    fp32(w / d) with d = fp32(e4m3 * gsc)."""
+    W = wl.weight(6, 256, seed=42).numpy()
+    W[1, 16:32] = 0.0
+    W[2, 32:48] *= 1e-6
+    W[3] *= 50.0
+    q4, sf, gsc = oracle.quantize_weight_nvfp4(W)
+    assert gsc == np.float32(np.abs(W).max()) / np.float32(2688.0)
+    codes = _unpack_nibbles(q4)
+    for n in range(W.shape[0]):
+        for b in range(16):
+            blk = W[n, 16 * b:16 * b + 16]
+            sb = np.float32(np.abs(blk).max()) / np.float32(6.0)
+            e = _nearest_code(Fraction(float(np.float32(sb / gsc))), E4M3_POS)
+            assert sf[n, b] == e, (n, b)
+            d = np.float32(np.float32(float(_e4m3_exact(e))) * gsc)
+            for j in range(16):
+                want = 0 if d == 0 else _rn_e2m1_exact(np.float32(blk[j] / d))
+                assert codes[n, 16 * b + j] == want, (n, b, j)
+
+
+def test_w4a16_nvfp4_factorisation_identity():
+    """The linear is gsc * x . (e2m1 * e4m3): a numpy fp64 matmul on weights decoded here."""
+    bits = wl.bf16_bits(wl.normal_bf16((5, 256), 1.0, seed=43))
+    W = wl.weight(9, 256, seed=44).numpy()
+    W[4, :16] = 0.0
+    q4, sf, gsc = oracle.quantize_weight_nvfp4(W)
+    codes = _unpack_nibbles(q4)
+    dq = np.array([[float(_e2m1_exact(int(codes[n, k])) * _e4m3_exact(int(sf[n, k // 16])))
+                    for k in range(256)] for n in range(9)])
+    x = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = (x @ dq.T) * float(gsc)
+    y, a = oracle.linear_w4a16_nvfp4(bits, q4, sf, gsc)
+    assert np.all(np.abs(y - ref) <= 1e-12 * a + 1e-300)
+    y2, _ = oracle.linear_w4a16_nvfp4(bits, q4, sf, gsc, rows=[4, 0])
+    assert np.array_equal(y2, y[[4, 0]])
+    # dequantized weights stay within half a grid step (plus saturation) of W
+    assert np.all(np.abs(dq * float(gsc) - W) <= np.abs(W).max() / 6 * 1.0 + 1e-30)
