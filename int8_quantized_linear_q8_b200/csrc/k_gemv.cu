@@ -116,12 +116,17 @@ __global__ __launch_bounds__(GEMV_THREADS) void k_w8a16_gemv(
 }
 
 // -------------------------------------------------------------------------- W8A8
-// acc = sum_k xq * q (int32, exact) from activation codes xq1 (and xq2) [M, K];
+// The static activation codes are computed in the kernel from the fp32 activations
+// (SmolVLM-Q8 Q8Linear.forward lowers to one delegated linear_q8ta_q8csw call that takes x
+// and its qparams): each lane quantizes exactly the 16 activations it feeds to its own MMA
+// k slots, with the fp32 steps of q8_quantize_static (static_codes16), so the codes are the
+// same bits without a pass through memory;
+// acc = sum_k xq * q (int32, exact) for the first-pass codes (and the residual's);
 // y[m, n] = s_w[n] * (s1 * (acc1 - z1 * wsum[n]) + s2 * (acc2 - z2 * wsum[n])) (+ bias[n]).
 template <int MT, int UNROLL, bool TWO>
 __global__ __launch_bounds__(GEMV_THREADS) void k_w8a8_gemv(
-    const int8_t* __restrict__ xq1, const int8_t* __restrict__ xq2, float s1, int z1, float s2,
-    int z2, const int8_t* __restrict__ q, const int32_t* __restrict__ wsum,
+    const float* __restrict__ x, float s1, int z1, float s2, int z2,
+    const int8_t* __restrict__ q, const int32_t* __restrict__ wsum,
     const float* __restrict__ s_w, const float* __restrict__ bias, float* __restrict__ y, int M,
     int N, int K) {
     __shared__ int red[GEMV_WARPS][TWO ? 2 : 1][MT][32][4];
@@ -149,13 +154,17 @@ __global__ __launch_bounds__(GEMV_THREADS) void k_w8a8_gemv(
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc1[mt][i] = acc2[mt][i] = 0;
 
-    // The activation codes are written by the kernel launched just before this one
-    // (programmatic dependent launch): wait for it before the first read.
+    const float inv1 = __fdiv_rn(1.0f, s1);
+    const float inv2 = TWO ? __fdiv_rn(1.0f, s2) : 0.0f;
+    const float z1f = (float)z1, z2f = (float)z2;
+
+    // Programmatic dependent launch: the previous kernel on the stream may have written x.
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const uint4 zero4 = make_uint4(0, 0, 0, 0);
     for (int c = warp; c < nchunks; c += GEMV_WARPS * UNROLL) {
         uint4 wa[UNROLL], wb[UNROLL], x1[UNROLL][MT], x2[UNROLL][MT];
+        float xf[UNROLL][MT][16];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
             const int cc = c + GEMV_WARPS * u;
@@ -166,8 +175,27 @@ __global__ __launch_bounds__(GEMV_THREADS) void k_w8a8_gemv(
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const bool ok = xv[mt] && kin;
-                x1[u][mt] = ok ? ldg_keep(xq1 + xoff[mt] + cc * 64) : zero4;
-                if (TWO) x2[u][mt] = ok ? ldg_keep(xq2 + xoff[mt] + cc * 64) : zero4;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 f = ok ? ldg_f4(x + xoff[mt] + cc * 64 + 4 * i)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    xf[u][mt][4 * i] = f.x; xf[u][mt][4 * i + 1] = f.y;
+                    xf[u][mt][4 * i + 2] = f.z; xf[u][mt][4 * i + 3] = f.w;
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int cc = c + GEMV_WARPS * u;
+            const bool kin = (cc < nchunks) && (cc * 64 + 16 * t < K);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t o1[4], o2[4];
+                static_codes16(xf[u][mt], s1, inv1, z1f, TWO, inv2, z2f, o1, o2);
+                // rows past M and k past K contribute nothing (code 0, not z)
+                const bool ok = xv[mt] && kin;
+                x1[u][mt] = ok ? make_uint4(o1[0], o1[1], o1[2], o1[3]) : zero4;
+                if (TWO) x2[u][mt] = ok ? make_uint4(o2[0], o2[1], o2[2], o2[3]) : zero4;
             }
         }
 #pragma unroll
@@ -238,7 +266,7 @@ cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s
 }
 
 template <int MT, int U, bool TWO>
-static cudaError_t launch_w8a8_gemv_t(dim3 grid, const int8_t* xq1, const int8_t* xq2, float s1,
+static cudaError_t launch_w8a8_gemv_t(dim3 grid, const float* x, float s1,
                                       int z1, float s2, int z2, const int8_t* q,
                                       const int32_t* wsum, const float* s_w, const float* bias,
                                       float* y, int M, int N, int K, cudaStream_t st) {
@@ -252,26 +280,26 @@ static cudaError_t launch_w8a8_gemv_t(dim3 grid, const int8_t* xq1, const int8_t
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_w8a8_gemv<MT, U, TWO>, xq1, xq2, s1, z1, s2, z2, q, wsum,
+    return cudaLaunchKernelEx(&cfg, k_w8a8_gemv<MT, U, TWO>, x, s1, z1, s2, z2, q, wsum,
                               s_w, bias, y, M, N, K);
 }
 
-cudaError_t launch_w8a8_gemv_codes(const int8_t* xq1, const int8_t* xq2, float s1, int z1,
-                                   int has2, float s2, int z2, const int8_t* q,
-                                   const int32_t* wsum, const float* s_w, const float* bias,
-                                   float* y, int64_t M, int64_t N, int K, cudaStream_t st) {
+cudaError_t launch_w8a8_gemv(const float* x, float s1, int z1, int has2, float s2, int z2,
+                             const int8_t* q, const int32_t* wsum, const float* s_w,
+                             const float* bias, float* y, int64_t M, int64_t N, int K,
+                             cudaStream_t st) {
     const unsigned gx = (unsigned)((N + 15) / 16);
     if (M <= 8) {
         dim3 grid(gx, 1);
-        return has2 ? launch_w8a8_gemv_t<1, 4, true>(grid, xq1, xq2, s1, z1, s2, z2, q, wsum, s_w,
+        return has2 ? launch_w8a8_gemv_t<1, 4, true>(grid, x, s1, z1, s2, z2, q, wsum, s_w,
                                                      bias, y, (int)M, (int)N, K, st)
-                    : launch_w8a8_gemv_t<1, 4, false>(grid, xq1, xq2, s1, z1, s2, z2, q, wsum,
+                    : launch_w8a8_gemv_t<1, 4, false>(grid, x, s1, z1, s2, z2, q, wsum,
                                                       s_w, bias, y, (int)M, (int)N, K, st);
     }
     dim3 grid(gx, (unsigned)((M + 15) / 16));
-    return has2 ? launch_w8a8_gemv_t<2, 2, true>(grid, xq1, xq2, s1, z1, s2, z2, q, wsum, s_w,
+    return has2 ? launch_w8a8_gemv_t<2, 2, true>(grid, x, s1, z1, s2, z2, q, wsum, s_w,
                                                  bias, y, (int)M, (int)N, K, st)
-                : launch_w8a8_gemv_t<2, 2, false>(grid, xq1, xq2, s1, z1, s2, z2, q, wsum, s_w,
+                : launch_w8a8_gemv_t<2, 2, false>(grid, x, s1, z1, s2, z2, q, wsum, s_w,
                                                   bias, y, (int)M, (int)N, K, st);
 }
 

@@ -42,6 +42,13 @@ q8_status w8a8_check_args(const float* x, const q8_qparams& first, const q8_qpar
                           const float* bias, const float* y, int64_t M, int64_t N, int64_t K);
 q8_status check_current_device();
 
+// k_w4a16.cu (NVFP4 weight-only twin)
+cudaError_t launch_quantize_weight_nvfp4(const float* W, int64_t N, int K, uint8_t* q4,
+                                         uint8_t* sf, float* gsc, cudaStream_t st, int num_sms);
+cudaError_t launch_w4a16_nvfp4(const uint16_t* x, const uint8_t* q4, const uint8_t* sf,
+                               const float* gsc, void* y, int y_bf16, int64_t M, int64_t N, int K,
+                               cudaStream_t st);
+
 // k_quant.cu
 // full: 0 = amax/127 on +-127, 1 = max(amax/127.5, FLT_EPSILON) on [-128, 127]
 cudaError_t launch_quantize_weight(const float* W, int64_t N, int K, int full, int8_t* q,
@@ -122,9 +129,9 @@ cudaError_t launch_gptq_int8(const float* W, const double* H, int64_t N, int K, 
 cudaError_t launch_w8a16_gemv(const uint16_t* x, const int8_t* q, const float* s_w,
                               const float* bias, void* y, int y_bf16, int64_t M, int64_t N, int K,
                               cudaStream_t st, int num_sms);
-cudaError_t launch_w8a8_gemv_codes(const int8_t* xq1, const int8_t* xq2, float s1, int z1,
-                                   int has2, float s2, int z2, const int8_t* q,
-                                   const int32_t* wsum, const float* s_w, const float* bias,
-                                   float* y, int64_t M, int64_t N, int K, cudaStream_t st);
+cudaError_t launch_w8a8_gemv(const float* x, float s1, int z1, int has2, float s2, int z2,
+                             const int8_t* q, const int32_t* wsum, const float* s_w,
+                             const float* bias, float* y, int64_t M, int64_t N, int K,
+                             cudaStream_t st);
 
 }  // namespace q8

@@ -55,10 +55,16 @@ int main(void) {
     expect("linear_w8a8_noalloc",
            q8_linear_w8a8_noalloc(NULL, qp, NULL, NULL, NULL, NULL, NULL, 8192, 16, 4096, NULL),
            Q8_ERR_NULL);
+    expect("quantize_weight_nvfp4", q8_quantize_weight_nvfp4(NULL, 4, 64, NULL, NULL, NULL, NULL),
+           Q8_ERR_NULL);
+    expect("linear_w4a16_nvfp4",
+           q8_linear_w4a16_nvfp4(NULL, NULL, NULL, NULL, NULL, Q8_BF16, 1, 16, 48, NULL),
+           Q8_ERR_SHAPE);
     expect("linear_dq8ca_q4gsw",
            q8_linear_dq8ca_q4gsw(NULL, NULL, NULL, 48, NULL, 1, 16, 256, NULL, 0, NULL),
            Q8_ERR_ARG);
-    if (q8_workspace_bytes(Q8_OP_LINEAR_W8A8, 4, 16, 64, 0) < 4 * 64) ++fails;
+    if (q8_workspace_bytes(Q8_OP_LINEAR_W8A8, 17, 16, 128, 0) < 17 * 128) ++fails;
+    if (q8_workspace_bytes(Q8_OP_LINEAR_W8A8, 4, 16, 64, 0) != 0) ++fails;
     if (q8_workspace_bytes(Q8_OP_GPTQ_INT8, 0, 8, 64, 128) < 3 * 64 * 64 * 8) ++fails;
     expect("gemm_s8s8_s32", q8_gemm_s8s8_s32(NULL, NULL, NULL, 4, 0, 256, NULL), Q8_ERR_SHAPE);
     expect("selftest_bounded_wait", q8_selftest_bounded_wait(100000, NULL, NULL), Q8_ERR_NULL);

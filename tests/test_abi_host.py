@@ -60,8 +60,11 @@ def test_qparams_from_minmax_rejects(L):
 
 def test_workspace_sizes(L):
     assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 0, 16, 64) == 0
-    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 4, 16, 64, 0) >= 4 * 64
-    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 4, 16, 64, 1) >= 2 * 4 * 64
+    # up to 16 rows (or K < 128) the GEMV computes its codes in registers: no workspace
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 16, 16, 4096, 1) == 0
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 300, 16, 64, 1) == 0
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 17, 16, 128, 0) >= 17 * 128
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 17, 16, 128, 1) >= 2 * 17 * 128
     assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 4, 16, 63) == 0      # invalid K
 
 
@@ -89,9 +92,9 @@ def test_argument_validation_before_device(L):
                             None) == q8.Q8_ERR_ARG
     assert L.q8_linear_w8a8(good, q8.q8_qparams(0.1, 200), None, good, good, good, good, 1, 16,
                             64, good, 1024, None) == q8.Q8_ERR_ARG
-    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 4, 16, 64, None, 0,
+    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 17, 16, 128, None, 0,
                             None) == q8.Q8_ERR_WORKSPACE
-    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 4, 16, 64, good, 10,
+    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 17, 16, 128, good, 10,
                             None) == q8.Q8_ERR_WORKSPACE
     assert L.q8_quantize_weight_q4gs(good, 4, 64, 48, good, good, None, None) == q8.Q8_ERR_ARG
     assert L.q8_quantize_weight_q4gs(good, 4, 96, 64, good, good, None, None) == q8.Q8_ERR_SHAPE
@@ -182,6 +185,20 @@ def test_argument_validation_before_device(L):
                                     None) == q8.Q8_ERR_ALIGN
     assert L.q8_linear_w8a8_noalloc(good, qp, None, good, good, good, good, 0, 16, 64,
                                     None) == q8.Q8_OK
+    # NVFP4 weight-only twin
+    assert L.q8_quantize_weight_nvfp4(None, 4, 64, good, good, good, None) == q8.Q8_ERR_NULL
+    assert L.q8_quantize_weight_nvfp4(good, 4, 48, good, good, good, None) == q8.Q8_ERR_SHAPE
+    assert L.q8_quantize_weight_nvfp4(odd, 4, 64, good, good, good, None) == q8.Q8_ERR_ALIGN
+    assert L.q8_linear_w4a16_nvfp4(good, good, good, good, good, 7, 1, 16, 64, None) == \
+        q8.Q8_ERR_ARG
+    assert L.q8_linear_w4a16_nvfp4(good, good, good, good, good, q8.Q8_BF16, 1, 16, 48,
+                                   None) == q8.Q8_ERR_SHAPE
+    assert L.q8_linear_w4a16_nvfp4(good, good, good, good, good, q8.Q8_BF16, 0, 16, 64,
+                                   None) == q8.Q8_OK
+    assert L.q8_linear_w4a16_nvfp4(good, None, good, good, good, q8.Q8_BF16, 1, 16, 64,
+                                   None) == q8.Q8_ERR_NULL
+    assert L.q8_linear_w4a16_nvfp4(good, good, odd, good, good, q8.Q8_BF16, 1, 16, 64,
+                                   None) == q8.Q8_ERR_ALIGN
     # bounded-wait self-test
     assert L.q8_selftest_bounded_wait(100000, None, None) == q8.Q8_ERR_NULL
     assert L.q8_selftest_bounded_wait(10, good, None) == q8.Q8_ERR_ARG
