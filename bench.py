@@ -562,6 +562,40 @@ def bench_q4(dev, peaks, reps=5):
     return out
 
 
+def bench_w4a16(dev, peaks, reps=20):
+    """The NVFP4 weight-only twin on the W8A16 sweep's shapes and rows (same seeded weights,
+    quantized to E2M1 codes with E4M3 block scales): per-case device time from a graph of
+    `reps` launches alternating two weight copies; bytes = N*K/2 codes + N*K/16 scale bytes +
+    2MK + 2MN."""
+    import int8_quantized_linear_q8_b200 as q8
+
+    out = []
+    g = torch.Generator(device=dev)
+    for i, sh in enumerate(wl.W8A16_SWEEP_SHAPES):
+        g.manual_seed(wl.W8A16_SWEEP_SEED_W * 1000 + i)
+        W = torch.randn(sh.N, sh.K, generator=g, device=dev) * 0.02
+        copies = [q8.q8_quantize_weight_nvfp4(W), q8.q8_quantize_weight_nvfp4(W.clone())]
+        del W
+        for M in wl.W8A16_SWEEP_M:
+            g.manual_seed(wl.W8A16_SWEEP_SEED_X * 1000 + 10 * i + M)
+            x = torch.randn(M, sh.K, generator=g, device=dev).to(torch.bfloat16)
+            y = torch.empty(M, sh.N, dtype=torch.bfloat16, device=dev)
+            state = {"c": 0}
+
+            def fn():
+                q4, sf, gsc = copies[state["c"] % 2]
+                state["c"] += 1
+                q8.q8_linear_w4a16_nvfp4(x, q4, sf, gsc, y=y)
+
+            us = _graph_time(fn, reps)
+            b = sh.N * sh.K // 2 + sh.N * sh.K // 16 + 2 * M * sh.K + 2 * M * sh.N
+            out.append({"K": sh.K, "N": sh.N, "M": M, "us": round(us, 3),
+                        "GBps": round(b / us / 1e3, 1),
+                        "frac_hbm": round(b / us / 1e3 / peaks["hbm_gbs"], 4)})
+        del copies
+    return out
+
+
 def bench_quantizers(dev, peaks, reps=5):
     """The quantizers as HBM streams: weight codes on both grids (fp32 32000x4096 in),
     per-row activation qparams + codes (bf16 4096x4096), static activation codes with the
@@ -789,6 +823,7 @@ def run_ours(args):
     if dist.rank == 0 and not args.no_paths:
         result["paths"] = {
             "w8a16_bias": bias_case_times(sweep),
+            "w4a16_nvfp4": bench_w4a16(dev, peaks),
             "w8a8_static_k960": bench_w8a8_paths(dev),
             "w8a8_prefill_m4096": bench_w8a8_prefill(dev, peaks),
             "dq8ca_q4gsw": bench_q4(dev, peaks),

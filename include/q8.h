@@ -18,6 +18,8 @@
  *                act_observer, fix_q8ta_fake (linear_q8ta_q8csw operands)
  *   [ET-21229]   pytorch/executorch PR #21229 description: choose_qparams_affine
  *                and linear_dq8ca_q4gsw (8da4w)
+ *   [flashrt]    flashrt_structures/schemes.py (flashrt-structures 0.2.0): W8A16Decode and
+ *                its NVFP4 twin W4A16Decode
  *
  * Conventions shared by every call
  *   - Pointers named as device pointers must be device memory of the current
@@ -195,7 +197,41 @@ q8_status q8_qparams_from_minmax(float mn, float mx, q8_qparams* out);
 q8_status q8_quantize_weight_q4gs(const float* W, int64_t N, int64_t K, int G,
                                   uint8_t* q4, float* gs, float* c, void* stream);
 
+/* NVFP4 weight codes for the weight-only twin of the W8A16 decode linear
+ * ([flashrt] schemes.py, W4A16Decode: "E2M1 packed + block scale factors", one scale per
+ * 16-element block, bf16 activations; the page prints no quantization rule, so NVIDIA's
+ * NVFP4 layout is used):
+ *     gsc = amax(W) / (6 * 448)              (fp32; 1.0 when W is all zero)
+ *     per block b of 16 consecutive k of a row:
+ *       sb = amax_b / 6;  e = rn_e4m3(sb / gsc);  d = e4m3(e) * gsc     (fp32 steps)
+ *       code = rn_e2m1(W / d)                 (IEEE division; d == 0 gives codes 0)
+ * where rn_* round to the nearest representable value with ties to the even code and
+ * saturate at the largest finite magnitude (E2M1: sign bit 3, magnitudes 0, .5, 1, 1.5, 2,
+ * 3, 4, 6 for codes 0..7; E4M3: exponent bits 6..3 with bias 7, mantissa bits 2..0, largest
+ * 448); a value that rounds to magnitude 0 gets code 0.  Byte k/2 of row n holds code k in
+ * its low nibble (k even) or high nibble (k odd).
+ *   W device fp32 [N, K]; q4 device uint8 [N, K/2]; sf device uint8 [N, K/16] (E4M3 block
+ *   scales); gsc device fp32 [1] (written; used as scratch by the call before it is).
+ *   K % 32 == 0 (Q8_ERR_SHAPE otherwise).
+ * Codes, scale bytes and gsc are bit-identical to the CPU reference definition. */
+q8_status q8_quantize_weight_nvfp4(const float* W, int64_t N, int64_t K, uint8_t* q4,
+                                   uint8_t* sf, float* gsc, void* stream);
+
 /* -------------------------------------------------------------------- linears */
+
+/* W4A16 with NVFP4 weights, the weight-only twin of q8_linear_w8a16 ([flashrt] schemes.py,
+ * W4A16Decode: same decode band, half the weight bytes):
+ *     y[m,n] = gsc * sum_k x[m,k] * (e2m1(code[n,k]) * e4m3(sf[n,k/16]))
+ * The block-scaled weight e2m1 * e4m3 is exact in bf16 (at most 6 significant bits), so the
+ * sum runs on the bf16 tensor cores with fp32 accumulation; gsc and one rounding to yt come
+ * last.
+ *   x device bf16 [M, K]; q4, sf, gsc as written by q8_quantize_weight_nvfp4 (gsc is read
+ *   on the device); y device [M, N] of type yt (Q8_BF16 or Q8_F32).  K % 32 == 0.
+ * A GEMV streaming the packed codes from HBM (16 activation rows per pass). */
+q8_status q8_linear_w4a16_nvfp4(const void* x, const uint8_t* q4, const uint8_t* sf,
+                                const float* gsc, void* y, q8_dtype yt, int64_t M, int64_t N,
+                                int64_t K, void* stream);
+
 
 /* W8A16: bf16 activations times int8 weights, the scale applied after the sum
  * ([tiny-llm] factorisation identity y_j = s_j sum_i x_i q_ji; Int8Linear.forward):
@@ -230,10 +266,11 @@ q8_status q8_linear_w8a16_bias(const void* x, const int8_t* q, const float* s_w,
  *   workspace: device scratch of at least q8_workspace_bytes(Q8_OP_LINEAR_W8A8, M, N,
  *   K, second != NULL) bytes (may be NULL when that is 0); its contents on entry do not
  *   matter and are overwritten.
- * A first kernel writes the activation codes (q8_quantize_static) to the workspace; then
- * decode-sized M (<= 16) runs as a GEMV on the warp-level int8 MMA, larger M as a tcgen05
- * int8 GEMM (int32 accumulators in tensor memory) with the zero-point term and both
- * scales in its epilogue. */
+ * Decode-sized M (<= 16, or any M when K < 128) runs as one GEMV kernel on the warp-level
+ * int8 MMA that computes the activation codes in registers (the steps of
+ * q8_quantize_static) and needs no workspace.  Larger M first writes the codes to the
+ * workspace (q8_quantize_static), then runs a tcgen05 int8 GEMM (int32 accumulators in
+ * tensor memory) with the zero-point term and both scales in its epilogue. */
 q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* second,
                          const int8_t* q, const int32_t* wsum, const float* s_w,
                          float* y, int64_t M, int64_t N, int64_t K,

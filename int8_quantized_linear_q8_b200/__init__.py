@@ -38,6 +38,7 @@ SYMBOLS = (
     "q8_linear_w8a8_noalloc", "q8_selftest_bounded_wait",
     "q8_quantize_weight_grid", "q8_linear_w8a16_bias", "q8_linear_w8a8_bias",
     "q8_observe_residual_minmax", "q8_hessian_accumulate", "q8_gptq_int8",
+    "q8_quantize_weight_nvfp4", "q8_linear_w4a16_nvfp4",
 )
 # Built-in scratch of q8_linear_w8a8_noalloc (bytes).
 Q8_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -93,6 +94,10 @@ def _lib() -> ctypes.CDLL:
                                          ctypes.POINTER(q8_qparams)]
     L.q8_quantize_weight_q4gs.restype = st
     L.q8_quantize_weight_q4gs.argtypes = [_vp, _i64, _i64, st, _vp, _vp, _vp, _vp]
+    L.q8_quantize_weight_nvfp4.restype = st
+    L.q8_quantize_weight_nvfp4.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp]
+    L.q8_linear_w4a16_nvfp4.restype = st
+    L.q8_linear_w4a16_nvfp4.argtypes = [_vp, _vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp]
     L.q8_linear_w8a16.restype = st
     L.q8_linear_w8a16.argtypes = [_vp, _vp, _vp, _vp, st, _i64, _i64, _i64, _vp]
     L.q8_linear_w8a16_bias.restype = st
@@ -273,7 +278,41 @@ def q8_quantize_weight_q4gs(W: torch.Tensor, G: int, q4=None, gs=None, stream=No
     return (q4, gs, c) if fold else (q4, gs)
 
 
+def q8_quantize_weight_nvfp4(W: torch.Tensor, q4=None, sf=None, gsc=None, stream=None):
+    """NVFP4 weight codes -> (q4 uint8 [N,K/2], sf uint8 [N,K/16] (E4M3 block scales),
+    gsc fp32 [1] on the device)."""
+    N, K = W.shape
+    _need(W, "W", torch.float32, (N, K))
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    q4 = _out(q4, "q4", torch.uint8, (N, K // 2), W.device)
+    sf = _out(sf, "sf", torch.uint8, (N, K // 16), W.device)
+    gsc = _out(gsc, "gsc", torch.float32, (1,), W.device)
+    _check(_lib().q8_quantize_weight_nvfp4(_ptr(W), N, K, _ptr(q4), _ptr(sf), _ptr(gsc),
+                                           _stream(stream)), "q8_quantize_weight_nvfp4")
+    return q4, sf, gsc
+
+
 # ---------------------------------------------------------------------------- linears
+
+
+def q8_linear_w4a16_nvfp4(x: torch.Tensor, q4: torch.Tensor, sf: torch.Tensor,
+                          gsc: torch.Tensor, y=None, out_dtype=torch.bfloat16,
+                          stream=None) -> torch.Tensor:
+    """bf16 activations x NVFP4 weights (codes, E4M3 block scales, device gsc [1])."""
+    M, K = x.shape
+    N = q4.shape[0]
+    _need(x, "x", torch.bfloat16, (M, K))
+    _need(q4, "q4", torch.uint8, (N, K // 2))
+    _need(sf, "sf", torch.uint8, (N, K // 16))
+    _need(gsc, "gsc", torch.float32, (1,))
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    y = _out(y, "y", out_dtype, (M, N), x.device)
+    yt = Q8_BF16 if y.dtype == torch.bfloat16 else Q8_F32
+    _check(_lib().q8_linear_w4a16_nvfp4(_ptr(x), _ptr(q4), _ptr(sf), _ptr(gsc), _ptr(y), yt,
+                                        M, N, K, _stream(stream)), "q8_linear_w4a16_nvfp4")
+    return y
 
 
 def q8_workspace_bytes(op: int, M: int, N: int, K: int, extra: int = 0) -> int:

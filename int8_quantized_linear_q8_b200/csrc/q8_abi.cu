@@ -130,12 +130,18 @@ constexpr int64_t kW8A8GemvMaxM = 16;
 constexpr int64_t kTcMinK = 128;
 constexpr int64_t kGptqMaxK = 16384;     // three K x K float64 work matrices (6 GB at the cap)
 
-// Workspace plans (byte offsets inside the caller's workspace).
+// Workspace plans (byte offsets inside the caller's workspace).  The W8A8 GEMV computes
+// its activation codes in registers and needs none; the tensor-core path keeps them in the
+// workspace between the quantizer and the GEMM.
+static inline bool w8a8_uses_gemv(int64_t M, int64_t K) {
+    return M <= kW8A8GemvMaxM || K < kTcMinK;
+}
 struct W8A8Plan {
     size_t xq1 = 0, xq2 = 0, bytes = 0;
 };
 static W8A8Plan plan_w8a8(int64_t M, int64_t K, int two) {
     W8A8Plan p;
+    if (w8a8_uses_gemv(M, K)) return p;
     const size_t codes = align_up((size_t)M * (size_t)K, 256);
     p.xq1 = 0;
     p.xq2 = two ? codes : 0;
@@ -363,6 +369,35 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) 
     return 0;
 }
 
+q8_status q8_quantize_weight_nvfp4(const float* W, int64_t N, int64_t K, uint8_t* q4, uint8_t* sf,
+                                   float* gsc, void* stream) {
+    if (!W || !q4 || !sf || !gsc) return Q8_ERR_NULL;
+    if (N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (K % 32) return Q8_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(q4) || !aligned16(sf) || !aligned4(gsc)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_quantize_weight_nvfp4(W, N, (int)K, q4, sf, gsc, (cudaStream_t)stream,
+                                                 sms));
+}
+
+q8_status q8_linear_w4a16_nvfp4(const void* x, const uint8_t* q4, const uint8_t* sf,
+                                const float* gsc, void* y, q8_dtype yt, int64_t M, int64_t N,
+                                int64_t K, void* stream) {
+    if (yt != Q8_F32 && yt != Q8_BF16) return Q8_ERR_ARG;
+    if (M < 0 || M > 0x7fffffff || N < 1 || N > 0x7fffffff) return Q8_ERR_SHAPE;
+    Q8_TRY(check_k(K));
+    if (K % 32) return Q8_ERR_SHAPE;
+    if (M == 0) return Q8_OK;
+    if (!x || !q4 || !sf || !gsc || !y) return Q8_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q4) || !aligned16(sf) || !aligned4(gsc)) return Q8_ERR_ALIGN;
+    int sms = 0;
+    Q8_TRY(current_device(sms));
+    return launched(launch_w4a16_nvfp4((const uint16_t*)x, q4, sf, gsc, y, yt == Q8_BF16, M, N,
+                                       (int)K, (cudaStream_t)stream));
+}
+
 q8_status q8_hessian_accumulate(const float* x, int64_t R, int64_t K, double* H, int reset,
                                 void* stream) {
     if (R < 0 || R > 0x7fffffff) return Q8_ERR_SHAPE;
@@ -416,17 +451,17 @@ q8_status q8_linear_w8a8_bias(const float* x, q8_qparams first, const q8_qparams
     int* status = nullptr;
     Q8_TRY(current_device(sms, &status));
     cudaStream_t st = (cudaStream_t)stream;
-    int8_t* xq1 = (int8_t*)workspace + plan.xq1;
-    int8_t* xq2 = two ? (int8_t*)workspace + plan.xq2 : nullptr;
     const float s2 = two ? second->scale : 1.0f;
     const int z2 = two ? second->zero_point : 0;
+    if (w8a8_uses_gemv(M, K))
+        return launched(launch_w8a8_gemv(x, first.scale, first.zero_point, two, s2, z2, q, wsum,
+                                         s_w, bias, y, M, N, (int)K, st));
+    int8_t* xq1 = (int8_t*)workspace + plan.xq1;
+    int8_t* xq2 = two ? (int8_t*)workspace + plan.xq2 : nullptr;
     Q8_TRY(launched(launch_quantize_static(x, M, (int)K, first.scale, first.zero_point, two, s2,
                                            z2, xq1, xq2, st, sms)));
-    if (M > kW8A8GemvMaxM && K >= kTcMinK)
-        return launched(launch_w8a8_tc(xq1, xq2, first.scale, first.zero_point, two, s2, z2, q,
-                                       wsum, s_w, bias, y, M, N, (int)K, st, sms, status));
-    return launched(launch_w8a8_gemv_codes(xq1, xq2, first.scale, first.zero_point, two, s2, z2,
-                                           q, wsum, s_w, bias, y, M, N, (int)K, st));
+    return launched(launch_w8a8_tc(xq1, xq2, first.scale, first.zero_point, two, s2, z2, q, wsum,
+                                   s_w, bias, y, M, N, (int)K, st, sms, status));
 }
 
 q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* gs, int G,
