@@ -266,11 +266,12 @@ q8_status q8_linear_w8a16_bias(const void* x, const int8_t* q, const float* s_w,
  *   workspace: device scratch of at least q8_workspace_bytes(Q8_OP_LINEAR_W8A8, M, N,
  *   K, second != NULL) bytes (may be NULL when that is 0); its contents on entry do not
  *   matter and are overwritten.
- * Decode-sized M (<= 16, or any M when K < 128) runs as one GEMV kernel on the warp-level
- * int8 MMA that computes the activation codes in registers (the steps of
- * q8_quantize_static) and needs no workspace.  Larger M first writes the codes to the
- * workspace (q8_quantize_static), then runs a tcgen05 int8 GEMM (int32 accumulators in
- * tensor memory) with the zero-point term and both scales in its epilogue. */
+ * Decode-sized M (<= 16, any M when K < 128, and small problems whose 16-row passes over the
+ * weight stay below 6 MB) runs as one GEMV kernel on the warp-level int8 MMA that computes
+ * the activation codes in registers (the steps of q8_quantize_static) and needs no
+ * workspace.  Larger problems first write the codes to the workspace (q8_quantize_static),
+ * then run a tcgen05 int8 GEMM (int32 accumulators in tensor memory) with the zero-point
+ * term and both scales in its epilogue. */
 q8_status q8_linear_w8a8(const float* x, q8_qparams first, const q8_qparams* second,
                          const int8_t* q, const int32_t* wsum, const float* s_w,
                          float* y, int64_t M, int64_t N, int64_t K,

@@ -123,25 +123,33 @@ q8_status check_current_device() {
     return current_device(sms);
 }
 
-// Activation rows up to which the W8A8 linear runs as a GEMV (weights streamed once per
-// 16 rows); above it the tensor-core GEMM takes over.  The tensor-core path loads K in
-// 128-byte steps and needs at least one whole step.
+// Activation rows up to which the W8A8 linear always runs as a GEMV (weights streamed once
+// per 16 rows); above it the tensor-core GEMM takes over, except for small problems: the
+// GEMM's fixed cost (quantizer pre-kernel, operand pipeline fill, one tile per CTA) is
+// ~8.5 us at K = 960, while the GEMV costs ~4 us plus ~0.55 us per MB of weight it
+// streams (measured on B200, K = 960 / 4096, N = 960..4096, M = 32..512), so the GEMV
+// keeps problems whose weight passes (ceil(M / 16) x N x K bytes, x 1.6 for two passes)
+// stay below 6 MB.  The tensor-core path loads K in 128-byte steps and needs at least one
+// whole step.
 constexpr int64_t kW8A8GemvMaxM = 16;
+constexpr int64_t kW8A8GemvSmallBytes = (int64_t)6 << 20;
 constexpr int64_t kTcMinK = 128;
 constexpr int64_t kGptqMaxK = 16384;     // three K x K float64 work matrices (6 GB at the cap)
 
 // Workspace plans (byte offsets inside the caller's workspace).  The W8A8 GEMV computes
 // its activation codes in registers and needs none; the tensor-core path keeps them in the
 // workspace between the quantizer and the GEMM.
-static inline bool w8a8_uses_gemv(int64_t M, int64_t K) {
-    return M <= kW8A8GemvMaxM || K < kTcMinK;
+static inline bool w8a8_uses_gemv(int64_t M, int64_t N, int64_t K, int two) {
+    if (M <= kW8A8GemvMaxM || K < kTcMinK) return true;
+    const double passes = (double)((M + 15) / 16) * (double)N * (double)K * (two ? 1.6 : 1.0);
+    return passes <= (double)kW8A8GemvSmallBytes;
 }
 struct W8A8Plan {
     size_t xq1 = 0, xq2 = 0, bytes = 0;
 };
-static W8A8Plan plan_w8a8(int64_t M, int64_t K, int two) {
+static W8A8Plan plan_w8a8(int64_t M, int64_t N, int64_t K, int two) {
     W8A8Plan p;
-    if (w8a8_uses_gemv(M, K)) return p;
+    if (w8a8_uses_gemv(M, N, K, two)) return p;
     const size_t codes = align_up((size_t)M * (size_t)K, 256);
     p.xq1 = 0;
     p.xq2 = two ? codes : 0;
@@ -355,7 +363,7 @@ q8_status q8_linear_w8a16_bias(const void* x, const int8_t* q, const float* s_w,
 size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) {
     if (M < 0 || N < 1 || check_k(K) != Q8_OK) return 0;
     switch (op) {
-        case Q8_OP_LINEAR_W8A8: return plan_w8a8(M, K, extra != 0).bytes;
+        case Q8_OP_LINEAR_W8A8: return plan_w8a8(M, N, K, extra != 0).bytes;
         case Q8_OP_GPTQ_INT8:
             if (K > kGptqMaxK || !gptq_block_ok(extra)) return 0;
             return plan_gptq(N, K).bytes;
@@ -444,7 +452,7 @@ q8_status q8_linear_w8a8_bias(const float* x, q8_qparams first, const q8_qparams
     Q8_TRY(w8a8_check_args(x, first, second, q, wsum, s_w, bias, y, M, N, K));
     if (M == 0) return Q8_OK;
     const int two = second != nullptr;
-    const W8A8Plan plan = plan_w8a8(M, K, two);
+    const W8A8Plan plan = plan_w8a8(M, N, K, two);
     if (plan.bytes > 0 && (!workspace || ws_bytes < plan.bytes)) return Q8_ERR_WORKSPACE;
     if (!aligned16(workspace)) return Q8_ERR_ALIGN;
     int sms = 0;
@@ -453,7 +461,7 @@ q8_status q8_linear_w8a8_bias(const float* x, q8_qparams first, const q8_qparams
     cudaStream_t st = (cudaStream_t)stream;
     const float s2 = two ? second->scale : 1.0f;
     const int z2 = two ? second->zero_point : 0;
-    if (w8a8_uses_gemv(M, K))
+    if (w8a8_uses_gemv(M, N, K, two))
         return launched(launch_w8a8_gemv(x, first.scale, first.zero_point, two, s2, z2, q, wsum,
                                          s_w, bias, y, M, N, (int)K, st));
     int8_t* xq1 = (int8_t*)workspace + plan.xq1;

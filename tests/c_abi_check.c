@@ -63,7 +63,7 @@ int main(void) {
     expect("linear_dq8ca_q4gsw",
            q8_linear_dq8ca_q4gsw(NULL, NULL, NULL, 48, NULL, 1, 16, 256, NULL, 0, NULL),
            Q8_ERR_ARG);
-    if (q8_workspace_bytes(Q8_OP_LINEAR_W8A8, 17, 16, 128, 0) < 17 * 128) ++fails;
+    if (q8_workspace_bytes(Q8_OP_LINEAR_W8A8, 17, 16384, 4096, 0) < 17 * 4096) ++fails;
     if (q8_workspace_bytes(Q8_OP_LINEAR_W8A8, 4, 16, 64, 0) != 0) ++fails;
     if (q8_workspace_bytes(Q8_OP_GPTQ_INT8, 0, 8, 64, 128) < 3 * 64 * 64 * 8) ++fails;
     expect("gemm_s8s8_s32", q8_gemm_s8s8_s32(NULL, NULL, NULL, 4, 0, 256, NULL), Q8_ERR_SHAPE);

@@ -63,8 +63,9 @@ def test_workspace_sizes(L):
     # up to 16 rows (or K < 128) the GEMV computes its codes in registers: no workspace
     assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 16, 16, 4096, 1) == 0
     assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 300, 16, 64, 1) == 0
-    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 17, 16, 128, 0) >= 17 * 128
-    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 17, 16, 128, 1) >= 2 * 17 * 128
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 17, 16, 128, 0) == 0       # small: GEMV
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 17, 16384, 4096, 0) >= 17 * 4096
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 17, 16384, 4096, 1) >= 2 * 17 * 4096
     assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 4, 16, 63) == 0      # invalid K
 
 
@@ -92,9 +93,9 @@ def test_argument_validation_before_device(L):
                             None) == q8.Q8_ERR_ARG
     assert L.q8_linear_w8a8(good, q8.q8_qparams(0.1, 200), None, good, good, good, good, 1, 16,
                             64, good, 1024, None) == q8.Q8_ERR_ARG
-    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 17, 16, 128, None, 0,
+    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 17, 16384, 4096, None, 0,
                             None) == q8.Q8_ERR_WORKSPACE
-    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 17, 16, 128, good, 10,
+    assert L.q8_linear_w8a8(good, qp, None, good, good, good, good, 17, 16384, 4096, good, 10,
                             None) == q8.Q8_ERR_WORKSPACE
     assert L.q8_quantize_weight_q4gs(good, 4, 64, 48, good, good, None, None) == q8.Q8_ERR_ARG
     assert L.q8_quantize_weight_q4gs(good, 4, 96, 64, good, good, None, None) == q8.Q8_ERR_SHAPE

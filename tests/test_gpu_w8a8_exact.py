@@ -109,9 +109,12 @@ def _run(x, q, s_w, wsum, first, second, rows):
     return units
 
 
-# M <= 16 runs the GEMV, M > 16 the tensor-core GEMM.  One pass: 256-row weight tiles where
-# they give at least two tiles per SM (4096 x 4096), 128-row tiles otherwise.
+# M <= 16 and small problems (under 6 MB of 16-row weight passes: 32 x 960 x 960,
+# 64 x 960 x 960, 40 x 300 x 512) run the GEMV, larger ones the tensor-core GEMM.  One pass:
+# 256-row weight tiles where they give at least two tiles per SM (4096 x 4096), 128-row
+# tiles otherwise.
 ONE_PASS = [(1, 2560, 960), (5, 960, 960), (16, 1000, 4096), (17, 300, 4096),
+            (32, 960, 960), (40, 300, 512),
             (256, 960, 960), (2048, 2560, 960), (300, 520, 4096), (4096, 4096, 4096)]
 
 
@@ -123,7 +126,7 @@ def test_w8a8_one_pass_exact_accumulators(M, N, K):
     _run(x, q, s_w, wsum, (S1, Z1), None, rows)
 
 
-TWO_PASS = [(1, 2560, 960), (5, 960, 960), (16, 1000, 4096), (256, 2560, 960),
+TWO_PASS = [(1, 2560, 960), (5, 960, 960), (16, 1000, 4096), (64, 960, 960), (256, 2560, 960),
             (2048, 960, 960), (300, 520, 4096), (2048, 4096, 4096)]
 
 
