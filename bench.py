@@ -9,10 +9,10 @@ bf16 activations + bf16 outputs) per second.  Two copies of every weight rotate 
 steps (390 MB, over 3x the 126 MB L2), and within a step cases run M-major, so a weight
 is never re-read from L2.
 
-Extra sub-benchmarks (same JSON line, key "paths"): the sweep through the digit-plane
-form and with a bias, W8A8 static int8 linear (K = 960) and prefill (M = 4096, also with a
-bias), 8da4w, the quantizers (both weight grids), a Llama-shaped stack and the offline
-GPTQ path (calibration Hessian + GPTQ of one 11008 x 4096 layer).
+Extra sub-benchmarks (same JSON line, key "paths"): the sweep with a bias, the NVFP4
+weight-only twin on the sweep's shapes, W8A8 static int8 linear (K = 960) and prefill
+(M = 4096, also with a bias), 8da4w, the quantizers (both weight grids), a Llama-shaped
+stack and the offline GPTQ path (calibration Hessian + GPTQ of one 11008 x 4096 layer).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -57,13 +57,14 @@ def parse_args():
     p.add_argument("--eager", action="store_true",
                    help="launch the timed steps one by one instead of replaying CUDA graphs "
                         "(for profilers that cannot replay graph-captured launches)")
-    p.add_argument("--profile", choices=["w8a16", "w8a8", "q4"], default=None,
+    p.add_argument("--profile", choices=["w8a16", "w8a8", "q4", "w4a16", "quant"], default=None,
                    help="run only one kernel case --reps times (for ncu captures), then exit")
     p.add_argument("--pM", type=int, default=16)
     p.add_argument("--pN", type=int, default=32000)
     p.add_argument("--pK", type=int, default=4096)
     p.add_argument("--pG", type=int, default=32, help="8da4w group size (--profile q4)")
     p.add_argument("--reps", type=int, default=3)
+    p.add_argument("--ptwo", type=int, default=1, help="W8A8 two-pass (1) or one pass (0)")
     return p.parse_args()
 
 
@@ -906,8 +907,26 @@ def run_profile(args):
     elif args.profile == "w8a8":
         x = torch.randn(M, K, generator=g, device=dev) * 4
         y = torch.empty(M, N, device=dev)
+        sec = (0.05 / 255, 0) if args.ptwo else None
         for _ in range(args.reps):
-            q8.q8_linear_w8a8(x, (0.05, 3), q, ws, s, second=(0.05 / 255, 0), y=y)
+            q8.q8_linear_w8a8(x, (0.05, 3), q, ws, s, second=sec, y=y)
+    elif args.profile == "w4a16":
+        W = torch.randn(N, K, generator=g, device=dev) * 0.02
+        q4, sf, gsc = q8.q8_quantize_weight_nvfp4(W)
+        del W
+        x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        for _ in range(args.reps):
+            q8.q8_linear_w4a16_nvfp4(x, q4, sf, gsc, y=y)
+    elif args.profile == "quant":
+        # the quantizers on an fp32 [N, K] weight and fp32 / bf16 [M, K] activations
+        W = torch.randn(N, K, generator=g, device=dev) * 0.02
+        xf = torch.randn(M, K, generator=g, device=dev) * 4
+        xb = xf.to(torch.bfloat16)
+        for _ in range(args.reps):
+            q8.q8_quantize_weight(W, q=q, s_w=s, wsum=ws)
+            q8.q8_choose_qparams(xb)
+            q8.q8_quantize_static(xf, (0.05, 3), second=(0.05 / 255, 0))
     else:
         W = torch.randn(N, K, generator=g, device=dev) * 0.02
         q4, gs = q8.q8_quantize_weight_q4gs(W, args.pG)
