@@ -84,21 +84,26 @@ __host__ __device__ constexpr uint32_t tc_idesc_i8(int M, int N) {
     return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
 }
-__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, uint32_t accumulate) {
+// Called by all 32 lanes of the issuing warp with the same operands (the issuing loop stays
+// warp-uniform); one lane, picked by elect.sync, issues the instruction.
+__device__ __forceinline__ void tc_mma_i8_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
     const uint32_t z = 0;
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z),
         "r"(z), "r"(z)
         : "memory");
 }
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+__device__ __forceinline__ void tc_commit_warp(uint64_t* bar) {
     asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+        ::"r"(smem_u32(bar))
         : "memory");
 }
 __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -205,20 +210,20 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // the whole warp runs the loop (warp-uniform); one elected lane issues each op
+        {
             constexpr uint32_t idesc = tc_idesc_i8(TC_BM, C::BN);
             int s = 0, acc = 0;
             uint32_t ph = 0, acc_ph = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                if (!mbar_wait(&tempty[acc], acc_ph ^ 1u, status, abort_flag)) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], acc_ph ^ 1u, status, abort_flag)))
+                    break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(acc * C::ACC_COLS);
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&full[s], ph, status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+                    ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, status, abort_flag));
+                    if (!ok) break;
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + (size_t)s * C::STAGE_BYTES);
                     const uint64_t a1 = tc_desc_sw128(st);
@@ -228,18 +233,18 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
                     for (int k = 0; k < TC_BK / TC_UK; ++k) {
                         // advance 32 bytes of K inside the swizzled rows: +2 in 16-byte units
                         const uint32_t accumulate = (kb | k) != 0;
-                        tc_mma_i8(d, a1 + 2 * k, b + 2 * k, idesc, accumulate);
-                        if (C::TWO) tc_mma_i8(d + C::BN, a2 + 2 * k, b + 2 * k, idesc, accumulate);
+                        tc_mma_i8_warp(d, a1 + 2 * k, b + 2 * k, idesc, accumulate);
+                        if (C::TWO) tc_mma_i8_warp(d + C::BN, a2 + 2 * k, b + 2 * k, idesc, accumulate);
                     }
-                    tc_commit(&empty[s]);               // stage free once these MMAs finish
+                    tc_commit_warp(&empty[s]);          // stage free once these MMAs finish
                     if (++s == TC_STAGES) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit(&tfull[acc]);                 // accumulator ready for the epilogue
+                tc_commit_warp(&tfull[acc]);            // accumulator ready for the epilogue
                 if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
             }
             // all MMAs issued here are complete before tensor memory is released
-            tc_commit(mma_done);
+            tc_commit_warp(mma_done);
             mbar_drain(mma_done, 0, status);
         }
         __syncwarp();

@@ -117,21 +117,29 @@ __device__ __forceinline__ uint64_t qt_desc_sw128(uint32_t saddr) {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
            ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
-__device__ __forceinline__ void qt_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                           uint32_t idesc, uint32_t accumulate) {
+// The MMA issuer is a whole warp: all 32 lanes run the issuing loop with the same values
+// (its waits, counters and descriptors stay warp-uniform) and call these two with the same
+// operands; one lane, picked by elect.sync, issues the instruction.  Run from a single lane
+// inside `if (lane == 0)`, the same loop was divergent code and cost ~180 cycles per MMA
+// (8 MMAs and their stage's waits took ~2100 cycles; halving the MMAs did not shorten it).
+__device__ __forceinline__ void qt_mma_f16_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
     const uint32_t z = 0;
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z),
         "r"(z), "r"(z)
         : "memory");
 }
-__device__ __forceinline__ void qt_commit(uint64_t* bar) {
+__device__ __forceinline__ void qt_commit_warp(uint64_t* bar) {
     asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+        ::"r"(smem_u32(bar))
         : "memory");
 }
 // Issue a 32-column tensor-memory load; the caller waits once for a batch of them.
@@ -258,22 +266,21 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // the whole warp runs the loop; one elected lane issues each tcgen05 op
+        {
             constexpr uint32_t idesc = qt_idesc_bf16(QT_BM, BN);
             int st = 0, buf = 0;
             uint32_t ph = 0, bph = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                // MMA step within the current group (a running counter: this thread issues
+                // MMA step within the current group (a running counter: this warp issues
                 // every MMA of the CTA, so its loop must stay short -- a modulo per step
                 // made the issue loop, not the tensor core, the limit)
                 int in_group = 0;
                 int gin = 0;                        // group within the current buffer
                 for (int kb = 0; kb < nk && ok; ++kb) {
-                    if (!mbar_wait(&full[st], ph, status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+                    ok = __all_sync(0xffffffffu, mbar_wait(&full[st], ph, status, abort_flag));
+                    if (!ok) break;
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                     const uint32_t base = smem_u32(smem + (size_t)st * C::STAGE);
 #pragma unroll
@@ -285,28 +292,27 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                             qt_desc_sw128(base + C::A_BYTES + (k / KPB) * C::B_BOX) + 2 * (k % KPB);
                         if (in_group == 0 && gin == 0) {
                             // a new buffer: wait until the epilogue has drained it
-                            if (!mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
+                            ok = __all_sync(0xffffffffu,
+                                            mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag));
+                            if (!ok) break;
                             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                         }
-                        qt_mma_f16(tmem_base + (uint32_t)(buf * C::BUFW + gin * BN), a, b, idesc,
-                                   in_group != 0);
+                        qt_mma_f16_warp(tmem_base + (uint32_t)(buf * C::BUFW + gin * BN), a, b,
+                                        idesc, in_group != 0);
                         if (++in_group == steps_per_group) {
                             in_group = 0;
                             if (++gin == GPB) {
                                 gin = 0;
-                                qt_commit(&tfull[buf]);         // GPB group partials ready
+                                qt_commit_warp(&tfull[buf]);    // GPB group partials ready
                                 if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
                             }
                         }
                     }
-                    qt_commit(&empty[st]);                      // stage free after these MMAs
+                    qt_commit_warp(&empty[st]);                 // stage free after these MMAs
                     if (++st == C::STAGES) { st = 0; ph ^= 1u; }
                 }
             }
-            qt_commit(mma_done);
+            qt_commit_warp(mma_done);
             mbar_drain(mma_done, 0, status);
         }
         __syncwarp();
@@ -575,7 +581,8 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // the whole warp runs the loop; one elected lane issues each tcgen05 op
+        {
             constexpr uint32_t idesc = qt_idesc_bf16(QT_BM, BN);
             int st = 0, buf = 0;
             uint32_t ph = 0, bph = 0;
@@ -585,10 +592,8 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
                 unit_range(u, t, kb0, kb1);
                 int in_group = 0;                  // MMA step within the current group
                 for (int kb = kb0; kb < kb1 && ok; ++kb) {
-                    if (!mbar_wait(&aready[st], ph, status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+                    ok = __all_sync(0xffffffffu, mbar_wait(&aready[st], ph, status, abort_flag));
+                    if (!ok) break;
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                     const uint32_t base = smem_u32(smem + (size_t)st * C::STAGE);
 #pragma unroll
@@ -598,24 +603,24 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
                         const uint64_t b = qt_desc_sw128(base + C::A_BYTES + (k / KPB) * C::B_BOX) +
                                            2 * (k % KPB);
                         if (in_group == 0) {
-                            if (!mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
+                            ok = __all_sync(0xffffffffu,
+                                            mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag));
+                            if (!ok) break;
                             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                         }
-                        qt_mma_f16(tmem_base + (uint32_t)(buf * BN), a, b, idesc, in_group != 0);
+                        qt_mma_f16_warp(tmem_base + (uint32_t)(buf * BN), a, b, idesc,
+                                        in_group != 0);
                         if (++in_group == steps_per_group) {
                             in_group = 0;
-                            qt_commit(&tfull[buf]);
+                            qt_commit_warp(&tfull[buf]);
                             if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
                         }
                     }
-                    qt_commit(&empty[st]);
+                    qt_commit_warp(&empty[st]);
                     if (++st == C::STAGES) { st = 0; ph ^= 1u; }
                 }
             }
-            qt_commit(mma_done);
+            qt_commit_warp(mma_done);
             mbar_drain(mma_done, 0, status);
         }
         __syncwarp();
