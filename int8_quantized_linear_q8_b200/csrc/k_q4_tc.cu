@@ -692,35 +692,13 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
 #pragma unroll
             for (int j = 0; j < HC; ++j) acc[j] = 0.0f;
             bool live = true;
-            // group scales in chunks of 16 groups, one chunk ahead (a group's MMAs are far
-            // shorter than an L2 round trip)
-            constexpr int GC = 16;
-            float gcur[GC], gnxt[GC];
-            auto load_chunk = [&](float (&dst)[GC], int g0) {
-#pragma unroll
-                for (int i = 0; i < GC; i += 4) {
-                    // 16-byte loads only where aligned (a K-part may start at any group)
-                    if ((ngroups & 3) == 0 && ((g0 + i) & 3) == 0 && g0 + i + 3 < ngroups) {
-                        const float4 v = __ldg(reinterpret_cast<const float4*>(gsr + g0 + i));
-                        dst[i] = v.x; dst[i + 1] = v.y; dst[i + 2] = v.z; dst[i + 3] = v.w;
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            dst[i + u] = (g0 + i + u < ngroups) ? __ldg(gsr + g0 + i + u) : 0.f;
-                    }
-                }
-            };
-            load_chunk(gnxt, g0);
+            // the next group's scale is loaded while this group is processed (a group takes
+            // longer here than an L2 round trip); kept in scalar registers -- 16-group
+            // chunks in arrays went to local memory in this kernel
+            float gnext = (g0 < g1) ? __ldg(gsr + g0) : 0.f;
             for (int gi = g0; gi < g1; ++gi) {
-                const int li = gi - g0;
-                if (li % GC == 0) {
-#pragma unroll
-                    for (int i = 0; i < GC; ++i) gcur[i] = gnxt[i];
-                    if (gi + GC < g1) load_chunk(gnxt, gi + GC);
-                }
-                float gcur_v = gcur[0];
-#pragma unroll
-                for (int i = 1; i < GC; ++i) gcur_v = (li % GC == i) ? gcur[i] : gcur_v;
+                const float gcur_v = gnext;
+                if (gi + 1 < g1) gnext = __ldg(gsr + gi + 1);
                 const bool okw = mbar_wait(&tfull[buf], bph, status, abort_flag);
                 live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
