@@ -182,25 +182,28 @@ __global__ __launch_bounds__(TC_THREADS, 1) void k_gemm_tc(
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            tma_prefetch_desc(&amap1);
-            if (C::TWO) tma_prefetch_desc(&amap2);
-            tma_prefetch_desc(&bmap);
+        // the whole warp runs the loop (warp-uniform); lane 0 issues the copies
+        {
+            if (lane == 0) {
+                tma_prefetch_desc(&amap1);
+                if (C::TWO) tma_prefetch_desc(&amap2);
+                tma_prefetch_desc(&bmap);
+            }
             int s = 0, it = 0;
             uint32_t ph = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 const int m0 = (t % num_m) * TC_BM, n0 = (t / num_m) * C::BN;
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&empty[s], ph ^ 1u, status, abort_flag)) {
-                        ok = false;
-                        break;
+                    ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, status, abort_flag));
+                    if (!ok) break;
+                    if (lane == 0) {
+                        uint8_t* st = smem + (size_t)s * C::STAGE_BYTES;
+                        mbar_expect_tx(&full[s], (uint32_t)C::STAGE_BYTES);
+                        tma_load_2d(st, &amap1, kb * TC_BK, m0, &full[s]);
+                        if (C::TWO) tma_load_2d(st + C::A_BYTES, &amap2, kb * TC_BK, m0, &full[s]);
+                        tma_load_2d(st + C::A_TILES * C::A_BYTES, &bmap, kb * TC_BK, n0, &full[s]);
                     }
-                    uint8_t* st = smem + (size_t)s * C::STAGE_BYTES;
-                    mbar_expect_tx(&full[s], (uint32_t)C::STAGE_BYTES);
-                    tma_load_2d(st, &amap1, kb * TC_BK, m0, &full[s]);
-                    if (C::TWO) tma_load_2d(st + C::A_BYTES, &amap2, kb * TC_BK, m0, &full[s]);
-                    tma_load_2d(st + C::A_TILES * C::A_BYTES, &bmap, kb * TC_BK, n0, &full[s]);
                     ++it;
                     if (++s == TC_STAGES) { s = 0; ph ^= 1u; }
                 }

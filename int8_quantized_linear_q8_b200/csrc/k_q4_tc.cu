@@ -230,9 +230,12 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
-        if (lane == 0) {
-            tma_prefetch_desc(&amap);
-            tma_prefetch_desc(&bmap);
+        // the whole warp runs the loop (warp-uniform); lane 0 issues the copies
+        {
+            if (lane == 0) {
+                tma_prefetch_desc(&amap);
+                tma_prefetch_desc(&bmap);
+            }
             // Activation tiles are re-read by every weight tile: keep them in L2; weight
             // tiles are re-read only by the next few activation tiles; outputs stream out.
             const uint64_t keep = make_l2_policy_evict_last();
@@ -243,19 +246,19 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 const int n0 = (t / num_m) * QT_BM, m0 = (t % num_m) * BN;
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&empty[st], ph ^ 1u, status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* base = smem + (size_t)st * C::STAGE;
-                    mbar_expect_tx(&full[st], (uint32_t)C::STAGE);
-                    // the tensor maps view the bf16 matrices as bytes: K offset in bytes
+                    ok = __all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u, status, abort_flag));
+                    if (!ok) break;
+                    if (lane == 0) {
+                        uint8_t* base = smem + (size_t)st * C::STAGE;
+                        mbar_expect_tx(&full[st], (uint32_t)C::STAGE);
+                        // the tensor maps view the bf16 matrices as bytes: K offset in bytes
 #pragma unroll
-                    for (int h = 0; h < C::KBOX; ++h) {
-                        const int kx = (kb * C::BK + h * QT_BOXK) * 2;
-                        tma_load_2d_hint(base + h * C::A_BOX, &amap, kx, n0, &full[st], drop);
-                        tma_load_2d_hint(base + C::A_BYTES + h * C::B_BOX, &bmap, kx, m0, &full[st],
-                                         keep);
+                        for (int h = 0; h < C::KBOX; ++h) {
+                            const int kx = (kb * C::BK + h * QT_BOXK) * 2;
+                            tma_load_2d_hint(base + h * C::A_BOX, &amap, kx, n0, &full[st], drop);
+                            tma_load_2d_hint(base + C::A_BYTES + h * C::B_BOX, &bmap, kx, m0,
+                                             &full[st], keep);
+                        }
                     }
                     ++it;
                     if (++st == C::STAGES) { st = 0; ph ^= 1u; }
@@ -547,9 +550,12 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
-        if (lane == 0) {
-            tma_prefetch_desc(&qmap);
-            tma_prefetch_desc(&bmap);
+        // the whole warp runs the loop (warp-uniform); lane 0 issues the copies
+        {
+            if (lane == 0) {
+                tma_prefetch_desc(&qmap);
+                tma_prefetch_desc(&bmap);
+            }
             const uint64_t keep = make_l2_policy_evict_last();   // activations: re-read
             const uint64_t drop = make_l2_policy_evict_first();  // weight codes
             int st = 0, it = 0;
@@ -560,18 +566,18 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
                 unit_range(u, t, kb0, kb1);
                 const int n0 = (t / num_m) * QT_BM, m0 = (t % num_m) * BN;
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!mbar_wait(&empty[st], ph ^ 1u, status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* base = smem + (size_t)st * C::STAGE;
-                    mbar_expect_tx(&full[st], (uint32_t)C::TX);
+                    ok = __all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u, status, abort_flag));
+                    if (!ok) break;
+                    if (lane == 0) {
+                        uint8_t* base = smem + (size_t)st * C::STAGE;
+                        mbar_expect_tx(&full[st], (uint32_t)C::TX);
 #pragma unroll
-                    for (int h = 0; h < C::KBOX; ++h)
-                        tma_load_2d_hint(base + C::A_BYTES + h * C::B_BOX, &bmap,
-                                         (kb * C::BK + h * QT_BOXK) * 2, m0, &full[st], keep);
-                    tma_load_2d_hint(base + C::A_BYTES + C::B_BYTES, &qmap, kb * C::BK / 2, n0,
-                                     &full[st], drop);
+                        for (int h = 0; h < C::KBOX; ++h)
+                            tma_load_2d_hint(base + C::A_BYTES + h * C::B_BOX, &bmap,
+                                             (kb * C::BK + h * QT_BOXK) * 2, m0, &full[st], keep);
+                        tma_load_2d_hint(base + C::A_BYTES + C::B_BYTES, &qmap, kb * C::BK / 2, n0,
+                                         &full[st], drop);
+                    }
                     ++it;
                     if (++st == C::STAGES) { st = 0; ph ^= 1u; }
                 }
