@@ -339,9 +339,13 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
             for (int j = 0; j < HC; ++j) acc[j] = 0.0f;
             bool live = true;
             // Group scales stream in chunks of 16 groups, one chunk ahead of their use: a
-            // group's MMAs take ~10^2 cycles, an L2 round trip several hundred.
-            constexpr int GC = HC > 64 ? 8 : 16;      // (register budget with 128 columns)
+            // group's MMAs take ~10^2 cycles, an L2 round trip several hundred.  With 128
+            // columns per warp (256-row tiles, G >= 64: a group's MMAs take >= 512 cycles)
+            // one scalar loaded a group ahead does, and leaves the registers to the sums.
+            constexpr bool G1 = HC > 64;
+            constexpr int GC = G1 ? 1 : 16;
             float gcur[GC], gnxt[GC];
+            float gnext1 = G1 ? __ldg(gsr) : 0.f;
             auto load_chunk = [&](float (&dst)[GC], int g0) {
 #pragma unroll
                 for (int i = 0; i < GC; i += 4) {
@@ -356,7 +360,7 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
                     }
                 }
             };
-            load_chunk(gnxt, 0);
+            if (!G1) load_chunk(gnxt, 0);
             for (int gb = 0; gb < ngroups; gb += GPB) {      // one hand-off per GPB groups
                 const bool okw = mbar_wait(&tfull[buf], bph, status, abort_flag);
                 live = live && (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0);
@@ -364,14 +368,20 @@ __global__ __launch_bounds__(QT_THREADS, 1) void k_q4_gemm_tc(
 #pragma unroll
               for (int sub = 0; sub < GPB; ++sub) {
                 const int gi = gb + sub;
-                if (gi % GC == 0) {
+                float gsel;
+                if (G1) {
+                    gsel = gnext1;
+                    if (gi + 1 < ngroups) gnext1 = __ldg(gsr + gi + 1);
+                } else {
+                    if (gi % GC == 0) {
 #pragma unroll
-                    for (int i = 0; i < GC; ++i) gcur[i] = gnxt[i];
-                    if (gi + GC < ngroups) load_chunk(gnxt, gi + GC);
+                        for (int i = 0; i < GC; ++i) gcur[i] = gnxt[i];
+                        if (gi + GC < ngroups) load_chunk(gnxt, gi + GC);
+                    }
+                    gsel = gcur[0];
+#pragma unroll
+                    for (int i = 1; i < GC; ++i) gsel = (gi % GC == i) ? gcur[i] : gsel;
                 }
-                float gsel = gcur[0];
-#pragma unroll
-                for (int i = 1; i < GC; ++i) gsel = (gi % GC == i) ? gcur[i] : gsel;
                 const float gcur_v = gsel;
                 if (live) {
                     const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
