@@ -8,7 +8,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libq8.so")
 SOURCES = ["q8_abi.cu", "k_quant.cu", "k_gemv.cu", "k_gemv_tma.cu", "k_gemm_tc.cu",
-           "q8_noalloc.cu", "k_w4a16.cu", "k_q4.cu", "k_q4_tc.cu", "k_q4_tma.cu",
+           "q8_noalloc.cu", "k_w4a16.cu", "k_q4.cu", "k_q4_tc.cu", "k_q4_i8.cu", "k_q4_tma.cu",
            "k_gptq.cu"]
 HEADERS = ["q8_common.cuh", "q8_kernels.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

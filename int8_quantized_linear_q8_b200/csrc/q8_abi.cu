@@ -158,29 +158,53 @@ static W8A8Plan plan_w8a8(int64_t M, int64_t N, int64_t K, int two) {
 }
 
 // Activation rows up to which the 8da4w linear runs as a GEMV on the packed int4 weights;
-// above it the weights are expanded once per call to bf16 integers and the tensor-core
-// GEMM runs (see k_q4_tc.cu).
+// above it a tensor-core GEMM runs: for 17..64 rows the bf16 one that expands the int4
+// codes in shared memory (k_q4_gemm_fused); above 64 rows either the int8 one
+// (k_q4_gemm_i8: the codes expanded to int8 in shared memory, zero-point term in the
+// epilogue) or the bf16 one on a per-call bf16 copy of the weight (k_q4_gemm_tc).
 constexpr int64_t kQ4GemvMaxM = 16;
 
+// Above 64 rows: whether the int8 GEMM runs.  Its epilogue spends ~2300 cycles per group
+// and tile (conversion and zero-point term per element), against the bf16 GEMM's one
+// multiply-add per element, so it pays only with few groups.  Measured at K = 4096,
+// N = 11008 (us, bf16 vs int8): G = 256 at every M (M = 80: 61 vs 38, 512: 112 vs 67,
+// 2048: 207 vs 200); G = 128 where it needs at most 2/3 of the bf16 GEMM's rounds of
+// tiles over the SMs, or a single row of 192-row tiles (M = 128: 63 vs 55, 512: 120 vs
+// 102; not at 256: 92 vs 100, or 1024: 181 vs 195); G <= 64 never (G = 64, M = 512: 139
+// vs 175).
+static bool q4_use_i8(int64_t M, int64_t N, int G, int sms) {
+    if (G >= 256) return true;
+    if (G < 128 || sms < 1) return false;
+    const int64_t nt = (N + 127) / 128;
+    const int64_t wide = (M >= 2048 && G >= 64) ? 256 : 128;   // the bf16 GEMM's tile rows
+    const int64_t r_bf16 = ((M + wide - 1) / wide * nt + sms - 1) / sms;
+    const int64_t r_i8 = ((M + 191) / 192 * nt + sms - 1) / sms;
+    return M <= 192 || 3 * r_i8 <= 2 * r_bf16;
+}
+
 struct Q4Plan {
-    bool tc = false;
+    bool tc = false, i8 = false;
     size_t xq = 0, s = 0, z = 0, wb = 0, bytes = 0;
 };
-// sms: the device's SM count (sizes the K-split workspace of the fused GEMM, 17..64 rows)
+// sms: the device's SM count (sizes the K-split workspace of the fused GEMM, 17..64 rows,
+// and picks the GEMM above 64 rows)
 static Q4Plan plan_q4(int64_t M, int64_t N, int64_t K, int G, int sms) {
     Q4Plan p;
     if (M <= 0) return p;
     p.tc = M > kQ4GemvMaxM;
-    // GEMV path: int8 codes [M, K]; tensor-core path: bf16 (xq - z) [M, K] + bf16 weights
-    const size_t codes = (size_t)M * (size_t)K * (p.tc ? 2 : 1);
+    p.i8 = p.tc && !q4_tc_fused(M) && q4_use_i8(M, N, G, sms);
+    // int8 codes [M, K]; for the bf16 GEMMs bf16 (xq - z) [M, K] instead
+    const size_t codes = (size_t)M * (size_t)K * (p.tc && !p.i8 ? 2 : 1);
     p.xq = 0;
     p.s = align_up(codes, 256);
     p.z = p.s + align_up((size_t)M * 4, 256);
     p.wb = p.z + align_up((size_t)M * 4, 256);
-    // the bf16 copy of the weight where the GEMM does not expand the codes itself; else
-    // (at wb) the fused GEMM's K-split partial sums and tile counters, if it splits
+    // at wb: the int8 GEMM's per-group code sums (fp32 [N, K/G]), or the bf16 copy of the
+    // weight, or (17..64 rows) the fused GEMM's K-split partial sums, if it splits
     size_t rest = 0;
-    if (p.tc && !q4_tc_fused(M))
+    if (p.i8)
+        rest = align_up((size_t)N * (size_t)(K / G) * 4, 256);
+    else if (p.tc && !q4_tc_fused(M))
         rest = align_up((size_t)N * (size_t)K * 2, 256);
     else if (p.tc)
         rest = align_up(q4_fused_workspace_bytes(M, N, (int)K, G, sms), 256);
@@ -370,7 +394,7 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) 
         case Q8_OP_LINEAR_DQ8CA_Q4GSW: {
             if (!valid_group(extra) || K % 128 != 0 || K % extra != 0) return 0;
             int sms = 0;
-            if (M > kQ4GemvMaxM && q4_tc_fused(M) && current_device(sms) != Q8_OK) return 0;
+            if (M > kQ4GemvMaxM && current_device(sms) != Q8_OK) return 0;
             return plan_q4(M, N, K, extra, sms).bytes;
         }
     }
@@ -499,6 +523,14 @@ q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* g
             Q8_TRY(launched(launch_choose_qparams_shifted((const uint16_t*)x, M, (int)K, s, z, xz, st)));
             return launched(launch_q4_gemm_fused(q4, xz, gs, s, y, G, M, N, (int)K, fws, st, sms,
                                                  status));
+        }
+        if (plan.i8) {
+            int8_t* xq8 = (int8_t*)(ws + plan.xq);
+            float* sums16 = (float*)(ws + plan.wb);
+            Q8_TRY(launched(launch_choose_qparams((const uint16_t*)x, M, (int)K, s, z, xq8, st)));
+            Q8_TRY(launched(launch_q4_group_sums16(q4, N, (int)K, G, sums16, st, sms)));
+            return launched(launch_q4_gemm_i8(xq8, z, s, q4, gs, sums16, y, G, M, N, (int)K, st,
+                                              sms, status));
         }
         uint16_t* wb = (uint16_t*)(ws + plan.wb);
         Q8_TRY(launched(launch_q4_expand_bf16(q4, N, (int)K, wb, st, sms)));

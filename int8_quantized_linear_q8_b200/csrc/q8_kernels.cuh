@@ -99,6 +99,13 @@ cudaError_t launch_q4_tma(const uint16_t* x, int8_t* xq, float* s, int32_t* z, b
                           const uint8_t* q4, const float* gs, int G, float* y, int64_t M,
                           int64_t N, int K, cudaStream_t st, int num_sms, int* status);
 
+// k_q4_i8.cu
+cudaError_t launch_q4_group_sums16(const uint8_t* q4, int64_t N, int K, int G, float* sums16,
+                                   cudaStream_t st, int num_sms);
+cudaError_t launch_q4_gemm_i8(const int8_t* xq, const int32_t* z, const float* s,
+                              const uint8_t* q4, const float* gs, const float* sums16, float* y,
+                              int G, int64_t M, int64_t N, int K, cudaStream_t st, int num_sms,
+                              int* status);
 // k_q4_tc.cu
 cudaError_t launch_q4_expand_bf16(const uint8_t* q4, int64_t N, int K, uint16_t* wb,
                                   cudaStream_t st, int num_sms);

@@ -429,8 +429,12 @@ def test_dq8ca_q4gsw_config(M, G):
                                      (8, 2000, 6144, 64), (12, 700, 4224, 32), (4, 11008, 4096, 256),
                                      # rows longer than the stream keeps in registers
                                      (1, 300, 12288, 64), (3, 500, 10240, 128),
-                                     # 256-row activation tiles: ragged last tile, odd N
-                                     (2100, 300, 512, 64), (2048, 129, 256, 256),
+                                     # above 64 rows, ragged last tiles and odd N: the bf16
+                                     # GEMM (G <= 64; 256-row tiles from 2048 rows) and the
+                                     # int8 one (G = 256; G = 128 with few tiles)
+                                     (2100, 300, 512, 64), (600, 18500, 256, 64),
+                                     (2048, 129, 256, 256), (300, 19000, 512, 256),
+                                     (150, 5000, 1024, 128),
                                      # 17..64 rows: the GEMM expands the int4 codes itself
                                      (33, 1000, 2176, 64), (64, 300, 4096, 256),
                                      (20, 129, 128, 32), (50, 257, 1024, 128)])
@@ -468,12 +472,13 @@ def test_dq8ca_decode_workspace_codes(M, K, G):
 
 
 @pytest.mark.parametrize("M,K", [(300, 256), (5, 256), (16, 4096), (1, 12288), (3, 2304),
-                                 (40, 512)])
+                                 (40, 512), (65, 768), (1000, 1024)])
 def test_dq8ca_group_partials_exact(M, K):
     """Unit group scales: y / s must be the exact integer sum_k (xq - z) q4 (one fp32
-    rounding of s * T).  Above 16 rows this is the bf16 tensor-core path (17..64 rows with the
-    int4 -> bf16 expansion inside the GEMM); up to 16 rows the decode stream, whose in-kernel
-    activation codes and zero points must then be the oracle's bit for bit."""
+    rounding of s * T).  Above 64 rows this is the int8 tensor-core GEMM (its zero-point term
+    and int32 -> fp32 steps must be exact), 17..64 rows the bf16 one with the int4 -> bf16
+    expansion inside; up to 16 rows the decode stream, whose in-kernel activation codes and
+    zero points must then be the oracle's bit for bit."""
     N, G = 200, 256
     g = torch.Generator().manual_seed(4242)
     x = wl.normal_bf16((M, K), 1.0, seed=4243 + M)
