@@ -300,7 +300,7 @@ q8_status q8_linear_w8a8_bias(const float* x, q8_qparams first, const q8_qparams
  *   it receives the activation codes, scales and zero points.  Above 64 rows the
  *   contraction runs either as a tcgen05 int8 GEMM (codes expanded to int8 in shared
  *   memory, the zero-point term z[m] * sum_{k in g} q4[n,k] and both scales applied in the
- *   epilogue; used for G = 256, and for G = 128 where its tiles fall better on the SMs) or
+ *   epilogue; used for G = 256, and for G = 128 below 2048 rows) or
  *   as a bf16 GEMM on exact small integers; both give the same fp32 results. */
 q8_status q8_linear_dq8ca_q4gsw(const void* x, const uint8_t* q4, const float* gs, int G,
                                 float* y, int64_t M, int64_t N, int64_t K,
@@ -342,9 +342,8 @@ q8_status q8_gptq_int8(const float* W, const double* H, int64_t N, int64_t K, do
 
 /* Host.  Workspace bytes a linear needs for these sizes (0 if none).  `extra` is
  * "two-pass" (0/1) for Q8_OP_LINEAR_W8A8, G for Q8_OP_LINEAR_DQ8CA_Q4GSW and the block
- * size for Q8_OP_GPTQ_INT8.  The 8da4w size above 16 rows also depends on the current
- * device's SM count (it sizes the K split of the 17..64-row GEMM and picks the GEMM above
- * 64 rows).
+ * size for Q8_OP_GPTQ_INT8.  The 8da4w size for 17..64 rows also depends on the current
+ * device's SM count (it sizes the K split of the 17..64-row GEMM).
  * Returns 0 for invalid arguments as well; the linear then reports the error. */
 size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra);
 

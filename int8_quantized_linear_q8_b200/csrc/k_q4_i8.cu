@@ -100,8 +100,7 @@ __device__ __forceinline__ void qi_commit_warp(uint64_t* bar) {
         ::"r"(smem_u32(bar))
         : "memory");
 }
-// 16 or 32 consecutive accumulator columns of this warp's lane quarter; waited for
-// separately.
+// 16 consecutive accumulator columns of this warp's lane quarter; waited for separately.
 __device__ __forceinline__ void qi_ld_nowait(uint32_t taddr, uint32_t (&u)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -111,18 +110,13 @@ __device__ __forceinline__ void qi_ld_nowait(uint32_t taddr, uint32_t (&u)[16]) 
           "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
         : "r"(taddr));
 }
-__device__ __forceinline__ void qi_ld_nowait(uint32_t taddr, uint32_t (&u)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
-          "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
-          "=r"(u[13]), "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]),
-          "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]),
-          "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]),
-          "=r"(u[31])
-        : "r"(taddr));
+// Completes this thread's outstanding tcgen05.ld; the registers are tied to the wait so
+// that no use of them is scheduled before it.
+__device__ __forceinline__ void qi_wait_ld(uint32_t (&u)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(u[0]), "+r"(u[1]), "+r"(u[2]), "+r"(u[3]), "+r"(u[4]), "+r"(u[5]),
+                   "+r"(u[6]), "+r"(u[7]), "+r"(u[8]), "+r"(u[9]), "+r"(u[10]), "+r"(u[11]),
+                   "+r"(u[12]), "+r"(u[13]), "+r"(u[14]), "+r"(u[15])::"memory");
 }
 // (a.x, a.y) = (a.x + b.x * c.x, a.y + b.y * c.y), one packed fp32 instruction, each lane
 // rounded once like fmaf.
@@ -397,14 +391,17 @@ __global__ __launch_bounds__(QI_THREADS, 1) void k_q4_gemm_i8(
                 if (live) {
                     const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
                                            (uint32_t)(buf * BN + half * HC);
-                    // chunks of CW columns (16 with more than 64 columns per warp: registers
-                    // are short)
-                    constexpr int CW = HC > 64 ? 16 : 32;
+                    // 16-column chunks, double-buffered: the load of chunk c + 1 is in flight
+                    // while chunk c is processed, so a group exposes one tensor-memory
+                    // latency (two-chunk waits cost the kernel ~2300 cycles per group)
+                    constexpr int CW = 16, NC = HC / CW;
+                    uint32_t u[2][CW];
+                    qi_ld_nowait(taddr, u[0]);
+                    qi_wait_ld(u[0]);
 #pragma unroll
-                    for (int c0 = 0; c0 < HC / CW; ++c0) {
-                        uint32_t u[CW];
-                        qi_ld_nowait(taddr + c0 * CW, u);
-                        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    for (int c0 = 0; c0 < NC; ++c0) {
+                        if (c0 + 1 < NC) qi_ld_nowait(taddr + (c0 + 1) * CW, u[(c0 + 1) & 1]);
+                        const uint32_t(&uc)[CW] = u[c0 & 1];
 #pragma unroll
                         for (int j = 0; j < CW; j += 4) {
                             const float4 zz = *reinterpret_cast<const float4*>(zt + c0 * CW + j);
@@ -413,16 +410,17 @@ __global__ __launch_bounds__(QI_THREADS, 1) void k_q4_gemm_i8(
                                   c1y = kQiMagicF;
                             qi_fma2(c0x, c0y, zz.x, zz.y, qsum, qsum);
                             qi_fma2(c1x, c1y, zz.z, zz.w, qsum, qsum);
-                            float f0 = __int_as_float((int)u[j] + kQiMagicI);
-                            float f1 = __int_as_float((int)u[j + 1] + kQiMagicI);
-                            float f2 = __int_as_float((int)u[j + 2] + kQiMagicI);
-                            float f3 = __int_as_float((int)u[j + 3] + kQiMagicI);
+                            float f0 = __int_as_float((int)uc[j] + kQiMagicI);
+                            float f1 = __int_as_float((int)uc[j + 1] + kQiMagicI);
+                            float f2 = __int_as_float((int)uc[j + 2] + kQiMagicI);
+                            float f3 = __int_as_float((int)uc[j + 3] + kQiMagicI);
                             qi_sub2(f0, f1, c0x, c0y);          // 16 * T_g, exact
                             qi_sub2(f2, f3, c1x, c1y);
                             const int a = c0 * CW + j;
                             qi_fma2(acc[a], acc[a + 1], gs16, gs16, f0, f1);
                             qi_fma2(acc[a + 2], acc[a + 3], gs16, gs16, f2, f3);
                         }
+                        if (c0 + 1 < NC) qi_wait_ld(u[(c0 + 1) & 1]);
                     }
                 }
                 asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");

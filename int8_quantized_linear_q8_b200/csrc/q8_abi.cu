@@ -164,35 +164,27 @@ static W8A8Plan plan_w8a8(int64_t M, int64_t N, int64_t K, int two) {
 // epilogue) or the bf16 one on a per-call bf16 copy of the weight (k_q4_gemm_tc).
 constexpr int64_t kQ4GemvMaxM = 16;
 
-// Above 64 rows: whether the int8 GEMM runs.  Its epilogue spends ~2300 cycles per group
-// and tile (conversion and zero-point term per element), against the bf16 GEMM's one
-// multiply-add per element, so it pays only with few groups.  Measured at K = 4096,
-// N = 11008 (us, bf16 vs int8): G = 256 at every M (M = 80: 61 vs 38, 512: 112 vs 67,
-// 2048: 207 vs 200); G = 128 where it needs at most 2/3 of the bf16 GEMM's rounds of
-// tiles over the SMs, or a single row of 192-row tiles (M = 128: 63 vs 55, 512: 120 vs
-// 102; not at 256: 92 vs 100, or 1024: 181 vs 195); G <= 64 never (G = 64, M = 512: 139
-// vs 175).
-static bool q4_use_i8(int64_t M, int64_t N, int G, int sms) {
-    if (G >= 256) return true;
-    if (G < 128 || sms < 1) return false;
-    const int64_t nt = (N + 127) / 128;
-    const int64_t wide = (M >= 2048 && G >= 64) ? 256 : 128;   // the bf16 GEMM's tile rows
-    const int64_t r_bf16 = ((M + wide - 1) / wide * nt + sms - 1) / sms;
-    const int64_t r_i8 = ((M + 191) / 192 * nt + sms - 1) / sms;
-    return M <= 192 || 3 * r_i8 <= 2 * r_bf16;
-}
+// Above 64 rows: whether the int8 GEMM runs.  Its epilogue converts each group partial
+// and applies the zero-point term per element, against the bf16 GEMM's one multiply-add,
+// so it pays only with few groups; from 2048 rows the bf16 GEMM uses 256-row activation
+// tiles (twice the work per MMA).  Measured at K = 4096, N = 11008, us, bf16 / int8, at
+// M = 128, 512, 1024, 2048, 4096:
+//   G = 256: 62 / 37, 113 / 65, 169 / 116, 208 / 193, 371 / 344
+//   G = 128: 64 / 49, 121 / 90, 182 / 171, 235 / 293, 422 / 534
+//   G =  64: 68 / 77, 139 / 144, 210 / 279, 396 / 481, 748 / 883
+//   G =  32: 76 / 132, 164 / 254, 251 / 497, 466 / 864, 852 / 1589
+static bool q4_use_i8(int64_t M, int G) { return G >= 256 || (G == 128 && M < 2048); }
 
 struct Q4Plan {
     bool tc = false, i8 = false;
     size_t xq = 0, s = 0, z = 0, wb = 0, bytes = 0;
 };
-// sms: the device's SM count (sizes the K-split workspace of the fused GEMM, 17..64 rows,
-// and picks the GEMM above 64 rows)
+// sms: the device's SM count (sizes the K-split workspace of the fused GEMM, 17..64 rows)
 static Q4Plan plan_q4(int64_t M, int64_t N, int64_t K, int G, int sms) {
     Q4Plan p;
     if (M <= 0) return p;
     p.tc = M > kQ4GemvMaxM;
-    p.i8 = p.tc && !q4_tc_fused(M) && q4_use_i8(M, N, G, sms);
+    p.i8 = p.tc && !q4_tc_fused(M) && q4_use_i8(M, G);
     // int8 codes [M, K]; for the bf16 GEMMs bf16 (xq - z) [M, K] instead
     const size_t codes = (size_t)M * (size_t)K * (p.tc && !p.i8 ? 2 : 1);
     p.xq = 0;
@@ -394,7 +386,7 @@ size_t q8_workspace_bytes(q8_op op, int64_t M, int64_t N, int64_t K, int extra) 
         case Q8_OP_LINEAR_DQ8CA_Q4GSW: {
             if (!valid_group(extra) || K % 128 != 0 || K % extra != 0) return 0;
             int sms = 0;
-            if (M > kQ4GemvMaxM && current_device(sms) != Q8_OK) return 0;
+            if (M > kQ4GemvMaxM && q4_tc_fused(M) && current_device(sms) != Q8_OK) return 0;
             return plan_q4(M, N, K, extra, sms).bytes;
         }
     }

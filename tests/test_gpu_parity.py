@@ -431,7 +431,7 @@ def test_dq8ca_q4gsw_config(M, G):
                                      (1, 300, 12288, 64), (3, 500, 10240, 128),
                                      # above 64 rows, ragged last tiles and odd N: the bf16
                                      # GEMM (G <= 64; 256-row tiles from 2048 rows) and the
-                                     # int8 one (G = 256; G = 128 with few tiles)
+                                     # int8 one (G = 256; G = 128 below 2048 rows)
                                      (2100, 300, 512, 64), (600, 18500, 256, 64),
                                      (2048, 129, 256, 256), (300, 19000, 512, 256),
                                      (150, 5000, 1024, 128),
