@@ -536,7 +536,8 @@ def bias_case_times(sweep: W8A16Sweep):
 
 def bench_q4(dev, peaks, reps=5):
     """8da4w: x bf16 [M, 4096] (M in 1, 64, 512, 4096), int4 weights [11008, 4096] with
-    fp32 group scales (G in 32, 128); incl. the per-row qparams pre-kernel."""
+    fp32 group scales (G in 32, 128; and G = 256 at M = 512, 4096, where the int8 GEMM runs
+    at every M); incl. the per-row qparams pre-kernel."""
     import int8_quantized_linear_q8_b200 as q8
 
     out = []
@@ -544,9 +545,10 @@ def bench_q4(dev, peaks, reps=5):
     g = torch.Generator(device=dev)
     g.manual_seed(wl.Q4_SEED_W)
     W = torch.randn(N, K, generator=g, device=dev) * 0.02
-    for G in wl.Q4_G:
+    cases = [(G, wl.Q4_M) for G in wl.Q4_G] + [(256, (512, 4096))]
+    for G, Ms in cases:
         q4, gs = q8.q8_quantize_weight_q4gs(W, G)
-        for M in wl.Q4_M:
+        for M in Ms:
             g.manual_seed(wl.Q4_SEED_X + M)
             x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
             y = torch.empty(M, N, device=dev)
