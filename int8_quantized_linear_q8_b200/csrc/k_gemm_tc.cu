@@ -31,9 +31,9 @@
 
 namespace q8 {
 
-// EPI_W8A8_N128: the one-pass epilogue on 128-row weight tiles (for grids that 256-row
-// tiles would leave unbalanced)
-enum { EPI_S32 = 0, EPI_W8A8 = 1, EPI_TWO = 2, EPI_W8A8_N128 = 3 };
+// EPI_W8A8_N128 / _N160: the one-pass epilogue on 128- or 160-row weight tiles (for grids
+// that 256-row tiles would leave unbalanced)
+enum { EPI_S32 = 0, EPI_W8A8 = 1, EPI_TWO = 2, EPI_W8A8_N128 = 3, EPI_W8A8_N160 = 4 };
 
 constexpr int TC_BM = 128;          // accumulator rows (= tensor-memory lanes)
 constexpr int TC_BK = 128;          // bytes of K per stage (one 128-byte swizzle row)
@@ -45,13 +45,15 @@ constexpr int TC_TMEM_COLS = 512;
 template <int EPI>
 struct TcCfg {
     static constexpr bool TWO = EPI == EPI_TWO;
-    static constexpr int BN = TWO || EPI == EPI_W8A8_N128 ? 128 : 256;   // weight rows per tile
+    static constexpr int BN =                                  // weight rows per tile
+        TWO || EPI == EPI_W8A8_N128 ? 128 : EPI == EPI_W8A8_N160 ? 160 : 256;
     static constexpr int A_TILES = TWO ? 2 : 1;
     static constexpr int A_BYTES = TC_BM * TC_BK;              // 16 KB
     static constexpr int B_BYTES = BN * TC_BK;
     static constexpr int STAGE_BYTES = A_TILES * A_BYTES + B_BYTES;   // 48 KB
     static constexpr int ACC_COLS = TWO ? 2 * BN : BN;         // per accumulator buffer
     static_assert(2 * ACC_COLS <= TC_TMEM_COLS, "tensor memory");
+    static_assert(B_BYTES % 1024 == 0 && BN % 32 == 0 && BN <= 256, "tile shape");
     // + control (8 KB) + the epilogue's store-transpose tiles (4 warps x 32 x 36 floats)
     static constexpr size_t SMEM = (size_t)TC_STAGES * STAGE_BYTES + 8192 + 4 * 32 * 36 * 4;
 };
@@ -421,11 +423,19 @@ cudaError_t launch_w8a8_tc(const int8_t* xq1, const int8_t* xq2, float s1, int z
     (bias ? launch_tc<EPI_, true>(xq1, A2_, q, (int)M, (int)N, K, ep, st, num_sms, status)  \
           : launch_tc<EPI_, false>(xq1, A2_, q, (int)M, (int)N, K, ep, st, num_sms, status))
     if (has2) return TC_W8A8(EPI_TWO, xq2);
-    // 256-row weight tiles unless they would give fewer than two tiles per SM: then the
-    // last round of tiles leaves most SMs idle, and 128-row tiles halve that round
-    const int64_t tiles256 = ((M + TC_BM - 1) / TC_BM) * ((N + 255) / 256);
-    if (tiles256 < 2 * (int64_t)num_sms) return TC_W8A8(EPI_W8A8_N128, nullptr);
-    return TC_W8A8(EPI_W8A8, nullptr);
+    // Weight-tile rows: 256, 160 or 128, whichever gives the fewest rounds of tiles over
+    // the SMs weighted by a tile's cost (taken as its rows plus a fixed part worth 128 rows:
+    // pipeline fill and tail).  M = 2048, N = 2560: 160 rows, 2 rounds of 256 tiles instead
+    // of 3 rounds of 320 128-row ones; the Llama prefill shapes keep 256 rows.
+    const int64_t mt = (M + TC_BM - 1) / TC_BM;
+    auto cost = [&](int64_t bn) {
+        const int64_t tiles = mt * ((N + bn - 1) / bn);
+        return (tiles + num_sms - 1) / num_sms * (bn + 128);
+    };
+    const int64_t c256 = cost(256), c160 = cost(160), c128 = cost(128);
+    if (c256 <= c160 && c256 <= c128) return TC_W8A8(EPI_W8A8, nullptr);
+    if (c160 <= c128) return TC_W8A8(EPI_W8A8_N160, nullptr);
+    return TC_W8A8(EPI_W8A8_N128, nullptr);
 #undef TC_W8A8
 }
 
