@@ -69,6 +69,24 @@ def test_workspace_sizes(L):
     assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_W8A8, 4, 16, 63) == 0      # invalid K
 
 
+def _up(n):
+    return -(-n // 256) * 256
+
+
+@pytest.mark.parametrize("M,G,i8", [(65, 256, True), (4096, 256, True), (512, 128, True),
+                                    (2047, 128, True), (2048, 128, False), (512, 64, False),
+                                    (4096, 32, False)])
+def test_dq8ca_workspace_layout_above_64_rows(L, M, G, i8):
+    """Above 64 rows the 8da4w linear runs the int8 GEMM for G = 256 and for G = 128 below
+    2048 rows (int8 codes [M, K], s, z, then the fp32 group code sums [N, K/G]), else the
+    bf16 GEMM (bf16 codes [M, K], s, z, then the bf16 weight copy [N, K]); each part on a
+    256-byte boundary.  No device is needed to size it."""
+    N, K = 11008, 4096
+    head = _up(M * K * (1 if i8 else 2)) + 2 * _up(4 * M)
+    tail = _up(N * (K // G) * 4) if i8 else _up(N * K * 2)
+    assert q8.q8_workspace_bytes(q8.Q8_OP_LINEAR_DQ8CA_Q4GSW, M, N, K, G) == head + tail
+
+
 def _p(v):
     return ctypes.c_void_p(v)
 
