@@ -612,24 +612,55 @@ __global__ __launch_bounds__(QF_THREADS, 1) void k_q4_gemm_fused(
                     if (!ok) break;
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                     const uint32_t base = smem_u32(smem + (size_t)st * C::STAGE);
-#pragma unroll
-                    for (int k = 0; k < C::BK / QT_UK; ++k) {
-                        constexpr int KPB = QT_BOXK / QT_UK;
-                        const uint64_t a = qt_desc_sw128(base + (k / KPB) * C::A_BOX) + 2 * (k % KPB);
-                        const uint64_t b = qt_desc_sw128(base + C::A_BYTES + (k / KPB) * C::B_BOX) +
-                                           2 * (k % KPB);
+                    constexpr int MPS = C::BK / QT_UK;           // MMA steps per stage
+                    constexpr int KPB = QT_BOXK / QT_UK;
+                    if (KB > 1 && steps_per_group % MPS == 0) {
+                        // groups are whole stages: one buffer check and at most one hand-off
+                        // per stage, none between the MMAs (single-box stages only serve
+                        // G = 32: never)
                         if (in_group == 0) {
                             ok = __all_sync(0xffffffffu,
                                             mbar_wait(&tempty[buf], bph ^ 1u, status, abort_flag));
                             if (!ok) break;
                             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                         }
-                        qt_mma_f16_warp(tmem_base + (uint32_t)(buf * BN), a, b, idesc,
-                                        in_group != 0);
-                        if (++in_group == steps_per_group) {
+                        const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+#pragma unroll
+                        for (int k = 0; k < MPS; ++k) {
+                            const uint64_t a =
+                                qt_desc_sw128(base + (k / KPB) * C::A_BOX) + 2 * (k % KPB);
+                            const uint64_t b =
+                                qt_desc_sw128(base + C::A_BYTES + (k / KPB) * C::B_BOX) +
+                                2 * (k % KPB);
+                            qt_mma_f16_warp(d, a, b, idesc, (in_group | k) != 0);
+                        }
+                        in_group += MPS;
+                        if (in_group == steps_per_group) {
                             in_group = 0;
                             qt_commit_warp(&tfull[buf]);
                             if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < MPS; ++k) {
+                            const uint64_t a =
+                                qt_desc_sw128(base + (k / KPB) * C::A_BOX) + 2 * (k % KPB);
+                            const uint64_t b =
+                                qt_desc_sw128(base + C::A_BYTES + (k / KPB) * C::B_BOX) +
+                                2 * (k % KPB);
+                            if (in_group == 0) {
+                                ok = __all_sync(0xffffffffu, mbar_wait(&tempty[buf], bph ^ 1u,
+                                                                       status, abort_flag));
+                                if (!ok) break;
+                                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                            }
+                            qt_mma_f16_warp(tmem_base + (uint32_t)(buf * BN), a, b, idesc,
+                                            in_group != 0);
+                            if (++in_group == steps_per_group) {
+                                in_group = 0;
+                                qt_commit_warp(&tfull[buf]);
+                                if (++buf == C::NBUF) { buf = 0; bph ^= 1u; }
+                            }
                         }
                     }
                     qt_commit_warp(&empty[st]);
