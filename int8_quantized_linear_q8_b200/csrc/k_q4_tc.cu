@@ -3,12 +3,13 @@
 //   y[m, n] = s[m] * sum_g gs[n, g] * T_g[m, n],   T_g = sum_{k in g} (xq[m,k] - z[m]) q4[n,k]
 //
 // The group scale gs[n, g] multiplies every group partial, so the integer sums must leave
-// the tensor core once per group.  Doing that from an int8 MMA would cost three ALU
-// operations per output element per group (zero-point term, conversion, scale); here the
-// operands enter a bf16 MMA as exact small integers instead -- the codes q4 in [-8, 7] and
-// the shifted activation codes (xq - z) in [-255, 255] -- so every product is exact and
-// each group partial is an integer below 2^24 (|T_g| <= 256 * 255 * 8), exact in the fp32
-// accumulator.  The epilogue then needs one fp32 multiply-add per element and group.
+// the tensor core once per group.  From an int8 MMA that costs several ALU operations per
+// output element and group (conversion, zero-point term, scale; k_q4_i8.cu does it, and is
+// used where it measured faster: few groups per row); here the operands enter a bf16 MMA
+// as exact small integers instead -- the codes q4 in [-8, 7] and the shifted activation
+// codes (xq - z) in [-255, 255] -- so every product is exact and each group partial is an
+// integer below 2^24 (|T_g| <= 256 * 255 * 8), exact in the fp32 accumulator.  The
+// epilogue then needs one fp32 multiply-add per element and group.
 //
 // Operands (prepared by the two kernels below, into the caller's workspace):
 //   A = weights  bf16 [N, K]  (each int4 code as a bf16 integer)
@@ -22,9 +23,10 @@
 // 3 stages of two boxes for G >= 64, so that one barrier round covers 8 MMAs -- a wait
 // between MMAs leaves the tensor pipe idle for a few hundred cycles -- or 6 stages of one
 // box for G = 32, where a group hand-off comes every 2 MMAs anyway);
-// warp 1 tensor-memory allocator and MMA issuer (kind::f16, M = 128, N = BN, K = 16) --
-// one group's MMAs go into one of NBUF accumulator buffers, tcgen05.commit hands it to
-// the epilogue; warps 2-9 epilogue (two per tensor-memory lane quarter): tcgen05.ld of the
+// warp 1 tensor-memory allocator and MMA issuer (kind::f16, M = 128, N = BN, K = 16; the
+// whole warp runs the issuing loop, one elected lane issues) -- one group's MMAs go into
+// one of NBUF accumulator buffers, tcgen05.commit hands it to the epilogue; warps 2-9
+// epilogue (two per tensor-memory lane quarter): tcgen05.ld of the
 // group partials, fp32 multiply-add with the group scale into per-thread registers, at
 // the end of a tile y = s[m] * acc.
 #include "q8_kernels.cuh"
