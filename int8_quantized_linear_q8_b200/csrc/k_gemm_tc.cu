@@ -13,8 +13,10 @@
 // Structure: persistent CTAs (one per SM), 6 warps.
 //   warp 0   : TMA producer -- per 128-byte K step, the activation tile(s) (128 rows) and
 //              the weight tile (BN rows) land in a 4-stage shared-memory ring, 128-byte
-//              swizzled, signalled by an mbarrier with transaction bytes.
-//   warp 1   : allocates all 512 tensor-memory columns, then one lane issues
+//              swizzled, signalled by an mbarrier with transaction bytes (the whole warp
+//              runs the loop, lane 0 issues the copies).
+//   warp 1   : allocates all 512 tensor-memory columns, then runs the issuing loop as a
+//              whole warp, one elected lane issuing each
 //              tcgen05.mma.kind::i8 (M=128, K=32) into an int32 accumulator in tensor
 //              memory; tcgen05.commit releases each smem stage and, after the last K
 //              step, hands the accumulator to the epilogue.  Accumulators are double-
@@ -23,10 +25,10 @@
 //              32-lane quarter of tensor memory), zero-point term and scales in fp32;
 //              each warp's 32 x 32 output chunk goes through a padded shared-memory tile
 //              so that every store instruction covers 4 rows x 128 bytes.
-// Weight tiles are 256 rows (BN), or 128 where 256-row tiles would give fewer than two
-// tiles per SM, and 128 for the two-pass form (two accumulators per tile).
+// Weight tiles are 256, 160 or 128 rows (BN) for one pass, chosen on the host by rounds of
+// tiles over the SMs, and 128 for the two-pass form (two accumulators per tile).
 // Every wait is bounded (abort flag + status word), and tensor memory is released only
-// after the issuing thread has seen all of its MMAs complete.
+// after the issuing warp has seen all of its MMAs complete.
 #include "q8_kernels.cuh"
 
 namespace q8 {
