@@ -354,7 +354,7 @@ __global__ __launch_bounds__(QI_THREADS, 1) void k_q4_gemm_i8(
         // ---------------------------------------------------------------- epilogue
         // warp w (4..15): lane quarter w % 4 of the weight rows, column third (w - 4) / 4
         const int q = warp & 3;
-        const int half = (warp - 4) >> 2;                 // this warp's column block
+        const int blk = (warp - 4) >> 2;                  // this warp's column block
         const int et = threadIdx.x - 128;                 // 0 .. 32 * QI_EPI_WARPS - 1
         constexpr int HC = C::HC;
         int buf = 0;
@@ -371,7 +371,7 @@ __global__ __launch_bounds__(QI_THREADS, 1) void k_q4_gemm_i8(
             const int64_t rowg = (int64_t)(n < N ? n : 0) * ngroups;
             const float* gsr = gs + rowg;
             const float* qsr = sums16 + rowg;
-            const float* zt = z_tile + half * HC;
+            const float* zt = z_tile + blk * HC;
             float acc[HC];
 #pragma unroll
             for (int j = 0; j < HC; ++j) acc[j] = 0.0f;
@@ -390,7 +390,7 @@ __global__ __launch_bounds__(QI_THREADS, 1) void k_q4_gemm_i8(
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 if (live) {
                     const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
-                                           (uint32_t)(buf * BN + half * HC);
+                                           (uint32_t)(buf * BN + blk * HC);
                     // 16-column chunks, double-buffered: the load of chunk c + 1 is in flight
                     // while chunk c is processed, so a group exposes one tensor-memory
                     // latency (two-chunk waits cost the kernel ~2300 cycles per group)
@@ -431,8 +431,8 @@ __global__ __launch_bounds__(QI_THREADS, 1) void k_q4_gemm_i8(
             if (live && n < N) {
 #pragma unroll
                 for (int j = 0; j < HC; ++j) {
-                    const int m = m0 + half * HC + j;
-                    if (m < M) st_stream_f32(y + (int64_t)m * N + n, s_tile[half * HC + j] * acc[j]);
+                    const int m = m0 + blk * HC + j;
+                    if (m < M) st_stream_f32(y + (int64_t)m * N + n, s_tile[blk * HC + j] * acc[j]);
                 }
             }
             named_bar_sync(2, 32 * QI_EPI_WARPS);         // before s_tile is rewritten
